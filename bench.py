@@ -1,0 +1,347 @@
+"""Benchmark of the compressed-KV hot path: tq_quantize (prefill of the whole context) followed by
+tq_decode_attn (one decode query per sequence) on one Llama-3-8B-shaped layer (32 query heads,
+8 kv-heads, head_dim 128, context 32768, turbo3 keys = 3-bit + QJL m=128, 3-bit values).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line.  value = compressed-KV bytes read by decode / decode time (GB/s, whole job);
+quantize throughput is reported beside it.  Multi-GPU (torchrun): every rank runs its own
+independent replica of the workload (the path has no exchange step), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+import workloads as W
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+DEFAULT_WORKLOAD = "llama3_8b_32k"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------------------- CPU arm
+
+def oracle_sample(w: W.Workload, tokens: int):
+    """Oracle quantize + decode for one (batch, kv-head) unit over `tokens` tokens (CPU)."""
+    from oracle import tq_oracle as O
+    sw = w.scaled(T=tokens, B=1, Hkv=1, Hq=w.group)
+    K = W.make_kv(sw, "k").double().numpy()
+    V = W.make_kv(sw, "v").double().numpy()
+    q = W.make_queries(sw).double().numpy()
+    Pi, S = W.rotation_for(w), W.qjl_for(w)
+    t0 = time.perf_counter()
+    cache = O.quantize_cache(K, V, Pi, w.k_bits, w.v_bits, S)
+    t1 = time.perf_counter()
+    O.decode_attention(q, Pi, S, cache, w.k_bits, w.v_bits, tokens)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, sw
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 20.0):
+    tokens = 2048
+    qt, dt, sw = oracle_sample(w, tokens)
+    # grow the sample toward the time budget
+    while qt + dt < budget_s / 4 and tokens < w.T:
+        tokens = min(w.T, tokens * 2)
+        qt, dt, sw = oracle_sample(w, tokens)
+    dec_bytes = sw.decode_bytes()
+    cores = os.cpu_count()
+    return {
+        "value": dec_bytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+        "sample": f"one (batch, kv-head) unit of {w.name}: {tokens} tokens, {w.group} query heads; "
+                  f"numpy float64 (BLAS threads up to {cores})",
+        "quantize_tokens_per_s": tokens / qt, "decode_s": dt, "quantize_s": qt,
+    }
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    cb = cpu_baseline(w, budget_s=20.0)
+    steps = []
+    tokens = int(cb["sample"].split(": ")[1].split(" ")[0])
+    for _ in range(args.warmup + args.steps):
+        steps.append(oracle_sample(w, tokens))
+    timed = steps[args.warmup:]
+    dt = sum(s[1] for s in timed)
+    qt = sum(s[0] for s in timed)
+    dec_bytes = timed[0][2].decode_bytes() * len(timed)
+    value = dec_bytes / dt / 1e9
+    line = {
+        "impl": "reference", "metric": "compressed-KV decode-attn GB/s (% HBM peak); tq_quantize tokens/s",
+        "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * (dt + qt) / len(timed),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, sample_tokens=tokens),
+        "quantize_tokens_per_s": tokens * len(timed) / qt,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w: W.Workload, **extra):
+    c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.head_dim,
+         "context": w.T, "k_bits": w.k_bits, "v_bits": w.v_bits, "qjl_m": w.qjl_m,
+         "input_dtype": w.in_dtype, "quantize_chunk": w.chunk,
+         "l2": f"flushed before every kernel call ({L2_FLUSH_BYTES >> 20} MiB write)"}
+    c.update(extra)
+    return c
+
+
+# --------------------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, w):
+    import decode_attention_11_b200 as tq
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    params = tq.Params.create(W.rotation_for(w), W.qjl_for(w), w.k_bits, w.v_bits, device=dev)
+    K = W.make_kv(w, "k", device=dev)
+    V = W.make_kv(w, "v", device=dev)
+    q = W.make_queries(w, device=dev)
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m, device=dev)
+    out = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.decode_workspace_size(w.B, w.Hq, cache, w.T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n_chunks = math.ceil(w.T / w.chunk)
+
+    def quantize_all():
+        for s in range(0, w.T, w.chunk):
+            tq.quantize(params, K[:, :, s:s + w.chunk], V[:, :, s:s + w.chunk], cache, t_offset=s)
+
+    def step(ev):
+        flush.zero_()
+        ev[0].record(stream)
+        quantize_all()
+        ev[1].record(stream)
+        flush.zero_()
+        ev[2].record(stream)
+        tq.decode_attn(params, q, cache, w.T, out=out, workspace=ws)
+        ev[3].record(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_all0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_all1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t_all0.elapsed_time(t_all1)
+    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    d_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(total_ms, world)
+    q_tot = max_over_ranks(sum(q_ms), world)
+    d_tot = max_over_ranks(sum(d_ms), world)
+
+    dec_bytes = w.decode_bytes()
+    qnt_bytes = w.quantize_bytes()
+    hbm, tflops, peak_kind = load_peaks()
+    dec_gbs = world * dec_bytes * args.steps / (d_tot * 1e-3) / 1e9
+    q_tok_s = world * w.B * w.T * args.steps / (q_tot * 1e-3)
+    q_gbs = world * qnt_bytes * args.steps / (q_tot * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if rank == 0 or world > 1:
+        Kh = K.cpu().pin_memory()
+        Vh = V.cpu().pin_memory()
+        qh = q.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            K.copy_(Kh, non_blocking=True)
+            V.copy_(Vh, non_blocking=True)
+            q.copy_(qh, non_blocking=True)
+            quantize_all()
+            tq.decode_attn(params, q, cache, w.T, out=out, workspace=ws)
+            oh.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        e_steps = max(3, args.steps // 2)
+        a0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a0.elapsed_time(a1), world)
+        h2d = Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size() + qh.numel() * qh.element_size()
+        d2h = oh.numel() * oh.element_size()
+        e2e = {"value": world * dec_bytes * e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / e_steps}
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    dec_frac = (dec_bytes / (sum(d_ms) / len(d_ms) * 1e-3) / 1e9) / hbm
+    q_frac = (qnt_bytes / (sum(q_ms) / len(q_ms) * 1e-3) / 1e9) / hbm
+    dominant = "tq_quantize" if sum(q_ms) >= sum(d_ms) else "tq_decode_attn"
+
+    def roof(name, bytes_per_launch, ms):
+        achieved = bytes_per_launch / (ms * 1e-3) / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind}
+
+    per_launch_q = qnt_bytes / n_chunks
+    roof_q = roof("tq_quantize", per_launch_q, (sum(q_ms) / len(q_ms)) / n_chunks)
+    roof_d = roof("tq_decode_attn", dec_bytes, sum(d_ms) / len(d_ms))
+    cb = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
+    line = {
+        "metric": "compressed-KV decode-attn GB/s (% HBM peak); tq_quantize tokens/s",
+        "value": dec_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 mma / f32 accumulate (decode); f32+f64 (quantize)",
+        "data": "synthetic", "config": workload_config(w, parallelism=f"replicas x{world}"),
+        "decode_hbm_frac": dec_frac, "decode_ms": sum(d_ms) / len(d_ms),
+        "quantize_tokens_per_s": q_tok_s, "quantize_GBps": q_gbs, "quantize_hbm_frac": q_frac,
+        "quantize_ms": sum(q_ms) / len(q_ms),
+        "roofline": roof_q if dominant == "tq_quantize" else roof_d,
+        "roofline_decode": roof_d, "roofline_quantize": roof_q,
+        "cpu_baseline": cb, "e2e": e2e,
+        "gpu_launches": args.steps * (n_chunks + 3),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.CONFIG_ORDER)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = W.CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

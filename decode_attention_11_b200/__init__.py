@@ -1,0 +1,262 @@
+"""B200-native TurboQuant-style compressed-KV hot path: Python binding of the tq C ABI.
+
+Argument marshalling only: every step of the path runs in ``libtq_b200.so`` (CUDA kernels for
+sm_100a plus the host codebook builder).  PyTorch provides device memory and streams.  There is
+no fallback: if the shared library is missing or fails to load, every call raises.
+
+    import decode_attention_11_b200 as tq
+    params = tq.Params.create(Pi, S, k_bits=4, v_bits=4, device="cuda")
+    cache = tq.Cache.allocate(B, Hkv, T_cap, k_bits=4, v_bits=4, qjl_m=128, device="cuda")
+    tq.quantize(params, k, v, cache, t_offset=0)            # k, v: [B, Hkv, T_new, 128]
+    out = tq.decode_attn(params, q, cache, seq_len)          # q: [B, Hq, 128]
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
+
+TQ_OK = 0
+TQ_ERR_INVALID_ARG = 1
+TQ_ERR_UNSUPPORTED = 2
+TQ_ERR_NO_CONVERGENCE = 3
+TQ_ERR_WORKSPACE = 4
+TQ_ERR_CUDA = 5
+TQ_F32 = 0
+TQ_BF16 = 1
+
+# Functions declared in include/tq.h (checked by the test-suite against the header).
+EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codebook",
+            "tq_quantize", "tq_decode_workspace_size", "tq_decode_attn")
+
+
+class TqError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{status_string(status)}: {detail}")
+        self.status = status
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("T_cap", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("k_bits", ctypes.c_int), ("v_bits", ctypes.c_int),
+                ("qjl_m", ctypes.c_int),
+                ("k_codes", ctypes.c_void_p), ("k_signs", ctypes.c_void_p),
+                ("k_norm", ctypes.c_void_p), ("k_rnorm", ctypes.c_void_p),
+                ("v_codes", ctypes.c_void_p), ("v_norm", ctypes.c_void_p)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("Pi", ctypes.c_void_p), ("S", ctypes.c_void_p),
+                ("k_centroids", ctypes.c_void_p), ("k_thresholds", ctypes.c_void_p),
+                ("v_centroids", ctypes.c_void_p), ("v_thresholds", ctypes.c_void_p)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtq_b200.so (raises if it is missing: there is no other implementation)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} not built; run `python -m decode_attention_11_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.tq_status_string.restype = ctypes.c_char_p
+    L.tq_status_string.argtypes = [ctypes.c_int]
+    L.tq_last_error.restype = ctypes.c_char_p
+    L.tq_last_error.argtypes = []
+    L.tq_version.restype = ctypes.c_int
+    L.tq_build_codebook.restype = ctypes.c_int
+    L.tq_build_codebook.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                    ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float),
+                                    ctypes.POINTER(ctypes.c_double)]
+    L.tq_quantize.restype = ctypes.c_int
+    L.tq_quantize.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_void_p,
+                              ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                              ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache), ctypes.c_void_p]
+    L.tq_decode_workspace_size.restype = ctypes.c_size_t
+    L.tq_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache),
+                                           ctypes.c_int]
+    L.tq_decode_attn.restype = ctypes.c_int
+    L.tq_decode_attn.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int,
+                                 ctypes.c_int, ctypes.POINTER(_Cache), ctypes.c_int, ctypes.c_float,
+                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().tq_status_string(int(status)).decode()
+
+
+def last_error() -> str:
+    return lib().tq_last_error().decode()
+
+
+def _check(status: int) -> None:
+    if status != TQ_OK:
+        raise TqError(status, last_error())
+
+
+def version() -> int:
+    return int(lib().tq_version())
+
+
+def build_codebook(bits: int, max_iter: int = 100000, tol: float = 1e-13
+                   ) -> Tuple[np.ndarray, np.ndarray, float]:
+    """Lloyd-Max quantizer of N(0,1): (centroids float32[2^b], thresholds float32[2^b-1], distortion)."""
+    L = 1 << bits if 1 <= bits <= 8 else 1
+    c = np.zeros(max(L, 1), dtype=np.float32)
+    t = np.zeros(max(L - 1, 1), dtype=np.float32)
+    dist = ctypes.c_double(0.0)
+    _check(lib().tq_build_codebook(int(bits), int(max_iter), float(tol),
+                                   c.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                   t.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                   ctypes.byref(dist)))
+    return c[:L], t[:L - 1], float(dist.value)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if stream.cuda_stream else None
+
+
+@dataclasses.dataclass
+class Params:
+    """Per-layer constants on the device (fp32): rotation, sketch, codebooks."""
+
+    Pi: torch.Tensor
+    S: Optional[torch.Tensor]
+    k_centroids: torch.Tensor
+    k_thresholds: torch.Tensor
+    v_centroids: torch.Tensor
+    v_thresholds: torch.Tensor
+
+    @classmethod
+    def create(cls, Pi, S, k_bits: int, v_bits: int, device="cuda") -> "Params":
+        kc, kt, _ = build_codebook(k_bits)
+        vc, vt, _ = build_codebook(v_bits)
+        f = lambda x: torch.as_tensor(np.ascontiguousarray(x, dtype=np.float32)).to(device)
+        return cls(f(Pi), None if S is None else f(S), f(kc), f(kt), f(vc), f(vt))
+
+    def as_c(self) -> _Params:
+        return _Params(_ptr(self.Pi), _ptr(self.S), _ptr(self.k_centroids),
+                       _ptr(self.k_thresholds), _ptr(self.v_centroids), _ptr(self.v_thresholds))
+
+
+@dataclasses.dataclass
+class Cache:
+    """Packed cache arrays (caller-owned torch tensors; layout in include/tq.h)."""
+
+    B: int
+    Hkv: int
+    T_cap: int
+    k_bits: int
+    v_bits: int
+    qjl_m: int
+    k_codes: torch.Tensor
+    k_signs: Optional[torch.Tensor]
+    k_norm: torch.Tensor
+    k_rnorm: Optional[torch.Tensor]
+    v_codes: torch.Tensor
+    v_norm: torch.Tensor
+
+    @classmethod
+    def allocate(cls, B, Hkv, T_cap, k_bits, v_bits, qjl_m=128, device="cuda") -> "Cache":
+        u8 = dict(dtype=torch.uint8, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        return cls(B, Hkv, T_cap, k_bits, v_bits, qjl_m,
+                   torch.zeros(B, Hkv, T_cap, 16 * k_bits, **u8),
+                   torch.zeros(B, Hkv, T_cap, 16, **u8) if qjl_m else None,
+                   torch.zeros(B, Hkv, T_cap, **f32),
+                   torch.zeros(B, Hkv, T_cap, **f32) if qjl_m else None,
+                   torch.zeros(B, Hkv, T_cap, 16 * v_bits, **u8),
+                   torch.zeros(B, Hkv, T_cap, **f32))
+
+    @classmethod
+    def from_arrays(cls, arrays: dict, k_bits, v_bits, qjl_m, device="cuda") -> "Cache":
+        """Wrap host arrays (k_codes, k_signs, k_norm, k_rnorm, v_codes, v_norm) as a device cache."""
+        g = lambda n: None if arrays.get(n) is None else torch.as_tensor(
+            np.ascontiguousarray(arrays[n])).to(device)
+        kc = g("k_codes")
+        B, Hkv, T_cap = kc.shape[:3]
+        return cls(B, Hkv, T_cap, k_bits, v_bits, qjl_m, kc, g("k_signs") if qjl_m else None,
+                   g("k_norm"), g("k_rnorm") if qjl_m else None, g("v_codes"), g("v_norm"))
+
+    def as_c(self) -> _Cache:
+        return _Cache(self.B, self.Hkv, self.T_cap, 128, self.k_bits, self.v_bits, self.qjl_m,
+                      _ptr(self.k_codes), _ptr(self.k_signs), _ptr(self.k_norm),
+                      _ptr(self.k_rnorm), _ptr(self.v_codes), _ptr(self.v_norm))
+
+    def row_bytes(self) -> int:
+        return 16 * self.k_bits + (20 if self.qjl_m else 0) + 4 + 16 * self.v_bits + 4
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TQ_F32
+    if t.dtype == torch.bfloat16:
+        return TQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def quantize(params: Params, k: torch.Tensor, v: torch.Tensor, cache: Cache, t_offset: int = 0,
+             stream=None) -> None:
+    """Compress k, v ([B, Hkv, T_new, 128], same strides, last dim contiguous) into cache rows
+    [t_offset, t_offset + T_new)."""
+    if k.shape != v.shape or k.stride() != v.stride() or k.dtype != v.dtype:
+        raise ValueError("k and v must share shape, strides and dtype")
+    if k.dim() != 4 or k.shape[-1] != 128 or k.stride(-1) != 1:
+        raise ValueError("k must be [B, Hkv, T_new, 128] with a contiguous last dim")
+    c = cache.as_c()
+    p = params.as_c()
+    _check(lib().tq_quantize(ctypes.byref(p), k.data_ptr(), v.data_ptr(), _dtype_code(k),
+                             k.stride(0), k.stride(1), k.stride(2), k.shape[2], int(t_offset),
+                             ctypes.byref(c), _stream_ptr(stream)))
+
+
+def decode_workspace_size(B: int, Hq: int, cache: Cache, seq_len: int) -> int:
+    c = cache.as_c()
+    return int(lib().tq_decode_workspace_size(int(B), int(Hq), ctypes.byref(c), int(seq_len)))
+
+
+def decode_attn(params: Params, q: torch.Tensor, cache: Cache, seq_len: int,
+                out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                scale: float = 0.0, stream=None) -> torch.Tensor:
+    """Decode attention of q [B, Hq, 128] over the first seq_len cached tokens -> fp32 [B, Hq, 128]."""
+    if q.dim() != 3 or q.shape[-1] != 128 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous [B, Hq, 128] tensor")
+    B, Hq, _ = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, 128, dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, Hq, cache, seq_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    c = cache.as_c()
+    p = params.as_c()
+    _check(lib().tq_decode_attn(ctypes.byref(p), q.data_ptr(), _dtype_code(q), int(Hq),
+                                ctypes.byref(c), int(seq_len), float(scale), out.data_ptr(),
+                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                _stream_ptr(stream)))
+    return out
+
+
+__all__ = [
+    "LIB_PATH", "EXPORTED", "TqError", "lib", "status_string", "last_error", "version",
+    "build_codebook", "Params", "Cache", "quantize", "decode_workspace_size", "decode_attn",
+    "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
+    "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16",
+]

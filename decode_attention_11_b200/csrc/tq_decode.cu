@@ -1,0 +1,688 @@
+// tq_decode_attn: single-token decode attention directly over the packed cache.
+//
+// Scores follow the QJL-corrected estimator of the method statement,
+//   est_i = <q', khat'_i> + ||r_i|| sqrt(pi/2)/m <S q', 2 sign_i - 1>,  q' = Pi q,
+// with khat'_i = (n_i / sqrt(d)) c_K[idx_i] in the rotated basis (ai-news.ru overview, first and
+// second ideas plus the third, QJL, component; tproger.ru "Step 1: PolarQuant", "Step 2: QJL").
+// Softmax and the value sum also run in the rotated basis; one final o = Pi^T o' per head.
+//
+// Kernels (all on the caller's stream):
+//   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace.
+//   split   grid (splits, Hkv * head_groups, B).  A 4-warp CTA streams its token range through a
+//           4-stage cp.async pipeline (64 tokens per stage).  Each warp takes 16 tokens per stage:
+//           codes are turned into fp16 pairs by a lane-replicated shared-memory table (one load per
+//           two coordinates, no bank conflicts), and m16n8k16 tensor-core MMAs compute q'.khat
+//           (q' split into fp16 hi + lo rows), the QJL sign dot (signs -> +-0.5 by one half2 FMA)
+//           and P.vhat (P split into hi + lo rows).  Online softmax runs in log2 units.
+//           The CTA merges its 4 warps and writes one (max, sum, o'[128]) partial per head.
+//   reduce  log-sum-exp merge of the split partials, then o = Pi^T o'.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int WARPS = 4;
+constexpr int THREADS = 32 * WARPS;
+constexpr int STAGE_TOK = 16 * WARPS;  // 64 tokens per pipeline stage
+constexpr int NSTAGE = 4;
+constexpr int HG = 8;                  // query heads per MMA row block (hi rows 0-7, lo rows 8-15)
+constexpr int PART = 2 + D;            // (max, sum, o'[128]) per partial
+constexpr unsigned FULL = 0xffffffffu;
+
+struct DArgs {
+  int B, Hq, Hkv, g, hgroups, T_cap, seq_len, splits, tps;
+  float sK;   // scale*log2e/sqrt(d)                     (times n_i)
+  float sQ;   // scale*log2e*2*sqrt(pi/2)/m              (times ||r_i||; 2 undoes the +-0.5 signs)
+  const uint8_t* k_codes;
+  const uint8_t* k_signs;
+  const float* k_norm;
+  const float* k_rnorm;
+  const uint8_t* v_codes;
+  const float* v_norm;
+  const float* kc;
+  const float* vc;
+  const float* qrot;
+  const float* sq;
+  float* part;
+};
+
+// ------------------------------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// 16-byte async copy; src_bytes < 16 zero-fills the rest (src_bytes = 0: no global read).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __halves2half2(__float2half_rn(lo), __float2half_rn(hi));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Split x into fp16 hi + lo with x ~= hi + lo (about 22 significant bits).
+__device__ __forceinline__ void split_half(float x, float& hi, float& lo) {
+  hi = __half2float(__float2half_rn(x));
+  lo = x - hi;
+}
+
+// Sign bits -> +-0.5 fp16 pair: bits q and q+16 of w (1 <= q <= 10) placed in the mantissa of 1.0,
+// then one exact half2 FMA maps 1 + b*2^(q-10) to b - 0.5.
+template <int Q>
+__device__ __forceinline__ uint32_t sign_half2(uint32_t w) {
+  static_assert(Q >= 1 && Q <= 10, "mantissa position");
+  const uint32_t x = (w & (0x00010001u << Q)) | 0x3C003C00u;
+  const __half2 hx = *reinterpret_cast<const __half2*>(&x);
+  const float m = (float)(1 << (10 - Q));
+  const __half2 r = __hfma2(hx, __float2half2_rn(m), __float2half2_rn(-(m + 0.5f)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+// Pair p of a thread's 32-bit sign word (bits p and p+16).
+template <int P>
+__device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
+  if constexpr (P == 0) return sign_half2<1>(w << 1);
+  else if constexpr (P <= 10) return sign_half2<P>(w);
+  else return sign_half2<P - 10>(w >> 10);
+}
+
+// Pair p (0..15) of a thread's key-code chunk: 2*KB bits starting at bit 2*KB*p.
+template <int KB, int P>
+__device__ __forceinline__ uint32_t k_pair_index(const uint32_t (&c)[KB]) {
+  constexpr int off = 2 * KB * P;
+  constexpr int w = off / 32, sh = off % 32;
+  constexpr uint32_t mask = (1u << (2 * KB)) - 1u;
+  if constexpr (sh + 2 * KB <= 32) {
+    return (c[w] >> sh) & mask;
+  } else {
+    return __funnelshift_r(c[w], c[w + 1], sh) & mask;
+  }
+}
+
+// Value code nu (0..15) of a thread's 16-code value chunk held in a 64-bit integer.
+template <int VB, int NU>
+__device__ __forceinline__ uint32_t v_code(uint64_t c) {
+  return (uint32_t)(c >> (VB * NU)) & ((1u << VB) - 1u);
+}
+
+// ------------------------------------------------------------------------------------------ prep
+
+template <typename QT>
+__global__ void __launch_bounds__(D) prep_kernel(const QT* __restrict__ q, const float* __restrict__ Pi,
+                                                const float* __restrict__ S, int BH, int qjl,
+                                                float* __restrict__ qrot, float* __restrict__ sq) {
+  __shared__ float qs[HG][D];
+  __shared__ float qr[HG][D];
+  const int i = threadIdx.x;
+  const int h0 = blockIdx.x * HG;
+  const int nh = min(HG, BH - h0);
+  for (int r = 0; r < HG; ++r) {
+    float x = 0.0f;
+    if (r < nh) {
+      if constexpr (sizeof(QT) == 4) x = (float)q[(int64_t)(h0 + r) * D + i];
+      else x = __bfloat162float(q[(int64_t)(h0 + r) * D + i]);
+    }
+    qs[r][i] = x;
+  }
+  __syncthreads();
+  float acc[HG];
+#pragma unroll
+  for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
+  const float4* row = reinterpret_cast<const float4*>(Pi + (int64_t)i * D);
+  for (int j4 = 0; j4 < D / 4; ++j4) {
+    const float4 p = row[j4];
+#pragma unroll
+    for (int r = 0; r < HG; ++r) {
+      acc[r] = fmaf(p.x, qs[r][4 * j4 + 0], acc[r]);
+      acc[r] = fmaf(p.y, qs[r][4 * j4 + 1], acc[r]);
+      acc[r] = fmaf(p.z, qs[r][4 * j4 + 2], acc[r]);
+      acc[r] = fmaf(p.w, qs[r][4 * j4 + 3], acc[r]);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < HG; ++r) {
+    qr[r][i] = acc[r];
+    if (r < nh) qrot[(int64_t)(h0 + r) * D + i] = acc[r];
+  }
+  if (!qjl) return;
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
+  const float4* srow = reinterpret_cast<const float4*>(S + (int64_t)i * D);
+  for (int j4 = 0; j4 < D / 4; ++j4) {
+    const float4 p = srow[j4];
+#pragma unroll
+    for (int r = 0; r < HG; ++r) {
+      acc[r] = fmaf(p.x, qr[r][4 * j4 + 0], acc[r]);
+      acc[r] = fmaf(p.y, qr[r][4 * j4 + 1], acc[r]);
+      acc[r] = fmaf(p.z, qr[r][4 * j4 + 2], acc[r]);
+      acc[r] = fmaf(p.w, qr[r][4 * j4 + 3], acc[r]);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < HG; ++r)
+    if (r < nh) sq[(int64_t)(h0 + r) * D + i] = acc[r];
+}
+
+// ------------------------------------------------------------------------------------------ split
+
+template <int KB, int VB, bool QJL>
+struct Layout {
+  static constexpr int K_ROW = 16 * KB;
+  static constexpr int V_ROW = 16 * VB;
+  static constexpr int LUT_K = (1 << (2 * KB)) * 32;  // uint32 entries
+  static constexpr int LUT_V = (1 << (2 * VB)) * 32;
+  static constexpr int OFF_KC = 0;
+  static constexpr int OFF_SG = OFF_KC + STAGE_TOK * K_ROW;
+  static constexpr int OFF_VC = OFF_SG + (QJL ? STAGE_TOK * 16 : 0);
+  static constexpr int OFF_NK = OFF_VC + STAGE_TOK * V_ROW;
+  static constexpr int OFF_RN = OFF_NK + STAGE_TOK * 4;
+  static constexpr int OFF_NV = OFF_RN + (QJL ? STAGE_TOK * 4 : 0);
+  static constexpr int STAGE_BYTES = OFF_NV + STAGE_TOK * 4;
+  static constexpr int LUT_BYTES = 4 * (LUT_K + LUT_V);
+  static constexpr int MERGE_BYTES = 4 * (WARPS * HG * 2 + WARPS * HG * D);
+  static constexpr int PIPE_BYTES = NSTAGE * STAGE_BYTES;
+  static constexpr int SMEM = LUT_BYTES + (PIPE_BYTES > MERGE_BYTES ? PIPE_BYTES : MERGE_BYTES);
+  static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
+};
+
+template <int KB, int VB, bool QJL>
+__device__ __forceinline__ void load_stage(const DArgs& a, unsigned char* stage, int64_t row0,
+                                           int count) {
+  using Lay = Layout<KB, VB, QJL>;
+  const int tid = threadIdx.x;
+  // key codes: KB 16-byte chunks per token
+  {
+    const uint8_t* src = a.k_codes + row0 * Lay::K_ROW;
+    for (int i = tid; i < STAGE_TOK * KB; i += THREADS) {
+      const bool ok = i < count * KB;
+      cp_async16(stage + Lay::OFF_KC + 16 * i, ok ? src + 16 * i : a.k_codes, ok ? 16 : 0);
+    }
+  }
+  if constexpr (QJL) {
+    const uint8_t* src = a.k_signs + row0 * 16;
+    for (int i = tid; i < STAGE_TOK; i += THREADS) {
+      const bool ok = i < count;
+      cp_async16(stage + Lay::OFF_SG + 16 * i, ok ? src + 16 * i : a.k_signs, ok ? 16 : 0);
+    }
+  }
+  {
+    const uint8_t* src = a.v_codes + row0 * Lay::V_ROW;
+    for (int i = tid; i < STAGE_TOK * VB; i += THREADS) {
+      const bool ok = i < count * VB;
+      cp_async16(stage + Lay::OFF_VC + 16 * i, ok ? src + 16 * i : a.v_codes, ok ? 16 : 0);
+    }
+  }
+  for (int i = tid; i < STAGE_TOK; i += THREADS) {
+    const bool ok = i < count;
+    cp_async4(stage + Lay::OFF_NK + 4 * i, ok ? a.k_norm + row0 + i : a.k_norm, ok ? 4 : 0);
+    if constexpr (QJL)
+      cp_async4(stage + Lay::OFF_RN + 4 * i, ok ? a.k_rnorm + row0 + i : a.k_rnorm, ok ? 4 : 0);
+    cp_async4(stage + Lay::OFF_NV + 4 * i, ok ? a.v_norm + row0 + i : a.v_norm, ok ? 4 : 0);
+  }
+}
+
+// Value chunk of one token for this lane group (16 codes of VB bits) as a 64-bit integer.
+template <int VB>
+__device__ __forceinline__ uint64_t load_v_chunk(const unsigned char* row, int gid) {
+  if constexpr (VB == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * gid);
+    return (uint64_t)w.x | ((uint64_t)w.y << 32);
+  } else if constexpr (VB == 2) {
+    return (uint64_t)*reinterpret_cast<const uint32_t*>(row + 4 * gid);
+  } else {  // 6 bytes per lane group: read the aligned 12 bytes of the group pair
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(row + 12 * (gid >> 1));
+    const uint32_t w0 = p[0], w1 = p[1], w2 = p[2];
+    if (gid & 1) return (uint64_t)((w1 >> 16) | (w2 << 16)) | ((uint64_t)(w2 >> 16) << 32);
+    return (uint64_t)w0 | ((uint64_t)(w1 & 0xffffu) << 32);
+  }
+}
+
+template <int KB, int VB, bool QJL>
+__global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
+  using Lay = Layout<KB, VB, QJL>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* lutK = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* lutV = lutK + Lay::LUT_K;
+  unsigned char* pipe = smem + Lay::LUT_BYTES;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, t = lane & 3;
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y / a.hgroups, hg = blockIdx.y % a.hgroups;
+  const int b = blockIdx.z;
+  const int h0 = kvh * a.g + hg * HG;
+  const int nh = min(HG, a.g - hg * HG);
+  const int tok_begin = split * a.tps;
+  const int tok_end = min(a.seq_len, tok_begin + a.tps);
+  const int ntok = max(0, tok_end - tok_begin);
+  const int nstages = (ntok + STAGE_TOK - 1) / STAGE_TOK;
+  const int64_t row_base = ((int64_t)b * a.Hkv + kvh) * a.T_cap;
+
+  // Start the pipeline before building the tables.
+#pragma unroll
+  for (int s = 0; s < NSTAGE - 1; ++s) {
+    if (s < nstages)
+      load_stage<KB, VB, QJL>(a, pipe + s * Lay::STAGE_BYTES, row_base + tok_begin + s * STAGE_TOK,
+                              min(STAGE_TOK, ntok - s * STAGE_TOK));
+    cp_commit();
+  }
+
+  // Pair tables: entry e = lo | hi << B  ->  half2(c[lo], c[hi]), replicated per lane (bank = lane).
+  for (int i = tid; i < Lay::LUT_K; i += THREADS) {
+    const int e = i >> 5;
+    lutK[i] = pack_half2(a.kc[e & ((1 << KB) - 1)], a.kc[e >> KB]);
+  }
+  for (int i = tid; i < Lay::LUT_V; i += THREADS) {
+    const int e = i >> 5;
+    lutV[i] = pack_half2(a.vc[e & ((1 << VB) - 1)], a.vc[e >> VB]);
+  }
+
+  // A fragments: rows 0-7 = q' hi of the group's heads, rows 8-15 = q' lo; sq hi only.
+  uint32_t aq[8][4], asq[8][2];
+  {
+    const bool live = gid < nh;
+    const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? gid : 0)) * D;
+    const float* sp = a.sq + ((int64_t)b * a.Hq + h0 + (live ? gid : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = 16 * kk + 8 * half + 2 * t;
+        float x0 = live ? qp[c0] : 0.0f, x1 = live ? qp[c0 + 1] : 0.0f;
+        float h0f, l0f, h1f, l1f;
+        split_half(x0, h0f, l0f);
+        split_half(x1, h1f, l1f);
+        aq[kk][2 * half + 0] = pack_half2(h0f, h1f);
+        aq[kk][2 * half + 1] = pack_half2(l0f, l1f);
+        if constexpr (QJL) {
+          const float s0 = live ? sp[c0] : 0.0f, s1 = live ? sp[c0 + 1] : 0.0f;
+          asq[kk][half] = pack_half2(s0, s1);
+        } else {
+          asq[kk][half] = 0u;
+        }
+      }
+    }
+  }
+
+  float oacc[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
+  float m_run = -INFINITY, l_run = 0.0f;
+  const uint32_t lut_lane = (uint32_t)lane;
+
+  for (int st = 0; st < nstages; ++st) {
+    cp_wait<NSTAGE - 2>();
+    __syncthreads();
+    {
+      const int s = st + NSTAGE - 1;
+      if (s < nstages)
+        load_stage<KB, VB, QJL>(a, pipe + (s % NSTAGE) * Lay::STAGE_BYTES,
+                                row_base + tok_begin + s * STAGE_TOK,
+                                min(STAGE_TOK, ntok - s * STAGE_TOK));
+      cp_commit();
+    }
+    const int wtok0 = st * STAGE_TOK + 16 * warp;  // first token of this warp, relative to range
+    if (wtok0 >= ntok) continue;                    // warp-uniform
+    const unsigned char* stage = pipe + (st % NSTAGE) * Lay::STAGE_BYTES;
+
+    // ---- scores: S = Q' Khat^T (16 rows x 8 tokens per n-block) ----
+    float kacc[2][4], qacc[2][4];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = 0.0f;
+      const int r = 16 * warp + 8 * nb + gid;
+      uint32_t ck[KB];
+      const uint32_t* kw = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r * Lay::K_ROW + 4 * KB * t);
+#pragma unroll
+      for (int i = 0; i < KB; ++i) ck[i] = kw[i];
+#define TQ_KSTEP(KK)                                                                      \
+      {                                                                                   \
+        const uint32_t b0 = lutK[k_pair_index<KB, 2 * (KK)>(ck) * 32 + lut_lane];         \
+        const uint32_t b1 = lutK[k_pair_index<KB, 2 * (KK) + 1>(ck) * 32 + lut_lane];     \
+        mma16816(kacc[nb], aq[KK], b0, b1);                                               \
+      }
+      TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
+#undef TQ_KSTEP
+      if constexpr (QJL) {
+        const uint32_t sw = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r * 16 + 4 * t);
+#define TQ_SSTEP(KK)                                                                      \
+        {                                                                                 \
+          const uint32_t aa[4] = {asq[KK][0], 0u, asq[KK][1], 0u};                        \
+          mma16816(qacc[nb], aa, sign_pair<2 * (KK)>(sw), sign_pair<2 * (KK) + 1>(sw));   \
+        }
+        TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
+#undef TQ_SSTEP
+      }
+    }
+
+    // ---- online softmax (log2 units); this lane owns head gid, tokens 2t, 2t+1 (+8) ----
+    float sc[2][2], pv[2][2];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+      const int tl = 16 * warp + 8 * nb + 2 * t;  // token within the stage
+      const float2 nk = *reinterpret_cast<const float2*>(stage + Lay::OFF_NK + 4 * tl);
+      float2 rn = make_float2(0.f, 0.f);
+      if constexpr (QJL) rn = *reinterpret_cast<const float2*>(stage + Lay::OFF_RN + 4 * tl);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float n = e ? nk.y : nk.x;
+        const float rr = e ? rn.y : rn.x;
+        float s = (kacc[nb][e] + kacc[nb][2 + e]) * (n * a.sK);
+        if constexpr (QJL) s = fmaf(qacc[nb][e], rr * a.sQ, s);
+        const bool valid = (st * STAGE_TOK + tl + e) < ntok;
+        sc[nb][e] = valid ? s : -INFINITY;
+      }
+    }
+    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const bool grow = m_new > m_run;
+    if (__any_sync(FULL, grow)) {
+      const float alpha = grow ? ex2(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        oacc[i][0] *= alpha;
+        oacc[i][1] *= alpha;
+        oacc[i][2] *= alpha;
+        oacc[i][3] *= alpha;
+      }
+      l_run *= alpha;
+      m_run = m_new;
+    }
+    uint32_t ap[4];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+      const int tl = 16 * warp + 8 * nb + 2 * t;
+      const float2 nv = *reinterpret_cast<const float2*>(stage + Lay::OFF_NV + 4 * tl);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float p = (m_run == -INFINITY) ? 0.0f : ex2(sc[nb][e] - m_run);
+        l_run += p;
+        pv[nb][e] = p * (e ? nv.y : nv.x) * 0.08838834764831845f;  // p * nV / sqrt(128)
+      }
+      float h0f, l0f, h1f, l1f;
+      split_half(pv[nb][0], h0f, l0f);
+      split_half(pv[nb][1], h1f, l1f);
+      ap[2 * nb + 0] = pack_half2(h0f, h1f);  // rows gid   : hi
+      ap[2 * nb + 1] = pack_half2(l0f, l1f);  // rows gid+8 : lo
+    }
+
+    // ---- O' += P Vhat: 16 n-blocks of 8 dims; B holds token pairs (2t,2t+1), (2t+8,2t+9) ----
+    {
+      const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
+      const uint64_t cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gid);
+      const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gid);
+      const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gid);
+      const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gid);
+#define TQ_VSTEP(NU)                                                                        \
+      {                                                                                     \
+        const uint32_t e0 = v_code<VB, NU>(cv0) | (v_code<VB, NU>(cv1) << VB);              \
+        const uint32_t e1 = v_code<VB, NU>(cv2) | (v_code<VB, NU>(cv3) << VB);              \
+        mma16816(oacc[NU], ap, lutV[e0 * 32 + lut_lane], lutV[e1 * 32 + lut_lane]);         \
+      }
+      TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3) TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
+      TQ_VSTEP(8) TQ_VSTEP(9) TQ_VSTEP(10) TQ_VSTEP(11) TQ_VSTEP(12) TQ_VSTEP(13) TQ_VSTEP(14) TQ_VSTEP(15)
+#undef TQ_VSTEP
+    }
+  }
+  cp_wait<0>();
+  __syncthreads();  // pipeline buffers are reused for the merge below
+
+  // ---- merge the 4 warps of this CTA ----
+  float* mw = reinterpret_cast<float*>(pipe);  // [WARPS][HG]
+  float* lw = mw + WARPS * HG;                 // [WARPS][HG]
+  float* ow = lw + WARPS * HG;                 // [WARPS][HG][D]
+  float lq = l_run;
+  lq += __shfl_xor_sync(FULL, lq, 1);
+  lq += __shfl_xor_sync(FULL, lq, 2);
+  if (t == 0) {
+    mw[warp * HG + gid] = m_run;
+    lw[warp * HG + gid] = lq;
+  }
+#pragma unroll
+  for (int nu = 0; nu < 16; ++nu) {
+    float* o = ow + (warp * HG + gid) * D + 8 * nu + 2 * t;
+    o[0] = oacc[nu][0] + oacc[nu][2];
+    o[1] = oacc[nu][1] + oacc[nu][3];
+  }
+  __syncthreads();
+  for (int r = 0; r < nh; ++r) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, mw[w * HG + r]);
+    float L = 0.0f, O = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      const float mwr = mw[w * HG + r];
+      const float f = (mwr == -INFINITY) ? 0.0f : ex2(mwr - M);
+      L += f * lw[w * HG + r];
+      O += f * ow[(w * HG + r) * D + tid];
+    }
+    float* dst = a.part + (((int64_t)b * a.Hq + h0 + r) * a.splits + split) * PART;
+    dst[2 + tid] = O;
+    if (tid == 0) {
+      dst[0] = M;
+      dst[1] = L;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------ reduce
+
+__global__ void __launch_bounds__(D) reduce_kernel(const float* __restrict__ part, int splits,
+                                                  const float* __restrict__ Pi, float* __restrict__ out) {
+  __shared__ float ob[D];
+  const int bh = blockIdx.x, j = threadIdx.x;
+  const float* p = part + (int64_t)bh * splits * PART;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * PART]);
+  float L = 0.0f, O = 0.0f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float ms = p[s * PART];
+      const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
+      L += f * p[s * PART + 1];
+      O += f * p[s * PART + 2 + j];
+    }
+  }
+  ob[j] = L > 0.0f ? O / L : 0.0f;
+  __syncthreads();
+  float acc = 0.0f;  // o_i = sum_j Pi[j][i] o'_j
+  for (int jj = 0; jj < D; ++jj) acc = fmaf(Pi[jj * D + j], ob[jj], acc);
+  out[(int64_t)bh * D + j] = acc;
+}
+
+// ------------------------------------------------------------------------------------------ host
+
+struct Plan {
+  int hgroups, splits, tps;
+};
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return sms;
+}
+
+Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
+  Plan p;
+  const int g = Hq / Hkv;
+  p.hgroups = (g + HG - 1) / HG;
+  const int64_t units = (int64_t)B * Hkv * p.hgroups;
+  if (seq_len <= 0) {
+    p.splits = 1;
+    p.tps = STAGE_TOK;
+    return p;
+  }
+  const int64_t target = 4LL * sms;  // 2 resident CTAs per SM, two waves
+  int64_t splits = (target + units - 1) / units;
+  const int64_t max_splits = (seq_len + 4 * STAGE_TOK - 1) / (4 * STAGE_TOK);  // >= 4 stages each
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int64_t tps = (seq_len + splits - 1) / splits;
+  tps = (tps + STAGE_TOK - 1) / STAGE_TOK * STAGE_TOK;
+  p.tps = (int)tps;
+  p.splits = (int)((seq_len + tps - 1) / tps);
+  return p;
+}
+
+size_t workspace_bytes(int B, int Hq, const Plan& p) {
+  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART);
+}
+
+template <int KB, int VB, bool QJL>
+tq_status launch_split(const DArgs& a, dim3 grid, cudaStream_t stream) {
+  using Lay = Layout<KB, VB, QJL>;
+  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
+  split_kernel<KB, VB, QJL><<<grid, THREADS, Lay::SMEM, stream>>>(a);
+  return TQ_OK;
+}
+
+template <int KB, bool QJL>
+tq_status dispatch_v(int vb, const DArgs& a, dim3 grid, cudaStream_t s) {
+  switch (vb) {
+    case 2: return launch_split<KB, 2, QJL>(a, grid, s);
+    case 3: return launch_split<KB, 3, QJL>(a, grid, s);
+    default: return launch_split<KB, 4, QJL>(a, grid, s);
+  }
+}
+
+template <bool QJL>
+tq_status dispatch(int kb, int vb, const DArgs& a, dim3 grid, cudaStream_t s) {
+  switch (kb) {
+    case 2: return dispatch_v<2, QJL>(vb, a, grid, s);
+    case 3: return dispatch_v<3, QJL>(vb, a, grid, s);
+    default: return dispatch_v<4, QJL>(vb, a, grid, s);
+  }
+}
+
+}  // namespace
+}  // namespace tq
+
+extern "C" size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_len) {
+  using namespace tq;
+  if (!cache || B < 1 || Hq < 1 || cache->Hkv < 1 || Hq % cache->Hkv || seq_len < 0) return 0;
+  const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
+  return workspace_bytes(B, Hq, p);
+}
+
+extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, int Hq,
+                                    const tq_cache* cache, int seq_len, float scale, float* out,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  using namespace tq;
+  clear_error();
+  tq_status st = check_cache(cache);
+  if (st != TQ_OK) return st;
+  st = check_params(params, cache);
+  if (st != TQ_OK) return st;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, "q_dtype %d", q_dtype);
+  if (Hq < 1 || Hq % cache->Hkv) return fail(TQ_ERR_INVALID_ARG, "Hq %d vs Hkv %d", Hq, cache->Hkv);
+  if (seq_len < 0 || seq_len > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "seq_len %d outside [0, %d]", seq_len, cache->T_cap);
+  if (!q || !out || !workspace) return fail(TQ_ERR_INVALID_ARG, "q / out / workspace is NULL");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
+    return fail(TQ_ERR_INVALID_ARG, "q / out / workspace must be 16-byte aligned");
+  const int B = cache->B;
+  const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
+  const size_t need = workspace_bytes(B, Hq, plan);
+  if (ws_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+
+  const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)D);
+  float* ws = reinterpret_cast<float*>(workspace);
+  DArgs a;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = cache->Hkv;
+  a.g = Hq / cache->Hkv;
+  a.hgroups = plan.hgroups;
+  a.T_cap = cache->T_cap;
+  a.seq_len = seq_len;
+  a.splits = plan.splits;
+  a.tps = plan.tps;
+  a.sK = (float)((double)sc * 1.4426950408889634 / sqrt((double)D));
+  a.sQ = cache->qjl_m ? (float)((double)sc * 1.4426950408889634 * 2.0 * sqrt(M_PI / 2.0) / cache->qjl_m)
+                      : 0.0f;
+  a.k_codes = cache->k_codes;
+  a.k_signs = cache->k_signs;
+  a.k_norm = cache->k_norm;
+  a.k_rnorm = cache->k_rnorm;
+  a.v_codes = cache->v_codes;
+  a.v_norm = cache->v_norm;
+  a.kc = params->k_centroids;
+  a.vc = params->v_centroids;
+  a.qrot = ws;
+  a.sq = ws + (size_t)B * Hq * D;
+  a.part = ws + (size_t)2 * B * Hq * D;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  const int BH = B * Hq;
+  const int prep_grid = (BH + HG - 1) / HG;
+  if (q_dtype == TQ_F32)
+    prep_kernel<float><<<prep_grid, D, 0, s>>>(reinterpret_cast<const float*>(q), params->Pi,
+                                              params->S, BH, cache->qjl_m ? 1 : 0, ws,
+                                              ws + (size_t)BH * D);
+  else
+    prep_kernel<__nv_bfloat16><<<prep_grid, D, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(q),
+                                                      params->Pi, params->S, BH, cache->qjl_m ? 1 : 0,
+                                                      ws, ws + (size_t)BH * D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
+
+  const dim3 grid(plan.splits, cache->Hkv * plan.hgroups, B);
+  st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, a, grid, s)
+                    : dispatch<false>(cache->k_bits, cache->v_bits, a, grid, s);
+  if (st != TQ_OK) return st;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "split launch: %s", cudaGetErrorString(e));
+
+  reduce_kernel<<<BH, D, 0, s>>>(a.part, plan.splits, params->Pi, out);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}

@@ -1,0 +1,47 @@
+// Internal helpers shared by the host entry points and the kernels of the tq library.
+#pragma once
+
+#include <cstdarg>
+#include <cstddef>
+#include <cstdint>
+
+#include "tq.h"
+
+#ifndef __CUDACC__
+#define __host__
+#define __device__
+#endif
+
+namespace tq {
+
+constexpr int kHeadDim = 128;
+constexpr int kQjlRows = 128;
+
+// Thread-local error detail; returns `st` so callers can `return fail(...)`.
+tq_status fail(tq_status st, const char* fmt, ...);
+void clear_error();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Packed-row slot maps (the cache layout documented in tq.h).
+// Key-code rows and sign rows are ordered for the decode kernel's m16n8k16 B fragments:
+// thread tau of a quad owns coordinates 16*a + 8*h + 2*tau + e.
+__host__ __device__ inline int k_slot_of_coord(int j) {
+  const int a = j >> 4, h = (j >> 3) & 1, t = (j >> 1) & 3, e = j & 1;
+  return 32 * t + 4 * a + 2 * h + e;
+}
+// Value-code rows: lane group g of a warp owns coordinates 8*n + g.
+__host__ __device__ inline int v_slot_of_coord(int j) {
+  const int n = j >> 3, g = j & 7;
+  return 16 * g + n;
+}
+__host__ __device__ inline int sign_bit_of_row(int l) {
+  const int a = l >> 4, h = (l >> 3) & 1, t = (l >> 1) & 3, e = l & 1;
+  return 32 * t + (2 * a + h) + 16 * e;
+}
+
+// Validation shared by tq_quantize / tq_decode_attn.
+tq_status check_params(const tq_params* p, const tq_cache* c);
+tq_status check_cache(const tq_cache* c);
+
+}  // namespace tq

@@ -1,0 +1,165 @@
+/*
+ * tq.h -- C ABI of the B200 compressed-KV (TurboQuant-style) hot path.
+ *
+ * Three operations, each on plain pointers and sizes:
+ *
+ *   tq_build_codebook  host     Lloyd-Max quantizer of N(0,1) (computed once per bit width).
+ *   tq_quantize        device   rotate -> scalar-quantize -> pack -> 1-bit QJL sketch of K/V.
+ *   tq_decode_attn     device   single-token attention directly over the packed cache.
+ *
+ * Method sources (page and passage):
+ *   - ai-news.ru TurboQuant overview, paragraphs on the first and second ideas: multiply each
+ *     vector by a random orthogonal matrix so the coordinates become near-Gaussian, then apply a
+ *     Lloyd-Max grid precomputed once for that distribution; static codebook, no calibration.
+ *   - same page, next paragraph ("third component"): a 1-bit QJL correction of the residual.
+ *   - tproger.ru "Google TurboQuant in simple words", sections "Step 1: PolarQuant" (per-coordinate
+ *     Lloyd-Max with no per-group scale bits) and "Step 2: QJL" (one extra bit makes the residual
+ *     error unbiased); section "Benchmarks": a TQ3 block is 52 bytes per 128 values.
+ *   - inner-product estimator used for keys:
+ *       <q,k> ~= <q,k_mse> + ||r|| * sqrt(pi/2)/m * <S q, sign(S r)>,   S Gaussian m x d.
+ *
+ * Conventions (all functions):
+ *   - head_dim is 128.  Bit widths 2..4 for keys and values; qjl_m is 0 (off) or 128.
+ *   - The library never allocates device memory.  All device pointers are caller-owned and must
+ *     stay valid until the work enqueued on `stream` has finished.
+ *   - Device work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream) and is asynchronous.  Argument errors are detected on the host and returned before
+ *     anything is enqueued.  A launch failure returns TQ_ERR_CUDA; tq_last_error() then describes it.
+ *   - Every device pointer must be 16-byte aligned.
+ *
+ * Packed cache layout ([B, Hkv, T_cap] rows, each array contiguous, row r of (b,h,t) at
+ * ((b*Hkv + h)*T_cap + t)):
+ *   k_codes  uint8 [.., 16*k_bits]  key codes; v_codes uint8 [.., 16*v_bits] value codes.
+ *            A row is a little-endian bit stream (row bit k = bit k%8 of byte k/8); slot s holds
+ *            bits [b*s, b*s+b) = the Lloyd index (0 = most negative centroid) of one rotated
+ *            coordinate.  Key rows: coordinate j = 16*a + 8*h + 2*t + e sits at slot
+ *            32*t + 4*a + 2*h + e.  Value rows: coordinate j = 8*n + g sits at slot 16*g + n.
+ *   k_signs  uint8 [.., 16]  QJL bits: sketch row l = 16*a + 8*h + 2*t + e at row bit
+ *            32*t + (2*a + h) + 16*e; a bit is 1 when (S rho)_l >= 0.
+ *   k_norm, v_norm  float [..]  ||x|| of the original vector.
+ *   k_rnorm         float [..]  ||r|| = ||x|| * ||rho|| / sqrt(128), rho = u - c[idx].
+ *   Rotated normalized coordinates: u = sqrt(128) * Pi x / ||x|| (u = 0 when x = 0);
+ *   index = number of thresholds t_i with u >= t_i (a tie goes to the upper cell).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape */
+  TQ_ERR_UNSUPPORTED = 2,   /* head_dim != 128, bits outside 2..4, qjl_m not in {0,128} */
+  TQ_ERR_NO_CONVERGENCE = 3,/* Lloyd iteration did not reach the tolerance */
+  TQ_ERR_WORKSPACE = 4,     /* workspace smaller than tq_decode_workspace_size() */
+  TQ_ERR_CUDA = 5           /* CUDA runtime error (launch or device query) */
+} tq_status;
+
+enum { TQ_F32 = 0, TQ_BF16 = 1 };
+
+/* Static description of a status code.  Never NULL. */
+const char* tq_status_string(int status);
+
+/* Detail of the last failure on the calling thread ("" if none).  Valid until the next call
+ * into this library on the same thread. */
+const char* tq_last_error(void);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int tq_version(void);
+
+/*
+ * Lloyd-Max scalar quantizer of the standard normal density (host, double precision).
+ * Source: ai-news.ru overview, "second idea" (optimal grid for a known distribution, computed
+ * once, stored statically); tproger.ru "Step 1: PolarQuant" (per-coordinate Lloyd-Max).
+ *
+ *   bits        1..8
+ *   max_iter    iteration cap (> 0); tol: stop when the largest centroid move is < tol (> 0)
+ *   centroids   host float[1 << bits]  out: ascending, symmetric, each rounded to the nearest
+ *               fp16 value (so the decode path can use them as exact half-precision operands)
+ *   thresholds  host float[(1 << bits) - 1]  out: exact midpoints of adjacent stored centroids
+ *   distortion  host double* or NULL  out: E[(X - Q(X))^2] of the unrounded Lloyd solution
+ * Errors: TQ_ERR_INVALID_ARG (bits, max_iter, tol, null outputs), TQ_ERR_NO_CONVERGENCE.
+ * The caller owns all arrays.  Thread-safe; no device work.
+ */
+tq_status tq_build_codebook(int bits, int max_iter, double tol, float* centroids,
+                            float* thresholds, double* distortion);
+
+/* Caller-owned packed cache (device pointers; see the layout above).  k_signs and k_rnorm may
+ * be NULL when qjl_m == 0. */
+typedef struct {
+  int B, Hkv, T_cap, head_dim, k_bits, v_bits, qjl_m;
+  uint8_t* k_codes;
+  uint8_t* k_signs;
+  float* k_norm;
+  float* k_rnorm;
+  uint8_t* v_codes;
+  float* v_norm;
+} tq_cache;
+
+/* Per-layer constants (device pointers, caller-owned, fp32).
+ *   Pi            [128 x 128] row-major orthogonal rotation (u = sqrt(128) Pi x / ||x||)
+ *   S             [qjl_m x 128] row-major Gaussian sketch, entries exactly representable in fp16
+ *                 (may be NULL when qjl_m == 0)
+ *   k_centroids   [1 << k_bits], k_thresholds [(1 << k_bits) - 1]  from tq_build_codebook
+ *   v_centroids   [1 << v_bits], v_thresholds [(1 << v_bits) - 1] */
+typedef struct {
+  const float* Pi;
+  const float* S;
+  const float* k_centroids;
+  const float* k_thresholds;
+  const float* v_centroids;
+  const float* v_thresholds;
+} tq_params;
+
+/*
+ * Compress T_new new tokens of K and V into cache rows [t_offset, t_offset + T_new).
+ * Source: tproger.ru "Step 1: PolarQuant" and "Step 2: QJL"; ai-news.ru overview (rotation,
+ * Lloyd-Max, QJL residual); the estimator above fixes what is stored for keys.
+ *
+ *   k, v        device [B, Hkv, T_new, 128] of `dtype` (TQ_F32 or TQ_BF16); element (b,h,t,j) at
+ *               b*stride_b + h*stride_h + t*stride_t + j (strides in elements, shared by k and v;
+ *               the last dimension is contiguous; stride_t * element size a multiple of 16 bytes)
+ *   T_new       >= 0 (0 enqueues nothing);  0 <= t_offset, t_offset + T_new <= cache->T_cap
+ * Output bits are those of the float64 definition except where a rotated coordinate lies within
+ * about 1e-15 of a threshold (the kernel re-derives near-boundary cases in fp64).
+ * Errors: TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA.
+ */
+tq_status tq_quantize(const tq_params* params, const void* k, const void* v, int dtype,
+                      int64_t stride_b, int64_t stride_h, int64_t stride_t, int T_new,
+                      int t_offset, const tq_cache* cache, void* stream);
+
+/*
+ * Bytes of device workspace tq_decode_attn needs for these sizes on the current device
+ * (split-K partials plus the rotated queries).  Returns 0 on invalid sizes.
+ */
+size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_len);
+
+/*
+ * Single-token decode attention over the first seq_len cached tokens.
+ * Source: the estimator above (QJL-corrected scores); tproger.ru "Benchmarks" (4-bit TurboQuant
+ * attention speedups), ai-manual.ru M5 Max KV-cache benchmark (decode over turbo3/turbo4 caches).
+ *
+ *   q           device [B, Hq, 128] of q_dtype (TQ_F32 or TQ_BF16), contiguous
+ *   Hq          query heads; Hq % cache->Hkv == 0, query head h reads kv-head h / (Hq / Hkv)
+ *   seq_len     0 <= seq_len <= cache->T_cap (0 writes zeros)
+ *   scale       softmax scale; <= 0 selects 1/sqrt(128)
+ *   out         device float [B, Hq, 128]:  o = Pi^T sum_i softmax(scale * est_i) vhat'_i
+ *   workspace   device buffer of at least tq_decode_workspace_size() bytes, contents ignored
+ * est_i = <Pi q, (n_i/sqrt(d)) c_K[idx_i]> + ||r_i|| sqrt(pi/2)/m <S Pi q, 2 sign_i - 1>,
+ * vhat'_i = (nV_i/sqrt(d)) c_V[idxV_i]  (rotated basis).
+ * Errors: TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA.
+ */
+tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, int Hq,
+                         const tq_cache* cache, int seq_len, float scale, float* out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 CPU oracle.
+
+Small cases are compared element by element (several tiles plus a ragged tail); the full-size
+workloads are compared on sampled rows / heads that the oracle computes one by one."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_11_b200 as tq
+import workloads as W
+from oracle import tq_oracle as O
+
+from _parity import (EXEMPT_FRACTION_MAX, assert_attention_close, compare_quantized, gpu_inputs,
+                     oracle_cache_arrays, params_for)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "single_head_4k": dict(T=1000, B=1, Hkv=1, Hq=16),
+    "llama3_8b_32k": dict(T=777, B=1, Hkv=2, Hq=8),
+    "llama3_8b_128k_b4": dict(T=531, B=2, Hkv=2, Hq=8),
+    "llama3_70b_16k_b16": dict(T=613, B=2, Hkv=1, Hq=8),
+    "moe_1m": dict(T=900, B=1, Hkv=2, Hq=16, chunk=128),
+}
+
+
+def small(name):
+    return W.CONFIGS[name].scaled(**SMALL[name])
+
+
+def quantize_chunked(params, K, V, cache, t_offset, chunk):
+    T = K.shape[2]
+    for s in range(0, T, chunk):
+        tq.quantize(params, K[:, :, s:s + chunk], V[:, :, s:s + chunk], cache, t_offset=t_offset + s)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_quantize_parity_small(name):
+    w = small(name)
+    params = params_for(w)
+    K, V, Kh, Vh = gpu_inputs(w)
+    t_off = 17
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T + t_off + 9, w.k_bits, w.v_bits, w.qjl_m)
+    quantize_chunked(params, K, V, cache, t_off, w.chunk)
+    torch.cuda.synchronize()
+    stats = compare_quantized(w, cache, Kh, Vh, t_off)
+    assert stats["exempt_codes"] / stats["coords"] <= 10 * EXEMPT_FRACTION_MAX
+    # rows outside the written range are untouched
+    for arr in (cache.k_codes, cache.v_codes, cache.k_norm, cache.v_norm):
+        a = arr.cpu()
+        assert a[:, :, :t_off].abs().sum() == 0 and a[:, :, t_off + w.T:].abs().sum() == 0
+
+
+def test_quantize_streaming_equals_one_shot():
+    w = small("moe_1m")
+    params = params_for(w)
+    K, V, _, _ = gpu_inputs(w)
+    a = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    b = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    tq.quantize(params, K, V, a)
+    quantize_chunked(params, K, V, b, 0, 37)
+    torch.cuda.synchronize()
+    for x, y in zip((a.k_codes, a.k_signs, a.k_norm, a.k_rnorm, a.v_codes, a.v_norm),
+                    (b.k_codes, b.k_signs, b.k_norm, b.k_rnorm, b.v_codes, b.v_norm)):
+        assert torch.equal(x, y)
+
+
+def test_quantize_special_vectors():
+    """Zero vectors, basis vectors, rows of Pi (u hits sqrt(d) on one coordinate), tiny and huge
+    magnitudes, with fp32 and bf16 inputs."""
+    base = W.CONFIGS["llama3_8b_32k"].scaled(T=64, B=1, Hkv=1, Hq=4)
+    Pi = W.rotation_for(base)
+    rng = np.random.default_rng(3)
+    X = np.zeros((1, 1, 64, 128))
+    X[0, 0, 1:9] = np.eye(128)[[0, 5, 17, 64, 100, 127, 3, 9]]
+    X[0, 0, 9:17] = Pi[[0, 1, 2, 50, 77, 126, 127, 33]]
+    X[0, 0, 17:25] = rng.standard_normal((8, 128)) * 1e-30
+    X[0, 0, 25:33] = rng.standard_normal((8, 128)) * 1e30
+    X[0, 0, 33:] = rng.standard_normal((31, 128))
+    for dtype in (torch.float32, torch.bfloat16):
+        w = W.Workload(**{**base.__dict__, "in_dtype": "fp32" if dtype == torch.float32 else "bf16"})
+        params = params_for(w)
+        Kt = torch.tensor(X, dtype=dtype)
+        Vt = torch.tensor(X[:, :, ::-1].copy(), dtype=dtype)
+        cache = tq.Cache.allocate(1, 1, 64, w.k_bits, w.v_bits, w.qjl_m)
+        tq.quantize(params, Kt.cuda(), Vt.cuda(), cache)
+        torch.cuda.synchronize()
+        compare_quantized(w, cache, Kt.double().numpy(), Vt.double().numpy(), 0)
+        assert (cache.k_norm.cpu()[0, 0, 0] == 0) and (cache.k_rnorm.cpu()[0, 0, 0] == 0)
+
+
+def test_quantize_strided_input():
+    """k/v as views with a padded token stride (e.g. a slice of a larger KV buffer)."""
+    w = small("llama3_8b_32k")
+    params = params_for(w)
+    K, V, Kh, Vh = gpu_inputs(w)
+    bigK = torch.zeros(w.B, w.Hkv, w.T, 256, dtype=K.dtype, device="cuda")
+    bigV = torch.zeros_like(bigK)
+    bigK[..., 64:192] = K
+    bigV[..., 64:192] = V
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    tq.quantize(params, bigK[..., 64:192], bigV[..., 64:192], cache)
+    torch.cuda.synchronize()
+    compare_quantized(w, cache, Kh, Vh, 0)
+
+
+def decode_on_oracle_cache(w, seq_lens, scale=None, q_dtype=torch.float32):
+    K, V, Kh, Vh = gpu_inputs(w)
+    q = W.make_queries(w)
+    params = params_for(w)
+    T_cap = w.T + 5
+    arrays, _ = oracle_cache_arrays(w, Kh, Vh, T_cap)
+    cache = tq.Cache.from_arrays(arrays, w.k_bits, w.v_bits, w.qjl_m)
+    qd = q.to(q_dtype).cuda().contiguous()
+    qh = qd.double().cpu().numpy()
+    host = {k: v for k, v in arrays.items()}
+    results = []
+    for L in seq_lens:
+        out = tq.decode_attn(params, qd, cache, L, scale=scale or 0.0)
+        torch.cuda.synchronize()
+        ref = O.decode_attention(qh, W.rotation_for(w), W.qjl_for(w), host, w.k_bits, w.v_bits, L,
+                                 scale=scale)
+        results.append((out.cpu().numpy(), ref))
+    return results
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_parity_small(name):
+    w = small(name)
+    for got, ref in decode_on_oracle_cache(w, [w.T, w.T - 37, 65, 16, 1]):
+        assert_attention_close(got, ref)
+
+
+def test_decode_empty_context_is_zero():
+    w = small("llama3_8b_32k")
+    (got, ref), = decode_on_oracle_cache(w, [0])
+    assert np.all(got == 0) and np.all(ref == 0)
+
+
+def test_decode_scale_and_bf16_query():
+    w = small("llama3_8b_128k_b4")
+    for got, ref in decode_on_oracle_cache(w, [w.T], scale=0.05, q_dtype=torch.bfloat16):
+        assert_attention_close(got, ref)
+
+
+def test_decode_without_qjl():
+    base = small("llama3_8b_32k")
+    w = W.Workload(**{**base.__dict__, "qjl_m": 0})
+    for got, ref in decode_on_oracle_cache(w, [w.T, 100]):
+        assert_attention_close(got, ref)
+
+
+def test_quantize_then_decode_end_to_end():
+    w = small("llama3_8b_128k_b4")
+    params = params_for(w)
+    K, V, Kh, Vh = gpu_inputs(w)
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    tq.quantize(params, K, V, cache)
+    q = W.make_queries(w)
+    out = tq.decode_attn(params, q.cuda(), cache, w.T).cpu().numpy()
+    _, oc = oracle_cache_arrays(w, Kh, Vh)
+    ex = O.code_exempt(oc["k_u"], w.k_bits).sum() + O.code_exempt(oc["v_u"], w.v_bits).sum()
+    ref = O.decode_attention(q.double().numpy(), W.rotation_for(w), W.qjl_for(w), oc, w.k_bits,
+                             w.v_bits, w.T)
+    if ex == 0:
+        assert_attention_close(out, ref)
+    # against exact attention on the uncompressed K/V, 4-bit TurboQuant stays close
+    exact = O.exact_attention(q.double().numpy(), Kh, Vh)
+    assert np.linalg.norm(out - exact) / np.linalg.norm(exact) < 0.2
+
+
+# ------------------------------------------------------------------------------- full size
+
+FULL = ["llama3_8b_32k", "llama3_8b_128k_b4", "llama3_70b_16k_b16", "moe_1m"]
+
+
+def full_inputs(w):
+    K = W.make_kv(w, "k", device="cuda")
+    V = W.make_kv(w, "v", device="cuda")
+    return K, V
+
+
+def sample_rows(w, n, rng):
+    rows = {(0, 0, 0), (w.B - 1, w.Hkv - 1, w.T - 1), (0, w.Hkv - 1, w.T // 2)}
+    while len(rows) < n:
+        rows.add((int(rng.integers(w.B)), int(rng.integers(w.Hkv)), int(rng.integers(w.T))))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_quantize_sampled(name):
+    """Full-size quantize in the launch shape the benchmark times (config 5: 8192-token chunks);
+    sampled rows checked against the oracle on the exact inputs."""
+    w = W.CONFIGS[name]
+    params = params_for(w)
+    K, V = full_inputs(w)
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    quantize_chunked(params, K, V, cache, 0, w.chunk)
+    torch.cuda.synchronize()
+    rows = sample_rows(w, 256, np.random.default_rng(11))
+    idx = torch.tensor(rows, device="cuda")
+    Ks = K[idx[:, 0], idx[:, 1], idx[:, 2]].double().cpu().numpy()
+    Vs = V[idx[:, 0], idx[:, 1], idx[:, 2]].double().cpu().numpy()
+    compare_quantized(w, cache, Ks, Vs, 0, rows=rows)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_decode_sampled(name):
+    """Full-size decode in the benchmark's launch configuration.  One (batch, kv-head) slice of
+    the cache is written from the oracle's own quantization of the exact inputs; the query heads
+    reading that slice are compared with the oracle's decode over the same slice."""
+    w = W.CONFIGS[name]
+    params = params_for(w)
+    K, V = full_inputs(w)
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    quantize_chunked(params, K, V, cache, 0, w.chunk)
+    b, kvh = w.B - 1, w.Hkv - 1
+    Kh = K[b:b + 1, kvh:kvh + 1].double().cpu().numpy()
+    Vh = V[b:b + 1, kvh:kvh + 1].double().cpu().numpy()
+    del K, V
+    arrays, _ = oracle_cache_arrays(w.scaled(B=1, Hkv=1, Hq=w.group), Kh, Vh)
+    for key, arr in arrays.items():
+        getattr(cache, key)[b, kvh].copy_(torch.as_tensor(arr[0, 0]))
+    q = W.make_queries(w, device="cuda")
+    out = tq.decode_attn(params, q, cache, w.T)
+    torch.cuda.synchronize()
+    g = w.group
+    heads = list(range(kvh * g, (kvh + 1) * g))
+    got = out[b, heads].cpu().numpy()
+    ref = O.decode_attention(q[b:b + 1, heads].double().cpu().numpy(), W.rotation_for(w),
+                             W.qjl_for(w), arrays, w.k_bits, w.v_bits, w.T)[0]
+    assert_attention_close(got, ref)
