@@ -11,9 +11,9 @@
 //   split   grid (splits, Hkv * head_groups, B).  A 4-warp CTA streams its token range through a
 //           4-stage cp.async pipeline (64 tokens per stage).  Each warp takes 16 tokens per stage:
 //           codes are turned into fp16 pairs by a lane-replicated shared-memory table (one load per
-//           two coordinates, no bank conflicts), and m16n8k16 tensor-core MMAs compute q'.khat
-//           (q' split into fp16 hi + lo rows), the QJL sign dot (signs -> +-0.5 by one half2 FMA)
-//           and P.vhat (P split into hi + lo rows).  Online softmax runs in log2 units.
+//           two coordinates, no bank conflicts), and m16n8k16 tensor-core MMAs compute q'.khat,
+//           the QJL sign dot (q' and S q' split into fp16 hi + lo rows; signs -> +-0.5 by one
+//           half2 FMA) and P.vhat (P split into hi + lo rows).  Online softmax runs in log2 units.
 //           The CTA merges its 4 warps and writes one (max, sum, o'[128]) partial per head.
 //   reduce  log-sum-exp merge of the split partials, then o = Pi^T o'.
 #include <cuda_bf16.h>
@@ -100,11 +100,12 @@ __device__ __forceinline__ void split_half(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
-// Sign bits -> +-0.5 fp16 pair: bits q and q+16 of w (1 <= q <= 10) placed in the mantissa of 1.0,
-// then one exact half2 FMA maps 1 + b*2^(q-10) to b - 0.5.
+// Sign bits -> +-0.5 fp16 pair: bits q and q+16 of w (1 <= q <= 9) placed in the mantissa of 1.0
+// (fp16 0x3C00: mantissa bits 0-9 are zero, bit 10 is already an exponent bit), then one exact
+// half2 FMA maps 1 + b*2^(q-10) to b - 0.5.
 template <int Q>
 __device__ __forceinline__ uint32_t sign_half2(uint32_t w) {
-  static_assert(Q >= 1 && Q <= 10, "mantissa position");
+  static_assert(Q >= 1 && Q <= 9, "mantissa position");
   const uint32_t x = (w & (0x00010001u << Q)) | 0x3C003C00u;
   const __half2 hx = *reinterpret_cast<const __half2*>(&x);
   const float m = (float)(1 << (10 - Q));
@@ -115,8 +116,8 @@ __device__ __forceinline__ uint32_t sign_half2(uint32_t w) {
 template <int P>
 __device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
   if constexpr (P == 0) return sign_half2<1>(w << 1);
-  else if constexpr (P <= 10) return sign_half2<P>(w);
-  else return sign_half2<P - 10>(w >> 10);
+  else if constexpr (P <= 9) return sign_half2<P>(w);
+  else return sign_half2<P - 9>(w >> 9);
 }
 
 // Pair p (0..15) of a thread's key-code chunk: 2*KB bits starting at bit 2*KB*p.
@@ -311,8 +312,8 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
     lutV[i] = pack_half2(a.vc[e & ((1 << VB) - 1)], a.vc[e >> VB]);
   }
 
-  // A fragments: rows 0-7 = q' hi of the group's heads, rows 8-15 = q' lo; sq hi only.
-  uint32_t aq[8][4], asq[8][2];
+  // A fragments: rows 0-7 = hi parts of the group's heads, rows 8-15 = lo parts (q' and S q').
+  uint32_t aq[8][4], asq[8][4];
   {
     const bool live = gid < nh;
     const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? gid : 0)) * D;
@@ -330,9 +331,12 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
         aq[kk][2 * half + 1] = pack_half2(l0f, l1f);
         if constexpr (QJL) {
           const float s0 = live ? sp[c0] : 0.0f, s1 = live ? sp[c0 + 1] : 0.0f;
-          asq[kk][half] = pack_half2(s0, s1);
+          split_half(s0, h0f, l0f);
+          split_half(s1, h1f, l1f);
+          asq[kk][2 * half + 0] = pack_half2(h0f, h1f);
+          asq[kk][2 * half + 1] = pack_half2(l0f, l1f);
         } else {
-          asq[kk][half] = 0u;
+          asq[kk][2 * half + 0] = asq[kk][2 * half + 1] = 0u;
         }
       }
     }
@@ -380,11 +384,8 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
 #undef TQ_KSTEP
       if constexpr (QJL) {
         const uint32_t sw = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r * 16 + 4 * t);
-#define TQ_SSTEP(KK)                                                                      \
-        {                                                                                 \
-          const uint32_t aa[4] = {asq[KK][0], 0u, asq[KK][1], 0u};                        \
-          mma16816(qacc[nb], aa, sign_pair<2 * (KK)>(sw), sign_pair<2 * (KK) + 1>(sw));   \
-        }
+#define TQ_SSTEP(KK) \
+        mma16816(qacc[nb], asq[KK], sign_pair<2 * (KK)>(sw), sign_pair<2 * (KK) + 1>(sw));
         TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
 #undef TQ_SSTEP
       }
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
         const float n = e ? nk.y : nk.x;
         const float rr = e ? rn.y : rn.x;
         float s = (kacc[nb][e] + kacc[nb][2 + e]) * (n * a.sK);
-        if constexpr (QJL) s = fmaf(qacc[nb][e], rr * a.sQ, s);
+        if constexpr (QJL) s = fmaf(qacc[nb][e] + qacc[nb][2 + e], rr * a.sQ, s);
         const bool valid = (st * STAGE_TOK + tl + e) < ntok;
         sc[nb][e] = valid ? s : -INFINITY;
       }
