@@ -253,7 +253,7 @@ def run_gpu(args, w):
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_e2e:
         Kh = K.cpu().pin_memory()
         Vh = V.cpu().pin_memory()
         qh = q.cpu().pin_memory()
@@ -318,6 +318,8 @@ def run_gpu(args, w):
         "roofline_decode": roof_d, "roofline_quantize": roof_q,
         "cpu_baseline": cb, "e2e": e2e,
         "gpu_launches": args.steps * (n_chunks + 3),
+        "quantize_fp64_fixups": {"coords": tq.quantize_code_fixups(), "key_vectors": tq.quantize_vector_fixups(),
+                                 "calls": (args.warmup + args.steps) * n_chunks},
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
@@ -333,10 +335,15 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.CONFIG_ORDER)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
+    ap.add_argument("--context", type=int, default=None, help="override the workload's context")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = W.CONFIGS[args.workload]
+    if args.batch is not None or args.context is not None:
+        w = w.scaled(B=args.batch, T=args.context, name=w.name + "(resized)")
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -34,7 +34,9 @@ TQ_BF16 = 1
 
 # Functions declared in include/tq.h (checked by the test-suite against the header).
 EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codebook",
-            "tq_quantize", "tq_decode_workspace_size", "tq_decode_attn")
+            "tq_quantize", "tq_quantize_device_errors", "tq_quantize_vector_fixups",
+            "tq_quantize_code_fixups",
+            "tq_decode_workspace_size", "tq_decode_attn")
 
 
 class TqError(RuntimeError):
@@ -82,6 +84,12 @@ def lib() -> ctypes.CDLL:
     L.tq_quantize.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_void_p,
                               ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                               ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache), ctypes.c_void_p]
+    L.tq_quantize_device_errors.restype = ctypes.c_int
+    L.tq_quantize_device_errors.argtypes = []
+    L.tq_quantize_vector_fixups.restype = ctypes.c_longlong
+    L.tq_quantize_vector_fixups.argtypes = []
+    L.tq_quantize_code_fixups.restype = ctypes.c_longlong
+    L.tq_quantize_code_fixups.argtypes = []
     L.tq_decode_workspace_size.restype = ctypes.c_size_t
     L.tq_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache),
                                            ctypes.c_int]
@@ -228,6 +236,21 @@ def quantize(params: Params, k: torch.Tensor, v: torch.Tensor, cache: Cache, t_o
                              ctypes.byref(c), _stream_ptr(stream)))
 
 
+def quantize_device_errors() -> int:
+    """Device-side error bits recorded by tq_quantize (0 = none); synchronizes."""
+    return int(lib().tq_quantize_device_errors())
+
+
+def quantize_vector_fixups() -> int:
+    """Key vectors re-derived in fp64 by tq_quantize so far (diagnostic); synchronizes."""
+    return int(lib().tq_quantize_vector_fixups())
+
+
+def quantize_code_fixups() -> int:
+    """Coordinates re-derived in fp64 by tq_quantize so far (diagnostic); synchronizes."""
+    return int(lib().tq_quantize_code_fixups())
+
+
 def decode_workspace_size(B: int, Hq: int, cache: Cache, seq_len: int) -> int:
     c = cache.as_c()
     return int(lib().tq_decode_workspace_size(int(B), int(Hq), ctypes.byref(c), int(seq_len)))
@@ -256,7 +279,8 @@ def decode_attn(params: Params, q: torch.Tensor, cache: Cache, seq_len: int,
 
 __all__ = [
     "LIB_PATH", "EXPORTED", "TqError", "lib", "status_string", "last_error", "version",
-    "build_codebook", "Params", "Cache", "quantize", "decode_workspace_size", "decode_attn",
+    "build_codebook", "Params", "Cache", "quantize", "quantize_device_errors",
+    "quantize_vector_fixups", "quantize_code_fixups", "decode_workspace_size", "decode_attn",
     "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
     "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16",
 ]

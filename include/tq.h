@@ -134,6 +134,21 @@ tq_status tq_quantize(const tq_params* params, const void* k, const void* v, int
                       int t_offset, const tq_cache* cache, void* stream);
 
 /*
+ * Diagnostics of tq_quantize (host; synchronizes with the device).  The kernel never blocks
+ * without bound: every wait on tensor-core completion gives up after about two seconds, records
+ * the failure here and leaves its tile unwritten.
+ *   tq_quantize_device_errors   bit 0: a completion wait timed out; bit 1: shared memory not
+ *                               1024-byte aligned.  0 = no error since the library was loaded;
+ *                               -1 if the device could not be queried.
+ *   tq_quantize_vector_fixups   number of key vectors whose QJL sketch had a value too close to
+ *                               0 for the tensor-core path and was re-derived in fp64.
+ */
+int tq_quantize_device_errors(void);
+long long tq_quantize_vector_fixups(void);
+/* Number of single coordinates whose code was re-derived in fp64 (value near a threshold). */
+long long tq_quantize_code_fixups(void);
+
+/*
  * Bytes of device workspace tq_decode_attn needs for these sizes on the current device
  * (split-K partials plus the rotated queries).  Returns 0 on invalid sizes.
  */

@@ -34,6 +34,7 @@ def quantize_chunked(params, K, V, cache, t_offset, chunk):
     T = K.shape[2]
     for s in range(0, T, chunk):
         tq.quantize(params, K[:, :, s:s + chunk], V[:, :, s:s + chunk], cache, t_offset=t_offset + s)
+    assert tq.quantize_device_errors() == 0
 
 
 @pytest.mark.parametrize("name", list(SMALL))
