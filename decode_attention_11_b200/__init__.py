@@ -36,7 +36,8 @@ TQ_BF16 = 1
 EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codebook",
             "tq_quantize", "tq_quantize_device_errors", "tq_quantize_vector_fixups",
             "tq_quantize_code_fixups",
-            "tq_decode_workspace_size", "tq_decode_attn")
+            "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
+            "tq_decode_static_workspace_limit")
 
 
 class TqError(RuntimeError):
@@ -97,6 +98,12 @@ def lib() -> ctypes.CDLL:
     L.tq_decode_attn.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int,
                                  ctypes.c_int, ctypes.POINTER(_Cache), ctypes.c_int, ctypes.c_float,
                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    L.tq_decode_attn_static.restype = ctypes.c_int
+    L.tq_decode_attn_static.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_int,
+                                        ctypes.c_int, ctypes.POINTER(_Cache), ctypes.c_int,
+                                        ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
+    L.tq_decode_static_workspace_limit.restype = ctypes.c_size_t
+    L.tq_decode_static_workspace_limit.argtypes = []
     _lib = L
     return L
 
@@ -277,9 +284,35 @@ def decode_attn(params: Params, q: torch.Tensor, cache: Cache, seq_len: int,
     return out
 
 
+def decode_static_workspace_limit() -> int:
+    """Bytes of the fixed device scratch array behind decode_attn_static."""
+    return int(lib().tq_decode_static_workspace_limit())
+
+
+def decode_attn_static(params: Params, q: torch.Tensor, cache: Cache, seq_len: int,
+                       out: Optional[torch.Tensor] = None, scale: float = 0.0,
+                       stream=None) -> torch.Tensor:
+    """decode_attn for callers that cannot allocate device memory when they run decode (inside
+    an allocator callback, under a fixed-footprint runtime, in a plug-in host): the scratch lives
+    in a fixed device array inside the library.  Pass `out` to avoid the one allocation this
+    wrapper would otherwise make.  Calls that overlap on the device share that array and race."""
+    if q.dim() != 3 or q.shape[-1] != 128 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous [B, Hq, 128] tensor")
+    B, Hq, _ = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, 128, dtype=torch.float32, device=q.device)
+    c = cache.as_c()
+    p = params.as_c()
+    _check(lib().tq_decode_attn_static(ctypes.byref(p), q.data_ptr(), _dtype_code(q), int(Hq),
+                                       ctypes.byref(c), int(seq_len), float(scale), out.data_ptr(),
+                                       _stream_ptr(stream)))
+    return out
+
+
 __all__ = [
     "LIB_PATH", "EXPORTED", "TqError", "lib", "status_string", "last_error", "version",
     "build_codebook", "Params", "Cache", "quantize", "quantize_device_errors",
+    "decode_attn_static", "decode_static_workspace_limit",
     "quantize_vector_fixups", "quantize_code_fixups", "decode_workspace_size", "decode_attn",
     "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
     "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16",

@@ -687,3 +687,69 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free decode: the same kernels, with the scratch space in a fixed device array.
+//
+// Some callers cannot allocate device memory at the point where they run decode: code inside a
+// custom allocator or memory-pool callback (which would re-enter itself), runtimes that forbid
+// cudaMalloc after start-up so that the memory footprint stays fixed, and plug-in hosts that hand
+// a library only the tensors of one call.  For them the scratch lives in this array, which every
+// GPU that loads the library holds until the process exits.
+// ------------------------------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace tq {
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = (size_t)4 << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of g_static_ws on the current device, looked up once per device.
+tq_status static_workspace(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(TQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_ws);
+    if (e != cudaSuccess || !p)
+      return fail(TQ_ERR_CUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
+    g_static_ws_ptr[dev] = p;
+  }
+  *out = g_static_ws_ptr[dev];
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+extern "C" size_t tq_decode_static_workspace_limit(void) { return tq::kStaticWorkspaceBytes; }
+
+extern "C" tq_status tq_decode_attn_static(const tq_params* params, const void* q, int q_dtype,
+                                           int Hq, const tq_cache* cache, int seq_len,
+                                           float scale, float* out, void* stream) {
+  using namespace tq;
+  clear_error();
+  if (!cache) return fail(TQ_ERR_INVALID_ARG, "cache is NULL");
+  const size_t need = tq_decode_workspace_size(cache->B, Hq, cache, seq_len);
+  if (need == 0) return fail(TQ_ERR_INVALID_ARG, "invalid sizes B=%d Hq=%d Hkv=%d seq_len=%d",
+                             cache->B, Hq, cache->Hkv, seq_len);
+  if (need > kStaticWorkspaceBytes)
+    return fail(TQ_ERR_WORKSPACE,
+                "decode needs %zu bytes of scratch, above the %zu-byte static workspace; "
+                "use tq_decode_attn with a caller-allocated workspace",
+                need, kStaticWorkspaceBytes);
+  void* ws = nullptr;
+  const tq_status st = static_workspace(&ws);
+  if (st != TQ_OK) return st;
+  return tq_decode_attn(params, q, q_dtype, Hq, cache, seq_len, scale, out, ws,
+                        kStaticWorkspaceBytes, stream);
+}

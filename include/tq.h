@@ -173,6 +173,36 @@ tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, in
                          const tq_cache* cache, int seq_len, float scale, float* out,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * tq_decode_attn_static -- decode attention that allocates nothing and takes no workspace.
+ * The pages describe no counterpart: this is a deployment aid of this library.
+ *
+ * For callers that cannot allocate device memory when they run decode: code running inside a
+ * custom allocator or memory-pool callback (an allocation there would re-enter the allocator),
+ * runtimes that fix their device footprint at start-up and forbid later cudaMalloc, and plug-in
+ * hosts that pass a library only the tensors of one call.  Same arguments and results as
+ * tq_decode_attn without `workspace`/`workspace_bytes`: the scratch lives in a file-scope device
+ * array of tq_decode_static_workspace_limit() bytes (4 MiB) that every GPU loading the library
+ * holds until the process exits.  The function itself calls no cudaMalloc or cudaFree.
+ *
+ *   - Sizes whose scratch (tq_decode_workspace_size) exceeds the limit are rejected with
+ *     TQ_ERR_WORKSPACE before anything is enqueued; use tq_decode_attn for them.
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture begins.
+ *   - All calls on a device share the one array.  Calls whose device work may overlap (different
+ *     streams without ordering, or host threads racing on one device) corrupt each other's
+ *     results; order them on one stream or use tq_decode_attn with separate workspaces.
+ *   - No part of the array needs to start at zero: every byte a call reads was written earlier in
+ *     the same call, and the array keeps the last call's contents afterwards.
+ * Errors: as tq_decode_attn, plus TQ_ERR_WORKSPACE for sizes above the limit.
+ */
+tq_status tq_decode_attn_static(const tq_params* params, const void* q, int q_dtype, int Hq,
+                                const tq_cache* cache, int seq_len, float scale, float* out,
+                                void* stream);
+
+/* Size in bytes of the static scratch array used by tq_decode_attn_static. */
+size_t tq_decode_static_workspace_limit(void);
+
 #ifdef __cplusplus
 }
 #endif
