@@ -6,7 +6,7 @@
 // second ideas plus the third, QJL, component; tproger.ru "Step 1: PolarQuant", "Step 2: QJL").
 // Softmax and the value sum also run in the rotated basis; one final o = Pi^T o' per head.
 //
-// Kernels (all on the caller's stream):
+// Kernels (both on the caller's stream; the second is a programmatic dependent launch):
 //   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace.
 //   split   grid (splits, Hkv * head_groups, B).  A 4-warp CTA streams its token range through a
 //           4-stage cp.async pipeline (64 tokens per stage).  Each warp takes 16 tokens per stage:
@@ -15,7 +15,8 @@
 //           the QJL sign dot (q' and S q' split into fp16 hi + lo rows; signs -> +-0.5 by one
 //           half2 FMA) and P.vhat (P split into hi + lo rows).  Online softmax runs in log2 units.
 //           The CTA merges its 4 warps and writes one (max, sum, o'[128]) partial per head.
-//   reduce  log-sum-exp merge of the split partials, then o = Pi^T o'.
+//           The last CTA of each (batch, kv-head, head group) to finish (completion counter)
+//           merges the split partials by log-sum-exp and writes o = Pi^T o'.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -51,6 +52,9 @@ struct DArgs {
   const float* qrot;
   const float* sq;
   float* part;
+  int* counters;    // one per (batch, kv-head, head group); zeroed by prep
+  const float* Pi;  // final un-rotation
+  float* out;
 };
 
 // ------------------------------------------------------------------------------------------ PTX
@@ -126,12 +130,53 @@ __device__ __forceinline__ uint32_t k_pair_index(const uint32_t (&c)[KB]) {
   constexpr int off = 2 * KB * P;
   constexpr int w = off / 32, sh = off % 32;
   constexpr uint32_t mask = (1u << (2 * KB)) - 1u;
-  if constexpr (sh + 2 * KB <= 32) {
+  if constexpr (KB == 4) {
+    return __byte_perm(c[w], 0u, 0x4440u | (uint32_t)(sh / 8));  // byte sh/8, zero-extended
+  } else if constexpr (sh + 2 * KB <= 32) {
     return (c[w] >> sh) & mask;
   } else {
     return __funnelshift_r(c[w], c[w + 1], sh) & mask;
   }
 }
+
+// Value-code pair indices of tokens a and b (one lane group's 16 codes each): index of code nu is
+// code_a(nu) | code_b(nu) << VB.  For 4- and 2-bit codes the two chunks are interleaved field by
+// field with a few logic operations, after which every index is one byte / nibble extract.
+template <int VB>
+struct VPairs {
+  uint32_t w[VB == 3 ? 4 : 2 * (VB == 4 ? 2 : 1)];
+  __device__ __forceinline__ void build(uint64_t ca, uint64_t cb) {
+    if constexpr (VB == 4) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t a = (uint32_t)(h ? ca >> 32 : ca), b = (uint32_t)(h ? cb >> 32 : cb);
+        w[2 * h + 0] = (a & 0x0F0F0F0Fu) | ((b << 4) & 0xF0F0F0F0u);   // nu = 8h + 2k
+        w[2 * h + 1] = ((a >> 4) & 0x0F0F0F0Fu) | (b & 0xF0F0F0F0u);   // nu = 8h + 2k + 1
+      }
+    } else if constexpr (VB == 2) {
+      const uint32_t a = (uint32_t)ca, b = (uint32_t)cb;
+      w[0] = (a & 0x33333333u) | ((b << 2) & 0xCCCCCCCCu);   // nibble k: nu = 2k
+      w[1] = ((a >> 2) & 0x33333333u) | (b & 0xCCCCCCCCu);   // nibble k: nu = 2k + 1
+    } else {
+      w[0] = (uint32_t)ca;
+      w[1] = (uint32_t)(ca >> 32);
+      w[2] = (uint32_t)cb;
+      w[3] = (uint32_t)(cb >> 32);
+    }
+  }
+  template <int NU>
+  __device__ __forceinline__ uint32_t index() const {
+    if constexpr (VB == 4) {
+      return __byte_perm(w[2 * (NU >> 3) + (NU & 1)], 0u, 0x4440u | (uint32_t)((NU & 7) >> 1));
+    } else if constexpr (VB == 2) {
+      return (w[NU & 1] >> (4 * (NU >> 1))) & 0xFu;
+    } else {
+      const uint64_t ca = (uint64_t)w[0] | ((uint64_t)w[1] << 32);
+      const uint64_t cb = (uint64_t)w[2] | ((uint64_t)w[3] << 32);
+      return (uint32_t)((ca >> (3 * NU)) & 7u) | ((uint32_t)((cb >> (3 * NU)) & 7u) << 3);
+    }
+  }
+};
 
 // Value code nu (0..15) of a thread's 16-code value chunk held in a 64-bit integer.
 template <int VB, int NU>
@@ -141,61 +186,59 @@ __device__ __forceinline__ uint32_t v_code(uint64_t c) {
 
 // ------------------------------------------------------------------------------------------ prep
 
+// One 512-thread block per (batch, query head): q' = Pi q and sq = S q'.  Thread (i, k) forms the
+// partial dot product of row i with elements 32k..32k+31 (eight independent 16-byte loads, so one
+// memory round trip per matrix); block 0 also zeroes the split-completion counters.  The split
+// kernel is launched as a programmatic dependent of this one and starts its prologue early.
+constexpr int PREP_THREADS = 4 * D;
 template <typename QT>
-__global__ void __launch_bounds__(D) prep_kernel(const QT* __restrict__ q, const float* __restrict__ Pi,
-                                                const float* __restrict__ S, int BH, int qjl,
-                                                float* __restrict__ qrot, float* __restrict__ sq) {
-  __shared__ float qs[HG][D];
-  __shared__ float qr[HG][D];
-  const int i = threadIdx.x;
-  const int h0 = blockIdx.x * HG;
-  const int nh = min(HG, BH - h0);
-  for (int r = 0; r < HG; ++r) {
-    float x = 0.0f;
-    if (r < nh) {
-      if constexpr (sizeof(QT) == 4) x = (float)q[(int64_t)(h0 + r) * D + i];
-      else x = __bfloat162float(q[(int64_t)(h0 + r) * D + i]);
-    }
-    qs[r][i] = x;
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const QT* __restrict__ q,
+                                                           const float* __restrict__ Pi,
+                                                           const float* __restrict__ S, int qjl,
+                                                           float* __restrict__ qrot,
+                                                           float* __restrict__ sq,
+                                                           int* __restrict__ counters,
+                                                           int n_counters) {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  __shared__ __align__(16) float qs[D];
+  __shared__ __align__(16) float qr[D];
+  const int tid = threadIdx.x, i = tid >> 2, k = tid & 3;
+  const int64_t bh = blockIdx.x;
+  if (blockIdx.x == 0)
+    for (int c = tid; c < n_counters; c += PREP_THREADS) counters[c] = 0;
+  if (tid < D) {
+    if constexpr (sizeof(QT) == 4) qs[tid] = (float)q[bh * D + tid];
+    else qs[tid] = __bfloat162float(q[bh * D + tid]);
   }
   __syncthreads();
-  float acc[HG];
+  auto dot_row = [&](const float* M, const float* vec) {
+    const float4* row = reinterpret_cast<const float4*>(M + i * D + 32 * k);
+    const float4* v4 = reinterpret_cast<const float4*>(vec + 32 * k);
+    float4 p[8];
 #pragma unroll
-  for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
-  const float4* row = reinterpret_cast<const float4*>(Pi + (int64_t)i * D);
-  for (int j4 = 0; j4 < D / 4; ++j4) {
-    const float4 p = row[j4];
+    for (int c = 0; c < 8; ++c) p[c] = row[c];
+    float acc = 0.0f;
 #pragma unroll
-    for (int r = 0; r < HG; ++r) {
-      acc[r] = fmaf(p.x, qs[r][4 * j4 + 0], acc[r]);
-      acc[r] = fmaf(p.y, qs[r][4 * j4 + 1], acc[r]);
-      acc[r] = fmaf(p.z, qs[r][4 * j4 + 2], acc[r]);
-      acc[r] = fmaf(p.w, qs[r][4 * j4 + 3], acc[r]);
+    for (int c = 0; c < 8; ++c) {
+      const float4 x = v4[c];
+      acc = fmaf(p[c].x, x.x, acc);
+      acc = fmaf(p[c].y, x.y, acc);
+      acc = fmaf(p[c].z, x.z, acc);
+      acc = fmaf(p[c].w, x.w, acc);
     }
-  }
-#pragma unroll
-  for (int r = 0; r < HG; ++r) {
-    qr[r][i] = acc[r];
-    if (r < nh) qrot[(int64_t)(h0 + r) * D + i] = acc[r];
+    acc += __shfl_xor_sync(FULL, acc, 1);
+    acc += __shfl_xor_sync(FULL, acc, 2);
+    return acc;
+  };
+  const float v = dot_row(Pi, qs);
+  if (k == 0) {
+    qr[i] = v;
+    qrot[bh * D + i] = v;
   }
   if (!qjl) return;
   __syncthreads();
-#pragma unroll
-  for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
-  const float4* srow = reinterpret_cast<const float4*>(S + (int64_t)i * D);
-  for (int j4 = 0; j4 < D / 4; ++j4) {
-    const float4 p = srow[j4];
-#pragma unroll
-    for (int r = 0; r < HG; ++r) {
-      acc[r] = fmaf(p.x, qr[r][4 * j4 + 0], acc[r]);
-      acc[r] = fmaf(p.y, qr[r][4 * j4 + 1], acc[r]);
-      acc[r] = fmaf(p.z, qr[r][4 * j4 + 2], acc[r]);
-      acc[r] = fmaf(p.w, qr[r][4 * j4 + 3], acc[r]);
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < HG; ++r)
-    if (r < nh) sq[(int64_t)(h0 + r) * D + i] = acc[r];
+  const float w = dot_row(S, qr);
+  if (k == 0) sq[bh * D + i] = w;
 }
 
 // ------------------------------------------------------------------------------------------ split
@@ -214,7 +257,9 @@ struct Layout {
   static constexpr int OFF_NV = OFF_RN + (QJL ? STAGE_TOK * 4 : 0);
   static constexpr int STAGE_BYTES = OFF_NV + STAGE_TOK * 4;
   static constexpr int LUT_BYTES = 4 * (LUT_K + LUT_V);
-  static constexpr int MERGE_BYTES = 4 * (WARPS * HG * 2 + WARPS * HG * D);
+  // scratch after the pipeline: the CTA's own warp merge, then (last CTA) the split merge
+  static constexpr int MERGE_BYTES = 4 * (2 * HG + HG * D + 4 * HG * D + 4 * HG);
+  static_assert(MERGE_BYTES >= 4 * (WARPS * HG * 2 + WARPS * HG * D), "warp merge scratch");
   static constexpr int PIPE_BYTES = NSTAGE * STAGE_BYTES;
   static constexpr int SMEM = LUT_BYTES + (PIPE_BYTES > MERGE_BYTES ? PIPE_BYTES : MERGE_BYTES);
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
@@ -272,6 +317,90 @@ __device__ __forceinline__ uint64_t load_v_chunk(const unsigned char* row, int g
   }
 }
 
+// Log-sum-exp merge of the split partials of heads h0 .. h0+nh-1 of batch b, then o = Pi^T o'.
+// Run by the last CTA to finish; partials are read from L2 (written by other CTAs).
+__device__ void merge_splits(const DArgs& a, int b, int h0, int nh, unsigned char* scratch) {
+  const int tid = threadIdx.x;
+  const int S = a.splits;
+  float* Mr = reinterpret_cast<float*>(scratch);  // [HG]
+  float* Lr = Mr + HG;                             // [HG]
+  float* ob = Lr + HG;                             // [HG][D]
+  float* part4 = ob + HG * D;                      // [4][HG][D] partial sums over split groups
+  float* ls4 = part4 + 4 * HG * D;                 // [4][HG]
+  for (int r = 0; r < nh; ++r) {
+    const float* p = a.part + ((int64_t)b * a.Hq + h0 + r) * S * PART;
+    float m = -INFINITY;
+    for (int s2 = tid; s2 < S; s2 += THREADS) m = fmaxf(m, __ldcg(p + (int64_t)s2 * PART));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    if ((tid & 31) == 0) ob[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0) {
+      float M = -INFINITY;
+      for (int w = 0; w < WARPS; ++w) M = fmaxf(M, ob[w]);
+      Mr[r] = M;
+    }
+    __syncthreads();
+  }
+  // thread = (split group g, 4-dim slice j4): sum over splits s = g (mod 4)
+  const int g = tid >> 5, j4 = tid & 31;
+  for (int r = 0; r < nh; ++r) {
+    const float M = Mr[r];
+    const float* p = a.part + ((int64_t)b * a.Hq + h0 + r) * S * PART;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll 8
+      for (int s2 = g; s2 < S; s2 += 4) {
+        const float* ps = p + (int64_t)s2 * PART;
+        const float ms = __ldcg(ps);
+        const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
+        const float2 lo = __ldcg(reinterpret_cast<const float2*>(ps + 2 + 4 * j4));
+        const float2 hi = __ldcg(reinterpret_cast<const float2*>(ps + 4 + 4 * j4));
+        acc.x = fmaf(f, lo.x, acc.x);
+        acc.y = fmaf(f, lo.y, acc.y);
+        acc.z = fmaf(f, hi.x, acc.z);
+        acc.w = fmaf(f, hi.y, acc.w);
+        if (j4 == 0) lsum = fmaf(f, __ldcg(ps + 1), lsum);
+      }
+    }
+    float* dstp = part4 + (g * HG + r) * D + 4 * j4;
+    dstp[0] = acc.x;
+    dstp[1] = acc.y;
+    dstp[2] = acc.z;
+    dstp[3] = acc.w;
+    if (j4 == 0) ls4[g * HG + r] = lsum;
+  }
+  __syncthreads();
+  if (tid < nh) {
+    float L = 0.0f;
+    for (int gg = 0; gg < 4; ++gg) L += ls4[gg * HG + tid];
+    Lr[tid] = L;
+  }
+  __syncthreads();
+  for (int r = 0; r < nh; ++r) {
+    const float O = part4[(0 * HG + r) * D + tid] + part4[(1 * HG + r) * D + tid] +
+                    part4[(2 * HG + r) * D + tid] + part4[(3 * HG + r) * D + tid];
+    ob[r * D + tid] = Lr[r] > 0.0f ? O / Lr[r] : 0.0f;
+  }
+  __syncthreads();
+  // o_i = sum_j Pi[j][i] o'_j  (thread i; rows of Pi are read coalesced across threads)
+  float acc[HG];
+#pragma unroll
+  for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
+#pragma unroll 1
+  for (int j0 = 0; j0 < D; j0 += 32) {
+    float pj[32];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) pj[jj] = __ldg(a.Pi + (j0 + jj) * D + tid);
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj)
+#pragma unroll
+      for (int r = 0; r < HG; ++r) acc[r] = fmaf(pj[jj], ob[r * D + j0 + jj], acc[r]);
+  }
+  for (int r = 0; r < nh; ++r) a.out[((int64_t)b * a.Hq + h0 + r) * D + tid] = acc[r];
+}
+
 template <int KB, int VB, bool QJL>
 __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
   using Lay = Layout<KB, VB, QJL>;
@@ -312,6 +441,9 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
     lutV[i] = pack_half2(a.vc[e & ((1 << VB) - 1)], a.vc[e >> VB]);
   }
 
+  // Everything above reads only the cache; the rotated queries come from the prep kernel.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+
   // A fragments: rows 0-7 = hi parts of the group's heads, rows 8-15 = lo parts (q' and S q').
   uint32_t aq[8][4], asq[8][4];
   {
@@ -346,7 +478,8 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
   float m_run = -INFINITY, l_run = 0.0f;
-  const uint32_t lut_lane = (uint32_t)lane;
+  const uint32_t* lutK_lane = lutK + lane;  // replica of this lane: bank = lane
+  const uint32_t* lutV_lane = lutV + lane;
 
   for (int st = 0; st < nstages; ++st) {
     cp_wait<NSTAGE - 2>();
@@ -375,11 +508,8 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
 #pragma unroll
       for (int i = 0; i < KB; ++i) ck[i] = kw[i];
 #define TQ_KSTEP(KK)                                                                      \
-      {                                                                                   \
-        const uint32_t b0 = lutK[k_pair_index<KB, 2 * (KK)>(ck) * 32 + lut_lane];         \
-        const uint32_t b1 = lutK[k_pair_index<KB, 2 * (KK) + 1>(ck) * 32 + lut_lane];     \
-        mma16816(kacc[nb], aq[KK], b0, b1);                                               \
-      }
+      mma16816(kacc[nb], aq[KK], lutK_lane[k_pair_index<KB, 2 * (KK)>(ck) * 32],          \
+               lutK_lane[k_pair_index<KB, 2 * (KK) + 1>(ck) * 32]);
       TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
 #undef TQ_KSTEP
       if constexpr (QJL) {
@@ -451,12 +581,12 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
       const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gid);
       const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gid);
       const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gid);
+      VPairs<VB> p01, p89;
+      p01.build(cv0, cv1);
+      p89.build(cv2, cv3);
 #define TQ_VSTEP(NU)                                                                        \
-      {                                                                                     \
-        const uint32_t e0 = v_code<VB, NU>(cv0) | (v_code<VB, NU>(cv1) << VB);              \
-        const uint32_t e1 = v_code<VB, NU>(cv2) | (v_code<VB, NU>(cv3) << VB);              \
-        mma16816(oacc[NU], ap, lutV[e0 * 32 + lut_lane], lutV[e1 * 32 + lut_lane]);         \
-      }
+      mma16816(oacc[NU], ap, lutV_lane[p01.template index<NU>() * 32],                      \
+               lutV_lane[p89.template index<NU>() * 32]);
       TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3) TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
       TQ_VSTEP(8) TQ_VSTEP(9) TQ_VSTEP(10) TQ_VSTEP(11) TQ_VSTEP(12) TQ_VSTEP(13) TQ_VSTEP(14) TQ_VSTEP(15)
 #undef TQ_VSTEP
@@ -502,31 +632,19 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
       dst[1] = L;
     }
   }
-}
 
-// ------------------------------------------------------------------------------------------ reduce
-
-__global__ void __launch_bounds__(D) reduce_kernel(const float* __restrict__ part, int splits,
-                                                  const float* __restrict__ Pi, float* __restrict__ out) {
-  __shared__ float ob[D];
-  const int bh = blockIdx.x, j = threadIdx.x;
-  const float* p = part + (int64_t)bh * splits * PART;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * PART]);
-  float L = 0.0f, O = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float ms = p[s * PART];
-      const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
-      L += f * p[s * PART + 1];
-      O += f * p[s * PART + 2 + j];
-    }
-  }
-  ob[j] = L > 0.0f ? O / L : 0.0f;
+  // ---- the last CTA of this (batch, kv-head, head group) merges all splits and un-rotates ----
+  __shared__ int s_last;
+  __threadfence();
   __syncthreads();
-  float acc = 0.0f;  // o_i = sum_j Pi[j][i] o'_j
-  for (int jj = 0; jj < D; ++jj) acc = fmaf(Pi[jj * D + j], ob[jj], acc);
-  out[(int64_t)bh * D + j] = acc;
+  if (tid == 0) {
+    const int unit = (b * a.Hkv + kvh) * a.hgroups + hg;
+    s_last = atomicAdd(&a.counters[unit], 1) == a.splits - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  merge_splits(a, b, h0, nh, pipe);
 }
 
 // ------------------------------------------------------------------------------------------ host
@@ -558,8 +676,9 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
     p.tps = STAGE_TOK;
     return p;
   }
-  const int64_t target = 4LL * sms;  // 2 resident CTAs per SM, two waves
-  int64_t splits = (target + units - 1) / units;
+  // One wave of 2 resident CTAs per SM: the largest split count whose grid still fits it.
+  const int64_t slots = 2LL * sms;
+  int64_t splits = slots / units;
   const int64_t max_splits = (seq_len + 4 * STAGE_TOK - 1) / (4 * STAGE_TOK);  // >= 4 stages each
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
@@ -570,8 +689,11 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
   return p;
 }
 
-size_t workspace_bytes(int B, int Hq, const Plan& p) {
-  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART);
+// Workspace: q' and S q' [B*Hq][128] fp32, split partials [B*Hq][splits][130] fp32, then one
+// completion counter per (batch, kv-head, head group).
+size_t workspace_bytes(int B, int Hq, int Hkv, const Plan& p) {
+  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART) +
+         sizeof(int) * (size_t)B * Hkv * p.hgroups;
 }
 
 template <int KB, int VB, bool QJL>
@@ -580,7 +702,19 @@ tq_status launch_split(const DArgs& a, dim3 grid, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
-  split_kernel<KB, VB, QJL><<<grid, THREADS, Lay::SMEM, stream>>>(a);
+  // programmatic dependent launch: the prologue (tables, first cache stages) overlaps prep
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Lay::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL>, a);
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "split launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
 
@@ -609,7 +743,7 @@ extern "C" size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache,
   using namespace tq;
   if (!cache || B < 1 || Hq < 1 || cache->Hkv < 1 || Hq % cache->Hkv || seq_len < 0) return 0;
   const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
-  return workspace_bytes(B, Hq, p);
+  return workspace_bytes(B, Hq, cache->Hkv, p);
 }
 
 extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, int Hq,
@@ -630,7 +764,7 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
     return fail(TQ_ERR_INVALID_ARG, "q / out / workspace must be 16-byte aligned");
   const int B = cache->B;
   const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
-  const size_t need = workspace_bytes(B, Hq, plan);
+  const size_t need = workspace_bytes(B, Hq, cache->Hkv, plan);
   if (ws_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
 
@@ -663,15 +797,18 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   const int BH = B * Hq;
-  const int prep_grid = (BH + HG - 1) / HG;
+  const int n_counters = B * cache->Hkv * plan.hgroups;
+  a.counters = reinterpret_cast<int*>(ws + (size_t)2 * BH * D + (size_t)BH * plan.splits * PART);
+  a.Pi = params->Pi;
+  a.out = out;
   if (q_dtype == TQ_F32)
-    prep_kernel<float><<<prep_grid, D, 0, s>>>(reinterpret_cast<const float*>(q), params->Pi,
-                                              params->S, BH, cache->qjl_m ? 1 : 0, ws,
-                                              ws + (size_t)BH * D);
+    prep_kernel<float><<<BH, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), params->Pi, params->S,
+                                        cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D, a.counters,
+                                        n_counters);
   else
-    prep_kernel<__nv_bfloat16><<<prep_grid, D, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(q),
-                                                      params->Pi, params->S, BH, cache->qjl_m ? 1 : 0,
-                                                      ws, ws + (size_t)BH * D);
+    prep_kernel<__nv_bfloat16><<<BH, PREP_THREADS, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(q), params->Pi,
+                                                params->S, cache->qjl_m ? 1 : 0, ws,
+                                                ws + (size_t)BH * D, a.counters, n_counters);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
 
@@ -679,12 +816,6 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, a, grid, s)
                     : dispatch<false>(cache->k_bits, cache->v_bits, a, grid, s);
   if (st != TQ_OK) return st;
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "split launch: %s", cudaGetErrorString(e));
-
-  reduce_kernel<<<BH, D, 0, s>>>(a.part, plan.splits, params->Pi, out);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
 
