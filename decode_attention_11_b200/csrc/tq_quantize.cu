@@ -38,13 +38,14 @@ using namespace sm100;
 
 constexpr int D = kHeadDim;
 constexpr int TM = 128;          // tokens per tile (MMA M)
-constexpr int THREADS = 256;     // warpgroup 0: keys, warpgroup 1: values and signs
+constexpr int THREADS = 512;     // 16 warps: each epilogue thread owns one 32-coordinate chunk
 constexpr int TILE_BYTES = TM * D * 2;  // one fp16 [128 x 128] operand
 constexpr uint32_t IDESC = idesc_f16_f32(128, 128);
 constexpr uint32_t TMEM_COLS = 512;
 // Tensor-memory columns: Y_K, Y_V and S rho (fp32, 128 each), rho hi / lo (fp16 pairs, 64 each).
 constexpr uint32_t COL_K = 0, COL_V = 128, COL_S = 256, COL_RH = 384, COL_RL = 448;
 constexpr long long WAIT_LIMIT = 4000000000LL;  // ~2 s of SM clock
+constexpr float PI_SCALE = 256.0f;
 
 // Fast-path guard bands (normalized units): a value closer than this to a decision boundary is
 // re-derived in fp64.
@@ -93,12 +94,13 @@ struct __align__(1024) Smem {
   uint8_t sst[TM * 16];     // sign bits
   float kn[TM], vn[TM], rn[TM];
   double nrmk[TM], nrmv[TM];
-  float rho2[TM];
+  float sclk[TM], sclv[TM];  // u = y * scl (0 for a zero row)
+  float rho2[4][TM];         // ||rho||^2 partials of the four 32-coordinate chunks
   uint16_t fl[FL_CAP];      // deferred fixups: bit 15 = value side, bits 14..7 row, 6..0 coordinate
-  uint8_t vflag[TM];        // key row queued for the fp64 vector path
+  unsigned int vflag[TM];   // bit 0: key vector to fp64 path; bit 1: key list overflow; bit 2: value
   uint8_t vfl[TM];
   double fx64[D];           // exact residual of one vector (vector path)
-  double red64[8];
+  double red64[THREADS / 32];
   float kcent[16], kthr[16], vcent[16], vthr[16];
   uint8_t fcode[D];
   uint8_t fsign[D];
@@ -119,14 +121,26 @@ __device__ __forceinline__ uint64_t desc_at(const uint8_t* tile, int kstep) {
   return desc_sw128_kmajor(smem_u32(tile) + (kstep >> 2) * (TM * 128) + (kstep & 3) * 32);
 }
 
-// Load a row-major fp32 [128 x 128] matrix into an fp16 hi (+ optional lo) operand tile.
-__device__ void load_matrix(const float* M, uint8_t* hi, uint8_t* lo) {
-  for (int i = threadIdx.x; i < D * D; i += THREADS) {
-    const int r = i / D, k = i % D;
-    const float x = M[i];
-    const __half h = __float2half_rn(x);
-    *reinterpret_cast<__half*>(hi + sw_off(r, k)) = h;
-    if (lo) *reinterpret_cast<__half*>(lo + sw_off(r, k)) = __float2half_rn(x - __half2float(h));
+// Load a row-major fp32 [128 x 128] matrix, times `scale` (a power of two), into an fp16 hi
+// (+ optional lo) operand tile, one 16-byte chunk (8 consecutive elements of a row) per step.
+__device__ void load_matrix(const float* __restrict__ M, float scale, uint8_t* hi, uint8_t* lo) {
+  for (int i = threadIdx.x; i < D * D / 8; i += THREADS) {
+    const int r = i / 16, c = i % 16;
+    const float4 p0 = reinterpret_cast<const float4*>(M + r * D + 8 * c)[0];
+    const float4 p1 = reinterpret_cast<const float4*>(M + r * D + 8 * c)[1];
+    const float v[8] = {p0.x * scale, p0.y * scale, p0.z * scale, p0.w * scale,
+                        p1.x * scale, p1.y * scale, p1.z * scale, p1.w * scale};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2 hh = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+      const float2 hf = __half22float2(hh);
+      const __half2 ll = __floats2half2_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+      h[e] = *reinterpret_cast<const uint32_t*>(&hh);
+      l[e] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+    *reinterpret_cast<uint4*>(hi + sw_chunk(r, c)) = make_uint4(h[0], h[1], h[2], h[3]);
+    if (lo) *reinterpret_cast<uint4*>(lo + sw_chunk(r, c)) = make_uint4(l[0], l[1], l[2], l[3]);
   }
 }
 
@@ -154,31 +168,51 @@ __device__ __forceinline__ int search_pos(float a, const float* T, float& margin
   }
 }
 
-// Exact (fp64) rotated coordinate j of input row x (global memory, original dtype).
+// Part q (0..3) of the exact (fp64) dot product of Pi row j with input row x: elements
+// 32q..32q+31, all loads issued at once.  Four consecutive lanes form the whole sum (quad_sum).
 template <typename InT>
-__device__ __noinline__ double exact_u(const float* __restrict__ Pi, const InT* __restrict__ x,
-                                       int j, double n) {
-  double y0 = 0.0, y1 = 0.0, y2 = 0.0, y3 = 0.0;
-  const float4* pr = reinterpret_cast<const float4*>(Pi + j * D);
-#pragma unroll 8
-  for (int k4 = 0; k4 < D / 4; ++k4) {
-    float xv[4];
-    if constexpr (sizeof(InT) == 4) {
-      const float4 q = reinterpret_cast<const float4*>(x)[k4];
-      xv[0] = q.x; xv[1] = q.y; xv[2] = q.z; xv[3] = q.w;
-    } else {
-      const uint2 q = reinterpret_cast<const uint2*>(x)[k4];
-      const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-      const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
-      xv[0] = f0.x; xv[1] = f0.y; xv[2] = f1.x; xv[3] = f1.y;
+__device__ __forceinline__ double exact_dot_part(const float* __restrict__ Pi, const InT* __restrict__ x,
+                                                 int j, int q) {
+  const float4* pr = reinterpret_cast<const float4*>(Pi + j * D + 32 * q);
+  float4 p[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) p[c] = pr[c];
+  float xv[32];
+  if constexpr (sizeof(InT) == 4) {
+    const float4* xr = reinterpret_cast<const float4*>(x + 32 * q);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 t = xr[c];
+      xv[4 * c] = t.x; xv[4 * c + 1] = t.y; xv[4 * c + 2] = t.z; xv[4 * c + 3] = t.w;
     }
-    const float4 p = pr[k4];
-    y0 = fma((double)p.x, (double)xv[0], y0);
-    y1 = fma((double)p.y, (double)xv[1], y1);
-    y2 = fma((double)p.z, (double)xv[2], y2);
-    y3 = fma((double)p.w, (double)xv[3], y3);
+  } else {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + 32 * q);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 t = xr[c];
+      const uint32_t w4[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+        xv[8 * c + 2 * e] = f.x;
+        xv[8 * c + 2 * e + 1] = f.y;
+      }
+    }
   }
-  return sqrt((double)D) * ((y0 + y1) + (y2 + y3)) / n;
+  double y0 = 0.0, y1 = 0.0;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    y0 = fma((double)p[c].x, (double)xv[4 * c + 0], y0);
+    y1 = fma((double)p[c].y, (double)xv[4 * c + 1], y1);
+    y0 = fma((double)p[c].z, (double)xv[4 * c + 2], y0);
+    y1 = fma((double)p[c].w, (double)xv[4 * c + 3], y1);
+  }
+  return y0 + y1;
+}
+__device__ __forceinline__ double quad_sum(double v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
 }
 
 __device__ __forceinline__ int code_exact(double u, const float* thr, int nthr) {
@@ -255,8 +289,10 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int wg = tid >> 7;       // 0: keys, 1: values + signs
-  const int r = tid & 127;       // tile row = TMEM lane
+  // conversion: two threads per input row (K rows 0..127, V rows 128..255), 8 chunks each
+  const int crow = tid >> 1, cwhich = crow >> 7, cr = crow & 127, chalf = tid & 1;
+  // epilogues: thread = (tile row r = TMEM lane, 32-coordinate chunk ch)
+  const int r = tid & 127, ch = tid >> 7;
   constexpr int LK = 1 << KB, LV = 1 << VB;
 
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // operand tiles need 1024-byte alignment
@@ -278,8 +314,10 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   if (tid < LV) s.vcent[tid] = a.vc[tid];
   if (tid < LV - 1) s.vthr[tid] = a.vt[tid];
   if (tid < TM) s.vflag[tid] = 0;
-  load_matrix(a.Pi, s.pih, s.pil);
-  if (a.qjl) load_matrix(a.S, s.sm, nullptr);
+  // Pi enters as 2^8 Pi so that its fp16 lo part stays clear of the subnormal range (the hi + lo
+  // pair then carries ~22 significant bits of every entry); the 2^-8 is folded into u's scale.
+  load_matrix(a.Pi, PI_SCALE, s.pih, s.pil);
+  if (a.qjl) load_matrix(a.S, 1.0f, s.sm, nullptr);
 
   const int tiles_per_bh = (a.T_new + TM - 1) / TM;
   const int64_t total = (int64_t)a.B * a.Hkv * tiles_per_bh;
@@ -300,7 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // == (r & ~31) << 16
   // positive thresholds: T[j] = t[L/2 - 1 + j] (T[0] = 0)
   float TK[8], TV[8];
 #pragma unroll
@@ -315,53 +353,68 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
     tile_coords(tile, b, h, t0, nt);
     const int64_t row0 = ((int64_t)b * a.Hkv + h) * a.T_cap + a.t_offset + t0;
     const int64_t in_base = (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)t0 * a.st;
-    const InT* xrow = reinterpret_cast<const InT*>(wg == 0 ? a.k : a.v) + in_base + (int64_t)r * a.st;
     const bool live = r < nt;
 
-    // ---- 1. operands ready; convert this thread's row in place to fp16, norm in fp64 ----
-    // Codes depend only on the direction of x, so the row is scaled by 2^e (exact) to bring its
+    // ---- 1. operands ready; convert rows in place to fp16, norms in fp64 ----
+    // Codes depend only on the direction of x, so each row is scaled by 2^e (exact) to bring its
     // largest element to [2^14, 2^15) before the fp16 conversion; the stored norm is unscaled.
-    uint8_t* xt = wg == 0 ? s.xk : s.xv;
-    if constexpr (sizeof(InT) != 4) {
-      cp_async_wait_all();
-      __syncthreads();
-    }
-    double acc = 0.0;
-    float amax = 0.0f;
+    {
+      const InT* xrow = reinterpret_cast<const InT*>(cwhich == 0 ? a.k : a.v) + in_base + (int64_t)cr * a.st;
+      const bool clive = cr < nt;
+      uint8_t* xt = cwhich == 0 ? s.xk : s.xv;
+      if constexpr (sizeof(InT) != 4) {
+        cp_async_wait_all();
+        __syncthreads();
+      }
+      double acc = 0.0;
+      float amax = 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < 16; ++c) {
-      float v8[8];
-      row_chunk<InT>(xrow, xt, r, c, live, v8);
+      for (int c = 8 * chalf; c < 8 * chalf + 8; ++c) {
+        float v8[8];
+        row_chunk<InT>(xrow, xt, cr, c, clive, v8);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        acc = fma((double)v8[i], (double)v8[i], acc);
-        amax = fmaxf(amax, fabsf(v8[i]));
+        for (int i = 0; i < 8; ++i) {
+          acc = fma((double)v8[i], (double)v8[i], acc);
+          amax = fmaxf(amax, fabsf(v8[i]));
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      int ex = 0;
+      frexpf(amax, &ex);
+      const int e = amax > 0.0f ? max(-126, min(127, 15 - ex)) : 0;
+      const float p2 = __int_as_float((e + 127) << 23);  // 2^e
+#pragma unroll 1
+      for (int c = 8 * chalf; c < 8 * chalf + 8; ++c) {
+        float v8[8];
+        row_chunk<InT>(xrow, xt, cr, c, clive, v8);
+        uint32_t o[4], ol[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float x0 = v8[2 * i] * p2, x1 = v8[2 * i + 1] * p2;
+          const __half2 hh = __floats2half2_rn(x0, x1);
+          o[i] = *reinterpret_cast<const uint32_t*>(&hh);
+          if constexpr (sizeof(InT) == 4) {
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+            ol[i] = *reinterpret_cast<const uint32_t*>(&ll);
+          }
+        }
+        *reinterpret_cast<uint4*>(xt + sw_chunk(cr, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+        if constexpr (sizeof(InT) == 4)
+          if (cwhich == 0) *reinterpret_cast<uint4*>(s.xl + sw_chunk(cr, c)) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+      }
+      if (chalf == 0) {
+        const double n = sqrt(acc);
+        (cwhich == 0 ? s.nrmk : s.nrmv)[cr] = n;
+        (cwhich == 0 ? s.sclk : s.sclv)[cr] =
+            n > 0.0 ? (float)(sqrt((double)D) / (n * (double)p2 * (double)PI_SCALE)) : 0.0f;
       }
     }
-    int ex = 0;
-    frexpf(amax, &ex);
-    const int e = amax > 0.0f ? max(-126, min(127, 15 - ex)) : 0;
-    const float p2 = __int_as_float((e + 127) << 23);  // 2^e
-#pragma unroll 1
-    for (int c = 0; c < 16; ++c) {
-      float v8[8];
-      row_chunk<InT>(xrow, xt, r, c, live, v8);
-      uint32_t o[4], ol[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float x0 = v8[2 * i] * p2, x1 = v8[2 * i + 1] * p2;
-        const __half2 hh = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(hh);
-        const __half2 ll = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
-        o[i] = *reinterpret_cast<const uint32_t*>(&hh);
-        ol[i] = *reinterpret_cast<const uint32_t*>(&ll);
-      }
-      *reinterpret_cast<uint4*>(xt + sw_chunk(r, c)) = make_uint4(o[0], o[1], o[2], o[3]);
-      if (sizeof(InT) == 4 && wg == 0)
-        *reinterpret_cast<uint4*>(s.xl + sw_chunk(r, c)) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-    }
-    const double n = sqrt(acc);
-    (wg == 0 ? s.nrmk : s.nrmv)[r] = n;
+    // sign rows (and 3-bit value rows) are assembled with shared-memory atomics: clear them
+    for (int i = tid; i < TM * 4; i += THREADS) reinterpret_cast<uint32_t*>(s.sst)[i] = 0u;
+    if constexpr (VB == 3)
+      for (int i = tid; i < TM * 12; i += THREADS) reinterpret_cast<uint32_t*>(s.vst)[i] = 0u;
     if (tid == 0) {
       s.nfl = 0;
       s.nvfl = 0;
@@ -393,122 +446,120 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
       tile_coords(tile + gridDim.x, b2, h2, t02, nt2);
       issue_x_loads<InT>(s, a, b2, h2, t02, nt2);
     }
-    const float scl = n > 0.0 ? (float)(sqrt((double)D) / (n * (double)p2)) : 0.0f;
-    const bool zero = !(n > 0.0);
 
-    if (wg == 0) {
-      // ---- 3a. keys: codes, residual rho (fp16 hi + lo into tensor memory), ||rho||^2 ----
-      // Chunk ch holds coordinates 32ch + i.  Its codes occupy, for each tau, the 8 consecutive
-      // slots 32 tau + 8 ch + q of coordinates 32ch + 2 tau + {0,1,8,9,16,17,24,25}[q]: one
-      // byte-aligned field of 8 * k_bits bits.
+    // ---- 3a. keys: codes, residual rho (fp16 hi + lo into tensor memory), ||rho||^2 ----
+    // Chunk ch holds coordinates 32ch + i; for each tau its codes fill the 8 consecutive slots
+    // 32 tau + 8 ch + q of coordinates 32ch + 2 tau + {0,1,8,9,16,17,24,25}[q]: one
+    // byte-aligned field of 8 * k_bits bits at byte k_bits * (4 tau + ch).
+    {
+      const float scl = s.sclk[r];
+      const bool zero = scl == 0.0f;
       uint8_t* krow = s.kst + r * (16 * KB);
       float r2 = 0.0f;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t yr[32];
-        tmem_ld32(tmem + lane_base + COL_K + 32 * ch, yr);
-        tmem_wait_ld();
-        uint32_t hi[16], lo[16];
-        uint32_t fld[4] = {0u, 0u, 0u, 0u};
+      uint32_t yr[32];
+      tmem_ld32(tmem + lane_base + COL_K + 32 * ch, yr);
+      tmem_wait_ld();
+      uint32_t hi[16], lo[16];
+      uint32_t fld[4] = {0u, 0u, 0u, 0u};
+      uint32_t near = 0u;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float rr[2];
+      for (int i = 0; i < 32; i += 2) {
+        float rr[2];
 #pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int ii = i + e2;
-            const float u = __uint_as_float(yr[ii]) * scl;
-            const float aa = fabsf(u);
-            float margin;
-            const int kpos = search_pos<KB>(aa, TK, margin);
-            int idx = zero ? LK / 2 : (u >= 0.0f ? LK / 2 + kpos : LK / 2 - 1 - kpos);
-            float rho = u - s.kcent[idx];
-            if (fminf(margin, aa) < a.guard.code_k && live && !zero) {
-              const int slot = atomicAdd(&s.nfl, 1);
-              if (slot < FL_CAP) {
-                s.fl[slot] = (uint16_t)((r << 7) | (32 * ch + ii));
-              } else {  // list full: re-derive here
-                const double ud = exact_u<InT>(a.Pi, xrow, 32 * ch + ii, n);
-                idx = code_exact(ud, s.kthr, LK - 1);
-                rho = (float)(ud - (double)s.kcent[idx]);
-              }
-            }
-            rr[e2] = rho;
-            r2 = fmaf(rho, rho, r2);
-            const int tau = (ii & 7) >> 1, q = ((ii >> 4) << 2) | (((ii >> 3) & 1) << 1) | (ii & 1);
-            fld[tau] |= (uint32_t)idx << (KB * q);
-          }
-          const __half2 hh = __floats2half2_rn(rr[0], rr[1]);
-          const float2 hf = __half22float2(hh);
-          const __half2 ll = __floats2half2_rn(rr[0] - hf.x, rr[1] - hf.y);
-          hi[i / 2] = *reinterpret_cast<const uint32_t*>(&hh);
-          lo[i / 2] = *reinterpret_cast<const uint32_t*>(&ll);
-        }
-#pragma unroll
-        for (int tau = 0; tau < 4; ++tau) {
-          uint8_t* dst = krow + KB * (4 * tau + ch);
-          if constexpr (KB == 4) {
-            *reinterpret_cast<uint32_t*>(dst) = fld[tau];
-          } else if constexpr (KB == 2) {
-            *reinterpret_cast<uint16_t*>(dst) = (uint16_t)fld[tau];
-          } else {
-            dst[0] = (uint8_t)fld[tau];
-            dst[1] = (uint8_t)(fld[tau] >> 8);
-            dst[2] = (uint8_t)(fld[tau] >> 16);
-          }
-        }
-        if (a.qjl) {
-          tmem_st16(tmem + lane_base + COL_RH + 16 * ch, hi);
-          tmem_st16(tmem + lane_base + COL_RL + 16 * ch, lo);
-        }
-      }
-      if (a.qjl) tmem_wait_st();
-      s.kn[r] = (float)n;
-      s.rho2[r] = r2;
-    } else {
-      // ---- 3b. values: codes.  Coordinate 32ch + i sits at slot 16 (i % 8) + 4 ch + i / 8. ----
-      uint64_t acc64[8];
-#pragma unroll
-      for (int g = 0; g < 8; ++g) acc64[g] = 0ull;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t yr[32];
-        tmem_ld32(tmem + lane_base + COL_V + 32 * ch, yr);
-        tmem_wait_ld();
-        uint32_t fld[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float u = __uint_as_float(yr[i]) * scl;
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const int ii = i + e2;
+          const float u = __uint_as_float(yr[ii]) * scl;
           const float aa = fabsf(u);
           float margin;
-          const int kpos = search_pos<VB>(aa, TV, margin);
-          int idx = zero ? LV / 2 : (u >= 0.0f ? LV / 2 + kpos : LV / 2 - 1 - kpos);
-          if (fminf(margin, aa) < a.guard.code_v && live && !zero) {
-            const int slot = atomicAdd(&s.nfl, 1);
-            if (slot < FL_CAP)
-              s.fl[slot] = (uint16_t)(0x8000u | (r << 7) | (32 * ch + i));
-            else
-              idx = code_exact(exact_u<InT>(a.Pi, xrow, 32 * ch + i, n), s.vthr, LV - 1);
-          }
-          fld[i & 7] |= (uint32_t)idx << (VB * (i >> 3));
+          const int kpos = search_pos<KB>(aa, TK, margin);
+          const int idx = zero ? LK / 2 : (u >= 0.0f ? LK / 2 + kpos : LK / 2 - 1 - kpos);
+          const float rho = u - s.kcent[idx];
+          near |= (fminf(margin, aa) < a.guard.code_k ? 1u : 0u) << ii;
+          rr[e2] = rho;
+          r2 = fmaf(rho, rho, r2);
+          const int tau = (ii & 7) >> 1, q = ((ii >> 4) << 2) | (((ii >> 3) & 1) << 1) | (ii & 1);
+          fld[tau] |= (uint32_t)idx << (KB * q);
         }
+        const __half2 hh = __floats2half2_rn(rr[0], rr[1]);
+        const float2 hf = __half22float2(hh);
+        const __half2 ll = __floats2half2_rn(rr[0] - hf.x, rr[1] - hf.y);
+        hi[i / 2] = *reinterpret_cast<const uint32_t*>(&hh);
+        lo[i / 2] = *reinterpret_cast<const uint32_t*>(&ll);
+      }
 #pragma unroll
-        for (int g = 0; g < 8; ++g) acc64[g] |= (uint64_t)fld[g] << (4 * VB * ch);
+      for (int tau = 0; tau < 4; ++tau) {
+        uint8_t* dst = krow + KB * (4 * tau + ch);
+        if constexpr (KB == 4) {
+          *reinterpret_cast<uint32_t*>(dst) = fld[tau];
+        } else if constexpr (KB == 2) {
+          *reinterpret_cast<uint16_t*>(dst) = (uint16_t)fld[tau];
+        } else {
+          dst[0] = (uint8_t)fld[tau];
+          dst[1] = (uint8_t)(fld[tau] >> 8);
+          dst[2] = (uint8_t)(fld[tau] >> 16);
+        }
+      }
+      if (a.qjl) {
+        tmem_st16(tmem + lane_base + COL_RH + 16 * ch, hi);
+        tmem_st16(tmem + lane_base + COL_RL + 16 * ch, lo);
+        tmem_wait_st();
+      }
+      s.rho2[ch][r] = r2;
+      if (!(live && !zero)) near = 0u;
+      while (near) {  // queue coordinates near a threshold for the fp64 pass
+        const int ii = __ffs(near) - 1;
+        near &= near - 1;
+        const int slot = atomicAdd(&s.nfl, 1);
+        if (slot < FL_CAP) s.fl[slot] = (uint16_t)((r << 7) | (32 * ch + ii));
+        else atomicOr(&s.vflag[r], 2u);  // list full: the key row takes the fp64 vector path
+      }
+    }
+    // ---- 3b. values: codes.  Coordinate 32ch + i sits at slot 16 (i % 8) + 4 ch + i / 8: chunk ch
+    //          gives lane group g a field of 4 codes at bit v_bits (16 g + 4 ch). ----
+    {
+      const float scl = s.sclv[r];
+      const bool zero = scl == 0.0f;
+      uint32_t yr[32];
+      tmem_ld32(tmem + lane_base + COL_V + 32 * ch, yr);
+      tmem_wait_ld();
+      uint32_t near = 0u;
+      uint32_t f8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float u = __uint_as_float(yr[i]) * scl;
+        const float aa = fabsf(u);
+        float margin;
+        const int kpos = search_pos<VB>(aa, TV, margin);
+        const int idx = zero ? LV / 2 : (u >= 0.0f ? LV / 2 + kpos : LV / 2 - 1 - kpos);
+        near |= (fminf(margin, aa) < a.guard.code_v ? 1u : 0u) << i;
+        f8[i & 7] |= (uint32_t)idx << (VB * (i >> 3));
       }
       uint8_t* vrow = s.vst + r * (16 * VB);
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {  // 16 codes of lane group g: 2 * VB bytes at byte 2 * VB * g
+      for (int g = 0; g < 8; ++g) {
         if constexpr (VB == 4) {
-          reinterpret_cast<uint2*>(vrow)[g] = make_uint2((uint32_t)acc64[g], (uint32_t)(acc64[g] >> 32));
+          *reinterpret_cast<uint16_t*>(vrow + 8 * g + 2 * ch) = (uint16_t)f8[g];
         } else if constexpr (VB == 2) {
-          reinterpret_cast<uint32_t*>(vrow)[g] = (uint32_t)acc64[g];
+          vrow[4 * g + ch] = (uint8_t)f8[g];
         } else {
-          uint16_t* d16 = reinterpret_cast<uint16_t*>(vrow + 6 * g);
-          d16[0] = (uint16_t)acc64[g];
-          d16[1] = (uint16_t)(acc64[g] >> 16);
-          d16[2] = (uint16_t)(acc64[g] >> 32);
+          const int P = 48 * g + 12 * ch;  // 12-bit field: may straddle two words
+          uint32_t* w = reinterpret_cast<uint32_t*>(vrow);
+          atomicOr(&w[P >> 5], f8[g] << (P & 31));
+          if ((P & 31) > 20) atomicOr(&w[(P >> 5) + 1], f8[g] >> (32 - (P & 31)));
         }
       }
-      s.vn[r] = (float)n;
+      if (!(live && !zero)) near = 0u;
+      while (near) {
+        const int ii = __ffs(near) - 1;
+        near &= near - 1;
+        const int slot = atomicAdd(&s.nfl, 1);
+        if (slot < FL_CAP) s.fl[slot] = (uint16_t)(0x8000u | (r << 7) | (32 * ch + ii));
+        else atomicOr(&s.vflag[r], 4u);  // list full: this value row is re-derived whole in fp64
+      }
+    }
+    if (ch == 0) {
+      s.kn[r] = (float)s.nrmk[r];
+      s.vn[r] = (float)s.nrmv[r];
     }
     tc_fence_before();
     __syncthreads();
@@ -524,13 +575,20 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
       umma_commit(&s.bar_s);
     }
     {
+      // four threads per queued coordinate: one fp64 dot product each, one memory round trip
       const int nfl = min(s.nfl, FL_CAP);
-      for (int f = tid; f < nfl; f += THREADS) {
-        const uint32_t ent = s.fl[f];
+      for (int f0 = 0; f0 < nfl; f0 += THREADS / 4) {
+        const int f = f0 + (tid >> 2);
+        const bool have = f < nfl;
+        const uint32_t ent = have ? s.fl[f] : 0u;
         const bool val = ent & 0x8000u;
         const int rr = (ent >> 7) & 127, j = ent & 127;
         const InT* x = reinterpret_cast<const InT*>(val ? a.v : a.k) + in_base + (int64_t)rr * a.st;
-        const double ud = exact_u<InT>(a.Pi, x, j, val ? s.nrmv[rr] : s.nrmk[rr]);
+        const double part = have ? exact_dot_part<InT>(a.Pi, x, j, tid & 3) : 0.0;
+        const double dot = quad_sum(part);  // all lanes take part in the shuffle
+        if (!have || (tid & 3)) continue;
+        const double nn = val ? s.nrmv[rr] : s.nrmk[rr];
+        const double ud = sqrt((double)D) * dot / nn;
         if (val) {
           const uint32_t idx = (uint32_t)code_exact(ud, s.vthr, LV - 1);
           uint8_t* row = s.vst + rr * (16 * VB);
@@ -541,84 +599,111 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
           if (get_code(row, KB, k_slot_of_coord(j)) != idx) {
             set_code(row, KB, k_slot_of_coord(j), idx);
             // the residual fed to the sketch came from the other cell: redo the vector in fp64
-            if (a.qjl) s.vflag[rr] = 1;
+            if (a.qjl) atomicOr(&s.vflag[rr], 1u);
           }
         }
       }
       if (tid == 0 && s.nfl) atomicAdd(&g_quantize_code_fixups, (unsigned)min(s.nfl, FL_CAP));
     }
-
     if (a.qjl) {
-      if (wg == 1) {
-        if (!mbar_wait(&s.bar_s, phase, WAIT_LIMIT)) s.err = 1;
-        tc_fence_after();
-        uint32_t sw[4] = {0u, 0u, 0u, 0u};
-        bool flagged = false;
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t yr[32];
-          tmem_ld32(tmem + lane_base + COL_S + 32 * ch, yr);
-          tmem_wait_ld();
-          // sketch row l = 32ch + i = 16 kap + 8 h + 2 tau + e sits at bit 32 tau + (2 kap + h) + 16 e;
-          // within the chunk, kap - 2ch and h give 4ch + (0..3)
-          uint32_t nib[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // [tau][e]
+      if (!mbar_wait(&s.bar_s, phase, WAIT_LIMIT)) s.err = 1;
+      tc_fence_after();
+      // sketch row l = 32ch + i = 16 kap + 8 h + 2 tau + e sits at row bit 32 tau + (2 kap + h)
+      // + 16 e; chunk ch fills, for each tau and e, the nibble at bit 32 tau + 16 e + 4 ch.
+      uint32_t yr[32];
+      tmem_ld32(tmem + lane_base + COL_S + 32 * ch, yr);
+      tmem_wait_ld();
+      uint32_t nib[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // [tau][e]
+      bool flagged = false;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float sp = __uint_as_float(yr[i]);
-            const int tau = (i >> 1) & 3, e2 = i & 1, p = ((i >> 4) << 1) | ((i >> 3) & 1);
-            nib[2 * tau + e2] |= (sp >= 0.0f ? 1u : 0u) << p;
-            flagged |= fabsf(sp) < a.guard.sign;
-          }
+      for (int i = 0; i < 32; ++i) {
+        const float sp = __uint_as_float(yr[i]);
+        const int tau = (i >> 1) & 3, e2 = i & 1, pp = ((i >> 4) << 1) | ((i >> 3) & 1);
+        nib[2 * tau + e2] |= (sp >= 0.0f ? 1u : 0u) << pp;
+        flagged |= fabsf(sp) < a.guard.sign;
+      }
+      uint32_t* srow = reinterpret_cast<uint32_t*>(s.sst + r * 16);
 #pragma unroll
-          for (int tau = 0; tau < 4; ++tau) sw[tau] |= (nib[2 * tau] << (4 * ch)) | (nib[2 * tau + 1] << (16 + 4 * ch));
-        }
-        *reinterpret_cast<uint4*>(s.sst + r * 16) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-        s.rn[r] = (float)(s.nrmk[r] * sqrt((double)s.rho2[r]) / sqrt((double)D));
-        if (flagged && live) s.vflag[r] = 1;
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (s.err) break;
-      if (tid < TM && s.vflag[tid]) {
-        s.vfl[atomicAdd(&s.nvfl, 1)] = (uint8_t)tid;
-        s.vflag[tid] = 0;
-      }
-      __syncthreads();
+      for (int tau = 0; tau < 4; ++tau)
+        atomicOr(&srow[tau], (nib[2 * tau] << (4 * ch)) | (nib[2 * tau + 1] << (16 + 4 * ch)));
+      if (flagged && live) atomicOr(&s.vflag[r], 1u);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (s.err) break;
+    if (tid < TM) {
+      if (a.qjl)
+        s.rn[tid] = (float)(s.nrmk[tid] * sqrt((double)(s.rho2[0][tid] + s.rho2[1][tid] + s.rho2[2][tid] +
+                                                        s.rho2[3][tid])) / sqrt((double)D));
+      if (s.vflag[tid]) s.vfl[atomicAdd(&s.nvfl, 1)] = (uint8_t)tid;
+    }
+    __syncthreads();
 
-      // ---- 5. key vectors with a sketch value near 0 (or a corrected code): fp64 vector path ----
+    // ---- 5. rows re-derived whole in fp64: key vectors with a sketch value near 0 or a corrected
+    //         code, and rows whose near-threshold list overflowed ----
+    {
       const int nvf = s.nvfl;
       for (int f = 0; f < nvf; ++f) {
         const int rr = s.vfl[f];
+        const unsigned int fl = s.vflag[rr];
+        if (fl & 4) {  // value row
+          const double nv = s.nrmv[rr];
+          const InT* vx = reinterpret_cast<const InT*>(a.v) + in_base + (int64_t)rr * a.st;
+          {
+            const int j = tid >> 2;
+            const double dot = quad_sum(exact_dot_part<InT>(a.Pi, vx, j, tid & 3));
+            if ((tid & 3) == 0) {
+              const int idx = nv > 0.0 ? code_exact(sqrt((double)D) * dot / nv, s.vthr, LV - 1) : LV / 2;
+              s.fcode[v_slot_of_coord(j)] = (uint8_t)idx;
+            }
+          }
+          __syncthreads();
+          if (tid < 4 * VB) {
+            uint32_t word = 0;
+            for (int kk = 0; kk < 32; ++kk) {
+              const int P = 32 * tid + kk;
+              word |= (uint32_t)((s.fcode[P / VB] >> (P % VB)) & 1) << kk;
+            }
+            reinterpret_cast<uint32_t*>(s.vst + rr * (16 * VB))[tid] = word;
+          }
+          __syncthreads();
+        }
+        if (!(fl & 3)) continue;  // uniform: read from shared memory after a barrier
         const double nk = s.nrmk[rr];
         const InT* kx = reinterpret_cast<const InT*>(a.k) + in_base + (int64_t)rr * a.st;
-        if (tid < D) {
-          const int j = tid;
-          double rho;
-          int idx;
-          if (nk > 0.0) {
-            const double ud = exact_u<InT>(a.Pi, kx, j, nk);
-            idx = code_exact(ud, s.kthr, LK - 1);
-            rho = ud - (double)s.kcent[idx];
-          } else {
-            idx = LK / 2;
-            rho = -(double)s.kcent[idx];
+        {
+          const int j = tid >> 2;
+          const double dot = quad_sum(exact_dot_part<InT>(a.Pi, kx, j, tid & 3));
+          double rho = 0.0;
+          if ((tid & 3) == 0) {
+            int idx;
+            if (nk > 0.0) {
+              const double ud = sqrt((double)D) * dot / nk;
+              idx = code_exact(ud, s.kthr, LK - 1);
+              rho = ud - (double)s.kcent[idx];
+            } else {
+              idx = LK / 2;
+              rho = -(double)s.kcent[idx];
+            }
+            s.fx64[j] = rho;
+            s.fcode[k_slot_of_coord(j)] = (uint8_t)idx;
           }
-          s.fx64[j] = rho;
-          s.fcode[k_slot_of_coord(j)] = (uint8_t)idx;
           double q2 = rho * rho;
           for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xffffffffu, q2, o);
           if ((tid & 31) == 0) s.red64[tid >> 5] = q2;
         }
         __syncthreads();
-        if (tid >= D) {
-          const int l = tid - D;
+        if (a.qjl) {  // (S rho)_l from the exact fp16 copy of S in shared memory
+          const int l = tid >> 2, q = tid & 3;
           double sp0 = 0.0, sp1 = 0.0;
-          const float* srow = a.S + l * D;
-          for (int j = 0; j < D; j += 2) {
-            sp0 = fma((double)srow[j], s.fx64[j], sp0);
-            sp1 = fma((double)srow[j + 1], s.fx64[j + 1], sp1);
+#pragma unroll 8
+          for (int jj = 0; jj < 32; jj += 2) {
+            const int j = 32 * q + jj;
+            sp0 = fma((double)__half2float(*reinterpret_cast<const __half*>(s.sm + sw_off(l, j))), s.fx64[j], sp0);
+            sp1 = fma((double)__half2float(*reinterpret_cast<const __half*>(s.sm + sw_off(l, j + 1))), s.fx64[j + 1], sp1);
           }
-          s.fsign[sign_bit_of_row(l)] = (sp0 + sp1) >= 0.0 ? 1 : 0;
+          const double sp = quad_sum(sp0 + sp1);
+          if (q == 0) s.fsign[sign_bit_of_row(l)] = sp >= 0.0 ? 1 : 0;
         }
         __syncthreads();
         if (tid < 4 * KB) {
@@ -628,20 +713,20 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
             word |= (uint32_t)((s.fcode[P / KB] >> (P % KB)) & 1) << kk;
           }
           reinterpret_cast<uint32_t*>(s.kst + rr * (16 * KB))[tid] = word;
-        } else if (tid >= 32 && tid < 36) {
+        } else if (tid >= 32 && tid < 36 && a.qjl) {
           const int w = tid - 32;
           uint32_t word = 0;
           for (int kk = 0; kk < 32; ++kk) word |= (uint32_t)s.fsign[32 * w + kk] << kk;
           reinterpret_cast<uint32_t*>(s.sst + rr * 16)[w] = word;
-        } else if (tid == 64) {
-          const double q2 = s.red64[0] + s.red64[1] + s.red64[2] + s.red64[3];
+        } else if (tid == 64 && a.qjl) {
+          double q2 = 0.0;
+          for (int w = 0; w < THREADS / 32; ++w) q2 += s.red64[w];
           s.rn[rr] = (float)(nk * sqrt(q2) / sqrt((double)D));
         }
         __syncthreads();
       }
+      if (tid < TM) s.vflag[tid] = 0;
       if (tid == 0 && nvf) atomicAdd(&g_quantize_vector_fixups, (unsigned)nvf);
-    } else {
-      __syncthreads();
     }
 
     // ---- 6. coalesced stores of the tile's rows ----
