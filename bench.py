@@ -29,6 +29,39 @@ DEFAULT_WORKLOAD = "llama3_8b_32k"
 L2_FLUSH_BYTES = 256 << 20
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+KERNEL_SOURCES = {"tq_quantize": "decode_attention_11_b200/csrc/tq_quantize.cu",
+                  "tq_decode_attn": "decode_attention_11_b200/csrc/tq_decode.cu"}
+
+
+def source_digest(rel: str) -> str:
+    import hashlib
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def dram_traffic(kernel: str, workload: str, batch, context):
+    """DRAM bytes per launch of `kernel` (dram__bytes_read.sum + dram__bytes_write.sum) from a
+    committed ncu capture, scaled by batch to the launch timed here (traffic grows with the number
+    of (sequence, kv-head) units).  None when the kernel source changed since the capture or no
+    capture covers this workload."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture"
+    with open(TRAFFIC_FILE) as f:
+        table = json.load(f)
+    for e in table.get("captures", []):
+        if e["api"] != kernel or e["workload"] != workload or context is not None:
+            continue
+        if source_digest(KERNEL_SOURCES[kernel]) != e["source_sha256"]:
+            return None, "kernel changed since the capture"
+        full_b = W.CONFIGS[workload].B
+        b = batch if batch is not None else full_b
+        per_unit = e["bytes_per_launch"] / e["batch"]
+        note = "ncu capture at batch %d" % e["batch"] + ("" if b == e["batch"] else ", scaled to batch %d" % b)
+        return per_unit * b, note
+    return None, "no capture of this workload"
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -39,56 +72,90 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """SM clock and clock-event reasons sampled through NVML every millisecond while the timed
+    region runs (the region can be a few milliseconds long); nvidia-smi polling if NVML is
+    unavailable."""
 
-    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+             0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.samples = []  # (sm_mhz, sm_max_mhz, reasons bitmask, power_w)
+        self._stop = None
+        self._thread = None
+        self._smi = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device_index)
+        bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+        except Exception:
+            nv = None
+        if nv is not None:
+            self._stop = threading.Event()
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def run():
+                smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax,
+                                             int(get_reasons(h)), nv.nvmlDeviceGetPowerUsage(h) / 1e3))
+                    except Exception:
+                        pass
+                    self._stop.wait(0.001)
+
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+        else:
+            try:
+                self._smi = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.device_index),
+                     "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,power.draw",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self._smi = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._smi is not None:
+            self._smi.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                out, _ = self._smi.communicate(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self._smi.kill()
+                out, _ = self._smi.communicate()
+            for line in out.splitlines():
+                parts = [p.strip() for p in line.split(",")]
+                try:
+                    self.samples.append((float(parts[0]), float(parts[1]), int(parts[2], 16), float(parts[3])))
+                except (ValueError, IndexError):
+                    continue
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+        sm = [x[0] for x in self.samples]
+        reasons = set()
+        for x in self.samples:
+            for bit, name in self.NAMES.items():
+                if x[2] & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "sm_mhz_min": min(sm), "power_w_max": max(x[3] for x in self.samples),
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
@@ -298,8 +365,10 @@ def run_gpu(args, w):
 
     def roof(name, bytes_per_launch, ms):
         achieved = bytes_per_launch / (ms * 1e-3) / 1e9
+        traffic, note = dram_traffic(name, args.workload, args.batch, args.context)
         return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind}
+                "frac": achieved / hbm, "traffic": traffic, "traffic_note": note,
+                "algorithmic_bytes": bytes_per_launch, "peak_kind": peak_kind}
 
     per_launch_q = qnt_bytes / n_chunks
     roof_q = roof("tq_quantize", per_launch_q, (sum(q_ms) / len(q_ms)) / n_chunks)
