@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtq_b200.so")
-SOURCES = ["tq_host.cpp", "tq_quantize.cu", "tq_decode.cu"]
+SOURCES = ["tq_host.cpp", "tq_quantize.cu", "tq_quantize_pipe.cu", "tq_decode.cu"]
 HEADERS = [os.path.join(CSRC, "tq_internal.h"), os.path.join(CSRC, "tq_sm100.h"),
            os.path.join(INCLUDE, "tq.h")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

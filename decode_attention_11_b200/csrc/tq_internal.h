@@ -40,6 +40,15 @@ __host__ __device__ inline int sign_bit_of_row(int l) {
   return 32 * t + (2 * a + h) + 16 * e;
 }
 
+// bf16 quantize pipeline (tq_quantize_pipe.cu).  Sets *handled = false, and enqueues nothing,
+// when the inputs cannot be described by a TMA tensor map.
+tq_status quantize_bf16_pipeline(const tq_params* p, const void* k, const void* v, int64_t sb, int64_t sh,
+                                 int64_t st, int T_new, int t_offset, const tq_cache* c, int sms,
+                                 struct CUstream_st* stream, bool* handled);
+unsigned int pipe_device_errors();
+long long pipe_vector_fixups();
+long long pipe_code_fixups();
+
 // Validation shared by tq_quantize / tq_decode_attn.
 tq_status check_params(const tq_params* p, const tq_cache* c);
 tq_status check_cache(const tq_cache* c);

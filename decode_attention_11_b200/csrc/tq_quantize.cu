@@ -846,6 +846,12 @@ extern "C" tq_status tq_quantize(const tq_params* params, const void* k, const v
   // bands below are >= 4x those.  fp32 values enter as fp16(x) alone (relative 2^-12, ~2e-4 in u).
   a.guard = dtype == TQ_F32 ? Guards{4e-6f, 4e-3f, 3e-5f} : Guards{4e-6f, 4e-6f, 3e-5f};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == TQ_BF16) {
+    bool handled = false;
+    st = quantize_bf16_pipeline(params, k, v, stride_b, stride_h, stride_t, T_new, t_offset, cache, sms, s,
+                                &handled);
+    if (handled || st != TQ_OK) return st;
+  }
   return dtype == TQ_F32 ? launch<float>(cache->k_bits, cache->v_bits, a, sms, s)
                          : launch<__nv_bfloat16>(cache->k_bits, cache->v_bits, a, sms, s);
 }
@@ -853,17 +859,21 @@ extern "C" tq_status tq_quantize(const tq_params* params, const void* k, const v
 extern "C" int tq_quantize_device_errors(void) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, tq::g_quantize_error, sizeof(v)) != cudaSuccess) return -1;
-  return (int)v;
+  const unsigned int p = tq::pipe_device_errors();
+  if (p == 0xffffffffu) return -1;
+  return (int)(v | p);
 }
 
 extern "C" long long tq_quantize_vector_fixups(void) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, tq::g_quantize_vector_fixups, sizeof(v)) != cudaSuccess) return -1;
-  return (long long)v;
+  const long long p = tq::pipe_vector_fixups();
+  return p < 0 ? -1 : (long long)v + p;
 }
 
 extern "C" long long tq_quantize_code_fixups(void) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, tq::g_quantize_code_fixups, sizeof(v)) != cudaSuccess) return -1;
-  return (long long)v;
+  const long long p = tq::pipe_code_fixups();
+  return p < 0 ? -1 : (long long)v + p;
 }

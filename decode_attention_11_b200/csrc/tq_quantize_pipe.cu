@@ -1,0 +1,1246 @@
+// tq_quantize, bf16 inputs: a warp-specialised, TMA-fed pipeline on the sm_100a tensor cores.
+//
+// Method: ai-news.ru TurboQuant overview (random orthogonal rotation, then a Lloyd-Max grid
+// precomputed for the Gaussian, then a 1-bit QJL correction of the residual); tproger.ru
+// "Google TurboQuant in simple words", "Step 1: PolarQuant" (per-coordinate scalar quantizer, no
+// per-group scale) and "Step 2: QJL" (sign bits of a Gaussian projection of the residual).
+//
+// One persistent 512-thread CTA per SM walks 128-token tiles of (batch, kv-head) rows; the stages
+// of consecutive tiles overlap:
+//   warp 12      TMA producer: bf16 K and V tiles into a 3-slot ring (128-byte swizzle, the
+//                UMMA operand layout), completion on mbarriers.
+//   warps 0-3    conversion: each thread turns one row of a slot into fp16 in place (exact for
+//                bf16) and sums its squares (the stored norm, and the scale of u).
+//   warp 13      MMA issuer: Y = X (Pi_hi + Pi_lo)^T for K and V into one of two tensor-memory
+//                buffers; later S (rho_hi + rho_lo) for the QJL signs, A read from tensor memory.
+//   warps 4-11   epilogue: two warpgroups split the 128 coordinates of every row.  Codes come
+//                from a uniform-cell lookup table (one fma gives the cell, one compare against
+//                the cell's threshold gives the code); the key residual rho goes back into
+//                tensor memory as fp16 hi + lo over Y_K; the sketch lands over Y_V.  Rows are
+//                staged in shared memory and leave by bulk copies.
+//   warps 14-15  fixups: coordinates whose fast value lies within a guard band of a decision
+//                boundary (a threshold; 0 for a sign) are re-derived in fp64 from the original
+//                inputs after the tile has been stored, and patched in place.
+// Exactness: codes and sign bits equal those of the float64 definition except where the exact
+// value lies within ~1e-15 of a boundary.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "tq_internal.h"
+#include "tq_sm100.h"
+
+namespace tq {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = kHeadDim;
+constexpr int TM = 128;                     // tokens per tile (MMA M)
+constexpr int SLOTS = 3;                    // input ring: 3 x 32 KB
+constexpr int TILE_BYTES = TM * D * 2;      // one [128 x 128] 16-bit operand
+constexpr int THREADS = 512;
+constexpr int W_EPI = 4, N_EPI_WARPS = 8, EPI_THREADS = 256;
+constexpr int W_TMA = 12, W_MMA = 13, W_FIX = 14, N_FIX = 2;
+constexpr int N_CONV_WARPS = 4;
+constexpr uint32_t IDESC = idesc_f16_f32(128, 128);
+constexpr uint32_t TMEM_COLS = 512;         // two buffers x (Y_K | Y_V)
+constexpr int QCAP = 512;                   // fixup ring entries per CTA (>= 2 tiles' worth)
+constexpr int MAX_CTAS = 256;
+constexpr int LUT_N = 128;                  // cells of the code lookup tables
+constexpr float CELL_MAGIC = 8388608.0f + 64.0f;  // 2^23 + cell offset: fma(u, alpha, .) rounds to a cell
+constexpr float PI_SCALE = 256.0f;
+constexpr long long WAIT_LIMIT = 4000000000LL;    // ~2 s of SM clock
+constexpr float C_SCALE = 0.04419417382415922f;   // sqrt(128) / 256 (u = y * C_SCALE / ||x||)
+
+__device__ unsigned int g_pipe_error;         // bit 0: a wait timed out; bit 1: smem misaligned; bit 2: no LUT
+__device__ unsigned int g_pipe_vector_fixups;
+__device__ unsigned int g_pipe_code_fixups;
+
+// One queued fixup: row r of global tile `tile`, half e (coordinates and sketch rows 64e..64e+63).
+struct FixEntry {
+  uint32_t tile;
+  uint16_t r;
+  uint8_t e;
+  uint8_t flags;  // bit 0: key codes in kmask; bit 1: value codes in vmask; bit 2: sketch rows in smask
+  uint32_t kmask[2];
+  uint32_t vmask[2];
+  uint32_t smask[2];
+};
+__device__ FixEntry g_fix_ring[MAX_CTAS][QCAP];
+
+struct PArgs {
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  int64_t sb, sh, st;
+  int T_new, t_offset;
+  int B, Hkv, T_cap;
+  int qjl;
+  int tiles_per_bh;
+  int64_t total_tiles;
+  uint8_t* k_codes;
+  uint8_t* k_signs;
+  float* k_norm;
+  float* k_rnorm;
+  uint8_t* v_codes;
+  float* v_norm;
+  const float* Pi;
+  const float* S;
+  const float* kc;
+  const float* kt;
+  const float* vc;
+  const float* vt;
+  float band_code, band_sign;
+};
+
+struct __align__(1024) PSmem {
+  uint8_t slot[SLOTS][TILE_BYTES];  // bf16 tiles from TMA, fp16 after conversion (A operands)
+  uint8_t pih[TILE_BYTES];          // 2^8 Pi, fp16 hi (B operand: row n = output coordinate)
+  uint8_t pil[TILE_BYTES];          // 2^8 Pi, fp16 lo
+  uint8_t sm[TILE_BYTES];           // S, exact in fp16
+  // Staged output rows with a pitch of (row bytes + 4): the 32 rows a warp writes at one column
+  // land on 32 different banks.
+  uint8_t kst[TM * 68];             // key codes (16 * k_bits bytes per row)
+  uint8_t vst[TM * 68];             // value codes
+  uint8_t sst[TM * 20];             // sign bits
+  float kn[TM], vn[TM];             // staged norms
+  float sclk[2][TM], sclv[2][TM];   // per tile buffer: u = y * scl (0: zero or non-finite row)
+  float nrk[2][TM], nrv[2][TM];     // per tile buffer: ||x|| as stored
+  float rho2[2][TM];                // ||rho||^2 of each coordinate half
+  uint32_t klut[LUT_N];             // key cells: threshold (fp32) with the code below it in bits 0..3
+  uint32_t vlut[LUT_N];             // value cells, same format
+  double frho[N_FIX][D];            // fixup scratch: exact residual
+  uint8_t fcode[N_FIX][D];          // fixup scratch: codes by slot
+  uint8_t fsign[N_FIX][D];          // fixup scratch: sign bits by position
+  float kcent[16], kthr[16], vcent[16], vthr[16];
+  float alpha_k, alpha_v;
+  uint8_t zrow[2][TM];              // bit 0: key row takes no code fixups (zero / non-finite); bit 1: value row
+  uint64_t full[SLOTS], conv[SLOTS], empty[SLOTS];
+  uint64_t yfull[2], sfull[2], tfree[2], rinfo[2];
+  unsigned int rho_cnt[2];   // epilogue warps done with the residuals of buffer 0 / 1
+  uint32_t tmem_base;
+  unsigned int err;
+  unsigned int q_tail;       // fixup entries pushed
+  unsigned int q_pub;        // entries whose tiles are in global memory
+  unsigned int stored_seq;   // tiles published (progress signal for the fixup warps)
+  unsigned int main_done;
+  unsigned int fix_done[N_FIX];
+  unsigned int ep_abort;
+};
+
+static_assert(sizeof(PSmem) <= 232448, "shared memory per CTA");
+
+// Byte offset of 16-byte chunk c (0..15) of row r of a [128 x 128] 16-bit operand tile: two
+// 64-element K atoms of 16 KB, 8-row groups 1024 bytes apart, chunks XOR-swizzled by (r % 8)
+// (the layout TMA writes with 128-byte swizzle and UMMA reads).
+__device__ __forceinline__ uint32_t sw_chunk(int r, int c) {
+  return (uint32_t)((c >> 3) * (TM * 128) + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ uint64_t desc_at(const uint8_t* tile, int kstep) {
+  return desc_sw128_kmajor(smem_u32(tile) + (kstep >> 2) * (TM * 128) + (kstep & 3) * 32);
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+__device__ __forceinline__ unsigned int ld_acq(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];\n" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_rel(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;\n" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// Bounded wait on an mbarrier phase; gives up when another role has failed.  Each try_wait
+// suspends the thread in hardware until the phase completes or ~0.1 ms pass, so a waiting warp
+// takes no issue slots from the warps that do the work.
+__device__ __forceinline__ bool pwait(PSmem& s, uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity), "r"(100000u)
+        : "memory");
+    if (done) return true;
+    if (*reinterpret_cast<volatile unsigned int*>(&s.err)) return false;
+    if (clock64() - t0 > WAIT_LIMIT) {
+      atomicOr(&s.err, 1u);
+      return false;
+    }
+  }
+}
+
+// Row-major fp32 [128 x 128] matrix times `scale` (a power of two) into fp16 hi (+ lo) tiles.
+__device__ void load_matrix(const float* __restrict__ M, float scale, uint8_t* hi, uint8_t* lo) {
+  for (int i = threadIdx.x; i < D * D / 8; i += THREADS) {
+    const int r = i / 16, c = i % 16;
+    const float4 p0 = reinterpret_cast<const float4*>(M + r * D + 8 * c)[0];
+    const float4 p1 = reinterpret_cast<const float4*>(M + r * D + 8 * c)[1];
+    const float v[8] = {p0.x * scale, p0.y * scale, p0.z * scale, p0.w * scale,
+                        p1.x * scale, p1.y * scale, p1.z * scale, p1.w * scale};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2 hh = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+      const float2 hf = __half22float2(hh);
+      h[e] = h2_bits(hh);
+      l[e] = h2_bits(__floats2half2_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y));
+    }
+    *reinterpret_cast<uint4*>(hi + sw_chunk(r, c)) = make_uint4(h[0], h[1], h[2], h[3]);
+    if (lo) *reinterpret_cast<uint4*>(lo + sw_chunk(r, c)) = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+}
+
+// Uniform-cell code table for one codebook (one warp).  Cell k covers the u with
+// rint(u * alpha + 64) == k.  alpha makes every cell at least as narrow as the smallest gap
+// between thresholds (so a cell holds at most one threshold) and keeps every threshold at least
+// 0.05 cells from a cell edge (so a value within the guard band of a threshold always falls in
+// that threshold's cell).  Entry: the threshold in the cell (2^100 if none), whose fp32 mantissa
+// ends in at least four zero bits (a midpoint of two fp16 centroids), with the code just below
+// it in those bits.  Four-byte entries keep the 32 lanes of a warp on distinct banks unless
+// their cells are 32 apart.
+__device__ void build_lut(const float* t, int L, uint32_t* lut, float* alpha_out, unsigned int* err) {
+  const int lane = threadIdx.x & 31;
+  const int nt = L - 1;
+  float gap = INFINITY;
+  bool fmt = true;
+  for (int i = 0; i < nt; ++i) {
+    if (i + 1 < nt) gap = fminf(gap, t[i + 1] - t[i]);
+    fmt = fmt && (__float_as_uint(t[i]) & 15u) == 0u;
+  }
+  const float alpha = (1.0f + 0.4f * (float)lane / 32.0f) / gap;
+  bool ok = fmt && alpha * 11.5f < 62.0f;  // |u| <= sqrt(128) < 11.32: cells stay inside 2..126
+  for (int i = 0; i < nt; ++i) {
+    const float x = t[i] * alpha;
+    ok = ok && fabsf((x - floorf(x)) - 0.5f) >= 0.05f;
+  }
+  const unsigned int m = __ballot_sync(0xffffffffu, ok);
+  if (m == 0) {
+    if (lane == 0) atomicOr(err, 4u);
+    return;
+  }
+  const float a = __shfl_sync(0xffffffffu, alpha, __ffs(m) - 1);
+  if (lane == 0) *alpha_out = a;
+  for (int k = lane; k < LUT_N; k += 32) {
+    int below = 0, hit = -1;
+    for (int i = 0; i < nt; ++i) {
+      const int ck = (int)(__float_as_uint(fmaf(t[i], a, CELL_MAGIC)) & 0x7fffffu);
+      if (ck < k) ++below;
+      else if (ck == k) hit = i;
+    }
+    const uint32_t thr = hit >= 0 ? __float_as_uint(t[hit]) : 0x71800000u;  // 2^100: never reached
+    lut[k] = thr | (uint32_t)below;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Conversion of row r of a bf16 tile to fp16 in place.  ||x||^2 accumulates in fp32 (16 chains of
+// 8 exact squares, then a 4-level tree: relative error <= 11 * 2^-24).  Rows with ||x|| in
+// [4, 65504) convert unscaled: every element fits fp16, and elements below 2^-14 (fp16
+// subnormal, rounded to 2^-24) move u by at most 2^-18 / ||x|| <= 1e-6.  Other rows are
+// re-derived in fp64 and scaled by 2^e first (codes depend only on the direction of x).
+__device__ __forceinline__ void convert_row(uint8_t* tile, int r, const __nv_bfloat16* __restrict__ src,
+                                            float& nrm, float& scl, uint8_t& zero) {
+  uint4 raw16[16];  // all loads first: the in-place stores below would otherwise order them
+#pragma unroll
+  for (int q = 0; q < 16; ++q) raw16[q] = *reinterpret_cast<const uint4*>(tile + sw_chunk(r, q));
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint4 raw = raw16[q];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+      const int ai = (4 * q + e) & 15;
+      acc[ai] = fmaf(lo, lo, acc[ai]);
+      acc[ai] = fmaf(hi, hi, acc[ai]);
+      o[e] = h2_bits(__floats2half2_rn(lo, hi));
+    }
+    *reinterpret_cast<uint4*>(tile + sw_chunk(r, q)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+#pragma unroll
+  for (int h = 8; h > 0; h >>= 1)
+#pragma unroll
+    for (int i = 0; i < h; ++i) acc[i] += acc[i + h];
+  const float ss = acc[0];
+  if (ss >= 16.0f && ss < 65504.0f * 65504.0f) {
+    nrm = __fsqrt_rn(ss);
+    scl = C_SCALE * rsqrtf(ss);  // relative error ~2^-23: ~3e-7 in u near a threshold
+    zero = 0;
+    return;
+  }
+  // rare: tiny, huge, zero or non-finite rows, re-read from global memory
+  const uint4* g = reinterpret_cast<const uint4*>(src);
+  double ssd = 0.0;
+#pragma unroll 1
+  for (int q = 0; q < 16; ++q) {
+    const uint4 raw = g[q];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double lo = (double)__uint_as_float(w[e] << 16), hi = (double)__uint_as_float(w[e] & 0xffff0000u);
+      ssd = fma(lo, lo, ssd);
+      ssd = fma(hi, hi, ssd);
+    }
+  }
+  if (ssd == 0.0 || !isfinite(ssd)) {
+    // zero row (codes of u = 0), or inf / nan elements: the row enters the MMA as zeros
+#pragma unroll 1
+    for (int q = 0; q < 16; ++q) *reinterpret_cast<uint4*>(tile + sw_chunk(r, q)) = make_uint4(0u, 0u, 0u, 0u);
+    nrm = (float)sqrt(ssd);
+    scl = 0.0f;
+    zero = 1;
+    return;
+  }
+  const double n = sqrt(ssd);
+  int ex = 0;
+  frexp(n, &ex);
+  const int e = 14 - ex;  // n * 2^e in [2^13, 2^14)
+  const float p2a = ldexpf(1.0f, e / 2), p2b = ldexpf(1.0f, e - e / 2);
+#pragma unroll 1
+  for (int q = 0; q < 16; ++q) {
+    const uint4 raw = g[q];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = __uint_as_float(w[k] << 16) * p2a * p2b;
+      const float hi = __uint_as_float(w[k] & 0xffff0000u) * p2a * p2b;
+      o[k] = h2_bits(__floats2half2_rn(lo, hi));
+    }
+    *reinterpret_cast<uint4*>(tile + sw_chunk(r, q)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  nrm = (float)n;
+  scl = (float)((double)C_SCALE / ldexp(n, e));
+  zero = 0;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Epilogue pieces.  A thread owns TMEM lane r (one row) and a 32-column chunk at a time.
+
+// Values, chunk cc (0/1) of half e: coordinate 32(2e+cc)+i sits at value slot 16(i%8) + 8e +
+// 4cc + i/8, i.e. field g = i%8 (8 codes at byte v_bits * (2g + e)) position 4cc + i/8.
+template <int VB>
+__device__ __forceinline__ void v_chunk(const uint32_t (&y)[32], float sv, float sva, const uint32_t* vlut,
+                                        uint32_t (&f)[8], float& mn) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float yv = __uint_as_float(y[i]);
+    const uint32_t L = vlut[__float_as_uint(fmaf(yv, sva, CELL_MAGIC)) & (LUT_N - 1)];
+    const float d = fmaf(yv, sv, -__uint_as_float(L & ~15u));
+    const uint32_t code = (L & 15u) + (d >= 0.0f ? 1u : 0u);
+    mn = fminf(mn, fabsf(d));
+    f[i & 7] += code << (VB * (i >> 3));
+  }
+}
+// (Inline and unrolled: y stays in registers.  A call taking y by reference would place the
+// array in local memory for every chunk.)
+__device__ __forceinline__ uint32_t v_near(const uint32_t (&y)[32], float sv, float sva, const uint32_t* vlut,
+                                           float band) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float yv = __uint_as_float(y[i]);
+    const uint32_t L = vlut[__float_as_uint(fmaf(yv, sva, CELL_MAGIC)) & (LUT_N - 1)];
+    if (fabsf(fmaf(yv, sv, -__uint_as_float(L & ~15u))) < band) m |= 1u << i;
+  }
+  return m;
+}
+
+// Keys, chunk ch: coordinate 32ch + i = 16 kap + 8h + 2tau + eps sits at key slot
+// 32 tau + 8ch + p, p = 4(i/16) + 2h + eps: field tau (8 codes at byte k_bits * (4 tau + ch)).
+template <int KB>
+__device__ __forceinline__ void k_chunk(const uint32_t (&y)[32], float sk, float ska, const uint32_t* klut,
+                                        const float* kcent, uint32_t (&f)[4], uint32_t (&hi)[16],
+                                        uint32_t (&lo)[16], float& r2, float& mn) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    float rr[2];
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const int ii = i + e2;
+      const float yv = __uint_as_float(y[ii]);
+      const uint32_t L = klut[__float_as_uint(fmaf(yv, ska, CELL_MAGIC)) & (LUT_N - 1)];
+      const float d = fmaf(yv, sk, -__uint_as_float(L & ~15u));
+      const uint32_t code = (L & 15u) + (d >= 0.0f ? 1u : 0u);
+      const float rho = fmaf(yv, sk, -kcent[code]);
+      mn = fminf(mn, fabsf(d));
+      r2 = fmaf(rho, rho, r2);
+      rr[e2] = rho;
+      const int tau = (ii >> 1) & 3, p = ((ii >> 4) << 2) | (((ii >> 3) & 1) << 1) | (ii & 1);
+      f[tau] += code << (KB * p);
+    }
+    const __half2 hh = __floats2half2_rn(rr[0], rr[1]);
+    const float2 hf = __half22float2(hh);
+    hi[i >> 1] = h2_bits(hh);
+    lo[i >> 1] = h2_bits(__floats2half2_rn(rr[0] - hf.x, rr[1] - hf.y));
+  }
+}
+__device__ __forceinline__ uint32_t k_near(const uint32_t (&y)[32], float sk, float ska, const uint32_t* klut,
+                                           float band) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float yv = __uint_as_float(y[i]);
+    const uint32_t L = klut[__float_as_uint(fmaf(yv, ska, CELL_MAGIC)) & (LUT_N - 1)];
+    if (fabsf(fmaf(yv, sk, -__uint_as_float(L & ~15u))) < band) m |= 1u << i;
+  }
+  return m;
+}
+
+// Signs, chunk cc of half e: sketch row l = 64e + 32cc + i = 16 kap + 8h + 2tau + eps has row
+// bit 32 tau + 16 eps + 8e + (4cc + 2(i/16) + h): byte 4 tau + 2 eps + e, bit 4cc + 2(i/16) + h.
+// Here bit 2(i/16) + h of entry 2 tau + eps; the caller shifts by 4cc.
+__device__ __forceinline__ void s_chunk(const uint32_t (&y)[32], uint32_t (&sb)[8], float& mn) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float v = __uint_as_float(y[i]);
+    mn = fminf(mn, fabsf(v));
+    const int bit = 2 * (i >> 4) + ((i >> 3) & 1);
+    sb[((i >> 1) & 3) * 2 + (i & 1)] |= (v >= 0.0f ? 1u : 0u) << bit;
+  }
+}
+
+__device__ __forceinline__ uint32_t s_near(const uint32_t (&y)[32], float band) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (fabsf(__uint_as_float(y[i])) < band) m |= 1u << i;
+  return m;
+}
+
+// ---------------------------------------------------------------------------------------------
+// fp64 fixups (one warp per queued entry).
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// Code of an exact (fp64) coordinate through the cell table: the cell from u in fp32 (a threshold
+// is never within 0.05 cells of a cell edge, so rounding u cannot change which threshold the cell
+// holds), then an exact comparison against that threshold.
+__device__ __forceinline__ uint32_t code_lut(double u, const uint32_t* lut, float alpha) {
+  const uint32_t L = lut[__float_as_uint(fmaf((float)u, alpha, CELL_MAGIC)) & (LUT_N - 1)];
+  return (L & 15u) + (u >= (double)__uint_as_float(L & ~15u) ? 1u : 0u);
+}
+// Lane holds x[4 lane .. 4 lane + 3]; returns the exact dot product of Pi row j with x.
+__device__ __forceinline__ double pi_dot(const float* __restrict__ Pi, int j, const double (&x)[4]) {
+  const int lane = threadIdx.x & 31;
+  const float4 p = reinterpret_cast<const float4*>(Pi + j * D)[lane];
+  double acc = (double)p.x * x[0];
+  acc = fma((double)p.y, x[1], acc);
+  acc = fma((double)p.z, x[2], acc);
+  acc = fma((double)p.w, x[3], acc);
+  return warp_sum(acc);
+}
+__device__ __forceinline__ void load_row(const __nv_bfloat16* src, double (&x)[4]) {
+  const int lane = threadIdx.x & 31;
+  const uint2 w = reinterpret_cast<const uint2*>(src)[lane];
+  x[0] = (double)__uint_as_float(w.x << 16);
+  x[1] = (double)__uint_as_float(w.x & 0xffff0000u);
+  x[2] = (double)__uint_as_float(w.y << 16);
+  x[3] = (double)__uint_as_float(w.y & 0xffff0000u);
+}
+// Exact dot products of all 128 rows of a row-major fp32 [128 x 128] matrix M with a vector the
+// warp holds as v[4 lane .. 4 lane + 3] (fp64).  Rows go 8 per round with the next round's loads
+// in flight; the 8 partial sums are reduced across the warp by halving exchanges, after which
+// lane L holds row j0 + ((L >> 2) & 7) and lanes with L % 4 == 0 call sink(row, value).
+template <typename Sink>
+__device__ __forceinline__ void matvec8(const float* __restrict__ M, const double (&v)[4], Sink&& sink) {
+  const int lane = threadIdx.x & 31;
+  const float4* M4 = reinterpret_cast<const float4*>(M);
+  float4 cur[8], nxt[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) cur[q] = M4[q * 32 + lane];
+#pragma unroll 1
+  for (int j0 = 0; j0 < D; j0 += 8) {
+    if (j0 + 8 < D) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) nxt[q] = M4[(j0 + 8 + q) * 32 + lane];
+    }
+    double d[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      double acc = (double)cur[q].x * v[0];
+      acc = fma((double)cur[q].y, v[1], acc);
+      acc = fma((double)cur[q].z, v[2], acc);
+      d[q] = fma((double)cur[q].w, v[3], acc);
+    }
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    double e4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double send = b4 ? d[i] : d[i + 4];
+      e4[i] = (b4 ? d[i + 4] : d[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    double e2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const double send = b3 ? e4[i] : e4[i + 2];
+      e2[i] = (b3 ? e4[i + 2] : e4[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    double e1 = (b2 ? e2[1] : e2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? e2[0] : e2[1], 4);
+    e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
+    e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+    if ((lane & 3) == 0) sink(j0 + ((lane >> 2) & 7), e1);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cur[q] = nxt[q];
+  }
+}
+
+__device__ __forceinline__ uint32_t get_code(const uint8_t* row, int bits, int slot) {
+  const int P = bits * slot;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(row);
+  uint64_t v = w[P >> 5];
+  if ((P & 31) + bits > 32) v |= (uint64_t)w[(P >> 5) + 1] << 32;
+  return (uint32_t)(v >> (P & 31)) & ((1u << bits) - 1u);
+}
+// Atomic so that the two halves of a row can be patched by different warps.
+__device__ __forceinline__ void set_code(uint8_t* row, int bits, int slot, uint32_t code) {
+  const int P = bits * slot;
+  uint32_t* w = reinterpret_cast<uint32_t*>(row);
+  const int wi = P >> 5, sh = P & 31;
+  const uint64_t m = (uint64_t)((1u << bits) - 1u) << sh;
+  const uint64_t c = (uint64_t)code << sh;
+  atomicAnd(&w[wi], ~(uint32_t)m);
+  atomicOr(&w[wi], (uint32_t)c);
+  if (sh + bits > 32) {
+    atomicAnd(&w[wi + 1], ~(uint32_t)(m >> 32));
+    atomicOr(&w[wi + 1], (uint32_t)(c >> 32));
+  }
+}
+
+template <int KB, int VB>
+__device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEntry& E, int w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int LK = 1 << KB, LV = 1 << VB;
+  const int bh = (int)(E.tile / (uint32_t)a.tiles_per_bh);
+  const int t = (int)(E.tile % (uint32_t)a.tiles_per_bh) * TM + E.r;
+  const int b = bh / a.Hkv, h = bh % a.Hkv;
+  const int64_t in_off = (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)t * a.st;
+  const int64_t row = ((int64_t)b * a.Hkv + h) * a.T_cap + a.t_offset + t;
+  const double sqd = sqrt((double)D);
+  unsigned int ncodes = 0;
+  if (E.flags & 2) {
+    double x[4];
+    load_row(a.v + in_off, x);
+    const double n = sqrt(warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]));
+    uint8_t* vrow = a.v_codes + row * (16 * VB);
+    for (int hw = 0; hw < 2; ++hw) {
+      uint32_t m = E.vmask[hw];
+      while (m) {
+        const int j = 64 * E.e + 32 * hw + __ffs(m) - 1;
+        m &= m - 1;
+        const double dot = pi_dot(a.Pi, j, x);
+        const uint32_t code = n > 0.0 ? code_lut(sqd * dot / n, s.vlut, s.alpha_v) : (uint32_t)(LV / 2);
+        if (lane == 0 && get_code(vrow, VB, v_slot_of_coord(j)) != code) set_code(vrow, VB, v_slot_of_coord(j), code);
+        ++ncodes;
+      }
+    }
+  }
+  bool vec = false;  // a key code changed: every sign and ||r|| are re-derived
+  if (!(E.flags & 5)) return;
+  double x[4];
+  load_row(a.k + in_off, x);
+  const double nk = sqrt(warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]));
+  uint8_t* krow = a.k_codes + row * (16 * KB);
+  if (E.flags & 1) {
+    for (int hw = 0; hw < 2; ++hw) {
+      uint32_t m = E.kmask[hw];
+      while (m) {
+        const int j = 64 * E.e + 32 * hw + __ffs(m) - 1;
+        m &= m - 1;
+        const double dot = pi_dot(a.Pi, j, x);
+        const uint32_t code = nk > 0.0 ? code_lut(sqd * dot / nk, s.klut, s.alpha_k) : (uint32_t)(LK / 2);
+        const uint32_t old = __shfl_sync(0xffffffffu, lane == 0 ? get_code(krow, KB, k_slot_of_coord(j)) : 0u, 0);
+        if (old != code) {
+          if (lane == 0) set_code(krow, KB, k_slot_of_coord(j), code);
+          vec = true;  // the residual fed to the sketch came from the other cell
+        }
+        ++ncodes;
+      }
+    }
+  }
+  if (lane == 0 && ncodes) atomicAdd(&g_pipe_code_fixups, ncodes);
+  if (!a.qjl || (!vec && !(E.flags & 4))) return;
+  // Exact residual of the whole key vector (fp64): u, codes, rho.
+  double r2 = 0.0;
+  matvec8(a.Pi, x, [&](int j, double dot) {  // lane (4 q) receives Pi row j = j0 + q
+    const double u = nk > 0.0 ? sqd * dot / nk : 0.0;
+    const uint32_t code = nk > 0.0 ? code_lut(u, s.klut, s.alpha_k) : (uint32_t)(LK / 2);
+    const double rho = u - (double)s.kcent[code];
+    s.frho[w][j] = rho;
+    s.fcode[w][k_slot_of_coord(j)] = (uint8_t)code;
+    r2 = fma(rho, rho, r2);
+  });
+  r2 = warp_sum(r2);
+  __syncwarp();
+  double rl[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) rl[m] = s.frho[w][4 * lane + m];
+  if (!vec) {
+    // Codes unchanged: only the sketch rows whose fast value was near 0 need the exact sign.
+    uint32_t* srow = reinterpret_cast<uint32_t*>(a.k_signs + row * 16);
+    for (int hw = 0; hw < 2; ++hw) {
+      uint32_t m = E.smask[hw];
+      while (m) {
+        const int l = 64 * E.e + 32 * hw + __ffs(m) - 1;
+        m &= m - 1;
+        const float4 p = reinterpret_cast<const float4*>(a.S + l * D)[lane];
+        double acc = (double)p.x * rl[0];
+        acc = fma((double)p.y, rl[1], acc);
+        acc = fma((double)p.z, rl[2], acc);
+        acc = fma((double)p.w, rl[3], acc);
+        const double sp = warp_sum(acc);
+        if (lane == 0) {
+          const int bit = sign_bit_of_row(l);
+          if (sp >= 0.0) atomicOr(&srow[bit >> 5], 1u << (bit & 31));
+          else atomicAnd(&srow[bit >> 5], ~(1u << (bit & 31)));
+        }
+      }
+    }
+    if (lane == 0) atomicAdd(&g_pipe_vector_fixups, 1u);
+    return;
+  }
+  matvec8(a.S, rl, [&](int l, double sp) { s.fsign[w][sign_bit_of_row(l)] = sp >= 0.0 ? 1 : 0; });
+  __syncwarp();
+  if (lane < 4 * KB) {
+    uint32_t word = 0;
+    for (int kk = 0; kk < 32; ++kk) {
+      const int P = 32 * lane + kk;
+      word |= (uint32_t)((s.fcode[w][P / KB] >> (P % KB)) & 1) << kk;
+    }
+    reinterpret_cast<uint32_t*>(krow)[lane] = word;
+  } else if (lane >= 16 && lane < 20) {
+    const int q = lane - 16;
+    uint32_t word = 0;
+    for (int kk = 0; kk < 32; ++kk) word |= (uint32_t)s.fsign[w][32 * q + kk] << kk;
+    reinterpret_cast<uint32_t*>(a.k_signs + row * 16)[q] = word;
+  } else if (lane == 31) {
+    a.k_rnorm[row] = (float)(nk * sqrt(r2) / sqd);
+    atomicAdd(&g_pipe_vector_fixups, 1u);
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------------------------
+// The CTA's shared memory as PSmem (an address the compiler knows is shared).
+__device__ __forceinline__ PSmem& smem() {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  return *reinterpret_cast<PSmem*>(smem_raw);
+}
+
+__device__ __forceinline__ int64_t tile_of(int it) { return (int64_t)blockIdx.x + (int64_t)it * gridDim.x; }
+__device__ __forceinline__ void coords(const PArgs& a, int64_t tile, int& b, int& h, int& t0, int& nt) {
+  const int bh = (int)(tile / a.tiles_per_bh);
+  t0 = (int)(tile % a.tiles_per_bh) * TM;
+  nt = min(TM, a.T_new - t0);
+  b = bh / a.Hkv;
+  h = bh % a.Hkv;
+}
+
+// ================================================================ TMA producer (warp 12)
+__device__ __noinline__ void role_tma(const PArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                                      int n_tiles) {
+  PSmem& s = smem();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)tid; (void)warp; (void)lane;
+  // ================================================================ TMA producer
+  if (lane == 0) {
+    int issued = 0;
+    for (int it = 0; it < n_tiles; ++it) {
+      int b, h, t0, nt;
+      coords(a, tile_of(it), b, h, t0, nt);
+      bool ok = true;
+      for (int which = 0; which < 2 && ok; ++which) {
+        const int L = 2 * it + which, sl = L % SLOTS, u = L / SLOTS;
+        if (u >= 1 && !pwait(s, &s.empty[sl], (u - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&s.full[sl], TILE_BYTES);
+        const void* tm = which ? (const void*)tmv : (const void*)tmk;
+        tma_load_4d(smem_u32(s.slot[sl]), tm, &s.full[sl], 0, t0, h, b);
+        tma_load_4d(smem_u32(s.slot[sl] + TILE_BYTES / 2), tm, &s.full[sl], 64, t0, h, b);
+        ++issued;
+      }
+      if (!ok) break;
+    }
+    // every load issued has landed before the CTA may exit
+    for (int L = max(0, issued - SLOTS); L < issued; ++L) {
+      const long long t0 = clock64();
+      while (!mbar_test(&s.full[L % SLOTS], (L / SLOTS) & 1) && clock64() - t0 < WAIT_LIMIT) {
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// ================================================================ MMA issuer (warp 13)
+__device__ __noinline__ void role_mma(const PArgs& a, uint32_t tmem, int n_tiles) {
+  PSmem& s = smem();
+  const int lane = threadIdx.x & 31;
+  // Y_K = X_K (Pi_hi + Pi_lo)^T and Y_V likewise, into tensor-memory buffer (tile & 1).  The sketch
+  // MMA of a tile is issued by the epilogue warp that finishes its residuals last.
+  if (lane == 0) {
+    int it = 0;
+    for (; it < n_tiles; ++it) {
+      const int bb = it & 1, v = it >> 1;
+      const int LKd = 2 * it, LVd = 2 * it + 1;
+      const int sK = LKd % SLOTS, sV = LVd % SLOTS;
+      if (it >= 2 && !pwait(s, &s.tfree[bb], (v - 1) & 1)) break;
+      if (!pwait(s, &s.conv[sK], (LKd / SLOTS) & 1) || !pwait(s, &s.conv[sV], (LVd / SLOTS) & 1)) break;
+      tc_fence_after();
+      const uint32_t dk = tmem + 256 * bb, dv = dk + 128;
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        umma_f16(dk, desc_at(s.slot[sK], ks), desc_at(s.pih, ks), IDESC, ks > 0);
+        umma_f16(dk, desc_at(s.slot[sK], ks), desc_at(s.pil, ks), IDESC, 1);
+      }
+      umma_commit(&s.empty[sK]);
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        umma_f16(dv, desc_at(s.slot[sV], ks), desc_at(s.pih, ks), IDESC, ks > 0);
+        umma_f16(dv, desc_at(s.slot[sV], ks), desc_at(s.pil, ks), IDESC, 1);
+      }
+      umma_commit(&s.empty[sV]);
+      umma_commit(&s.yfull[bb]);
+    }
+    // every MMA issued has completed before tensor memory is released
+    if (it > 0) pwait(s, &s.yfull[(it - 1) & 1], ((it - 1) >> 1) & 1);
+  }
+  __syncwarp();
+}
+
+// ================================================================ conversion (warps 0-3)
+__device__ __noinline__ void role_conv(const PArgs& a, int n_tiles) {
+  PSmem& s = smem();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)tid; (void)warp; (void)lane;
+  // ================================================================ conversion
+  const int r = tid;  // row 0..127
+  for (int it = 0; it < n_tiles; ++it) {
+    int b, h, t0, nt;
+    coords(a, tile_of(it), b, h, t0, nt);
+    const int bb = it & 1, v = it >> 1;
+    if (it >= 2 && !pwait(s, &s.tfree[bb], (v - 1) & 1)) break;  // row info buffer is free
+    bool ok = true;
+    for (int which = 0; which < 2; ++which) {
+      const int L = 2 * it + which, sl = L % SLOTS, u = L / SLOTS;
+      if (!pwait(s, &s.full[sl], u & 1)) {
+        ok = false;
+        break;
+      }
+      float nrm = 0.0f, scl = 0.0f;
+      uint8_t zero = 1;
+      if (r < nt) {
+        const __nv_bfloat16* src = (which ? a.v : a.k) + (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)(t0 + r) * a.st;
+        convert_row(s.slot[sl], r, src, nrm, scl, zero);
+      }
+      if (which == 0) {
+        s.sclk[bb][r] = scl;
+        s.nrk[bb][r] = nrm;
+        s.zrow[bb][r] = zero;
+      } else {
+        s.sclv[bb][r] = scl;
+        s.nrv[bb][r] = nrm;
+        s.zrow[bb][r] |= (uint8_t)(zero << 1);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.conv[sl]);
+    }
+    if (!ok) break;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.rinfo[bb]);
+  }
+}
+
+// Rows [0, n) of a staged array (row bytes 16 * C, pitch `pitch`) to contiguous global memory.
+template <int C>
+__device__ __forceinline__ void copy_rows(const uint8_t* st, int pitch, uint8_t* g, int n, int t) {
+  uint4* dst = reinterpret_cast<uint4*>(g);
+  for (int c = t; c < n * C; c += EPI_THREADS) {
+    const int i = c / C, q = c - i * C;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(st + i * pitch + 16 * q);
+    dst[c] = make_uint4(src[0], src[1], src[2], src[3]);
+  }
+}
+
+// ================================================================ epilogue (warps 4-11)
+template <int KB, int VB>
+__device__ __noinline__ void role_epi(const PArgs& a, uint32_t tmem, int n_tiles) {
+  PSmem& s = smem();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ew = warp - W_EPI, e = ew >> 2;  // warpgroup e owns coordinates / sketch rows 64e..64e+63
+  const int r = (warp & 3) * 32 + lane;      // row = tensor-memory lane
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const bool leader = ew == 0 && lane == 0;
+  const bool qjl = a.qjl != 0;
+  unsigned int pend[2] = {0u, 0u};  // (leader) fixup entries queued up to the end of tile it-2 / it-1
+  const float band = a.band_code, sband = a.band_sign;
+  const float alpha_k = s.alpha_k, alpha_v = s.alpha_v;
+  for (int it = 0; it < n_tiles; ++it) {
+    const int64_t tile = tile_of(it);
+    int b, h, t0, nt;
+    coords(a, tile, b, h, t0, nt);
+    const int bb = it & 1, v = it >> 1;
+    const int64_t row0 = ((int64_t)b * a.Hkv + h) * a.T_cap + a.t_offset + t0;
+    bool bad = !pwait(s, &s.rinfo[bb], v & 1);
+    const float sk = s.sclk[bb][r], sv = s.sclv[bb][r];
+    const float nk = s.nrk[bb][r], nv = s.nrv[bb][r];
+    const uint8_t zr = s.zrow[bb][r];
+    bad |= !pwait(s, &s.yfull[bb], v & 1);
+    tc_fence_after();
+    const uint32_t tb = tmem + lane_base + 256 * bb;
+
+    // ---- values: chunk cc holds coordinates 64e + 32cc + i ----
+    uint32_t vf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    uint64_t vm = 0;
+    {
+      const float sva = sv * alpha_v;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t y[32];
+        tmem_ld32(tb + 128 + 64 * e + 32 * cc, y);
+        tmem_wait_ld();
+        uint32_t lf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        float mn = INFINITY;
+        v_chunk<VB>(y, sv, sva, s.vlut, lf, mn);
+        const int sh = 4 * VB * cc;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) vf[g] |= lf[g] << sh;
+        if (mn < band && !(zr & 2)) vm |= (uint64_t)v_near(y, sv, sva, s.vlut, band) << (32 * cc);
+      }
+    }
+    // ---- B1: every thread has stored its share of tile it-1 (staging is free again) ----
+    if (leader) s.ep_abort = *reinterpret_cast<volatile unsigned int*>(&s.err) != 0 || bad;
+    named_bar(1, EPI_THREADS);
+    if (leader && it >= 1) {  // fixups of tiles up to it-1 may run
+      __threadfence_block();
+      st_rel(&s.q_pub, pend[(it - 1) & 1]);
+      st_rel(&s.stored_seq, (unsigned)it);
+    }
+    if (s.ep_abort) break;
+    {
+      uint8_t* vrow = s.vst + r * (16 * VB + 4);
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        if constexpr (VB == 4) {
+          *reinterpret_cast<uint32_t*>(vrow + 8 * g + 4 * e) = vf[g];
+        } else if constexpr (VB == 2) {
+          *reinterpret_cast<uint16_t*>(vrow + 4 * g + 2 * e) = (uint16_t)vf[g];
+        } else {
+          uint8_t* p = vrow + 6 * g + 3 * e;
+          p[0] = (uint8_t)vf[g];
+          p[1] = (uint8_t)(vf[g] >> 8);
+          p[2] = (uint8_t)(vf[g] >> 16);
+        }
+      }
+    }
+    // ---- keys: codes, residual (fp16 hi + lo over Y_K), ||rho||^2 ----
+    uint64_t km = 0;
+    float r2 = 0.0f;
+    {
+      const float ska = sk * alpha_k;
+      uint8_t* krow = s.kst + r * (16 * KB + 4);
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const uint32_t col = tb + 64 * e + 32 * cc;
+        uint32_t y[32], hi[16], lo[16];
+        uint32_t f[4] = {0u, 0u, 0u, 0u};
+        float mn = INFINITY;
+        tmem_ld32(col, y);
+        tmem_wait_ld();
+        k_chunk<KB>(y, sk, ska, s.klut, s.kcent, f, hi, lo, r2, mn);
+        if (mn < band && !(zr & 1)) km |= (uint64_t)k_near(y, sk, ska, s.klut, band) << (32 * cc);
+        if (qjl) {
+          tmem_st16(col, hi);
+          tmem_st16(col + 16, lo);
+        }
+        const int ch = 2 * e + cc;  // field (tau, ch): 8 codes at byte k_bits * (4 tau + ch)
+#pragma unroll
+        for (int tau = 0; tau < 4; ++tau) {
+          if constexpr (KB == 4) {
+            *reinterpret_cast<uint32_t*>(krow + 16 * tau + 4 * ch) = f[tau];
+          } else if constexpr (KB == 2) {
+            *reinterpret_cast<uint16_t*>(krow + 8 * tau + 2 * ch) = (uint16_t)f[tau];
+          } else {
+            uint8_t* p = krow + 12 * tau + 3 * ch;
+            p[0] = (uint8_t)f[tau];
+            p[1] = (uint8_t)(f[tau] >> 8);
+            p[2] = (uint8_t)(f[tau] >> 16);
+          }
+        }
+      }
+    }
+    if (qjl) {
+      tmem_wait_st();
+      s.rho2[e][r] = r2;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {  // the last of the eight warps issues the sketch MMA: S (rho_hi + rho_lo)
+        unsigned int old;
+        asm volatile("atom.add.acq_rel.cta.shared::cta.u32 %0, [%1], 1;\n"
+                     : "=r"(old)
+                     : "r"(smem_u32(&s.rho_cnt[bb]))
+                     : "memory");
+        if (old == N_EPI_WARPS - 1) {
+          atomicExch(&s.rho_cnt[bb], 0u);
+          tc_fence_after();
+          const uint32_t dk = tmem + 256 * bb, dv = dk + 128;
+#pragma unroll 1
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t ah = dk + 32 * (ks >> 1) + 8 * (ks & 1);
+            umma_f16_ts(dv, ah, desc_at(s.sm, ks), IDESC, ks > 0);
+            umma_f16_ts(dv, ah + 16, desc_at(s.sm, ks), IDESC, 1);
+          }
+          umma_commit(&s.sfull[bb]);
+        }
+      }
+      __syncwarp();
+    }
+    if (e == 0) {
+      s.kn[r] = nk;
+      s.vn[r] = nv;
+    }
+    // ---- signs of S rho ----
+    bool sflag = false;
+    uint64_t sm = 0;
+    if (qjl) {
+      bad |= !pwait(s, &s.sfull[bb], v & 1);
+      tc_fence_after();
+      uint32_t sb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t y[32];
+        tmem_ld32(tb + 128 + 64 * e + 32 * cc, y);
+        tmem_wait_ld();
+        uint32_t lb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        float mn = INFINITY;
+        s_chunk(y, lb, mn);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) sb[q] |= lb[q] << (4 * cc);
+        if (mn < sband) sm |= (uint64_t)s_near(y, sband) << (32 * cc);
+      }
+      sflag = sm != 0;
+      uint8_t* srow = s.sst + r * 20;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) srow[4 * (q >> 1) + 2 * (q & 1) + e] = (uint8_t)sb[q];
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.tfree[bb]);  // tensor memory buffer and row info are free
+    // ---- queue fixups (rare) ----
+    if (r < nt && (km != 0 || vm != 0 || sflag)) {
+      const unsigned int slot = atomicAdd(&s.q_tail, 1u);
+      if (slot >= QCAP) {  // the entry QCAP back (from a stored tile) must be consumed first
+        const unsigned int m = slot - QCAP;
+        const long long tw = clock64();
+        while (ld_acq(&s.fix_done[m % N_FIX]) <= m / N_FIX) {
+          if (clock64() - tw > WAIT_LIMIT || *reinterpret_cast<volatile unsigned int*>(&s.err)) {
+            atomicOr(&s.err, 1u);
+            break;
+          }
+          __nanosleep(200);
+        }
+      }
+      FixEntry E;
+      E.tile = (uint32_t)tile;
+      E.r = (uint16_t)r;
+      E.e = (uint8_t)e;
+      E.flags = (uint8_t)((km ? 1 : 0) | (vm ? 2 : 0) | (sflag ? 4 : 0));
+      E.kmask[0] = (uint32_t)km;
+      E.kmask[1] = (uint32_t)(km >> 32);
+      E.vmask[0] = (uint32_t)vm;
+      E.vmask[1] = (uint32_t)(vm >> 32);
+      E.smask[0] = (uint32_t)sm;
+      E.smask[1] = (uint32_t)(sm >> 32);
+      g_fix_ring[blockIdx.x][slot % QCAP] = E;
+    }
+    fence_proxy_async_smem();
+    named_bar(2, EPI_THREADS);
+    // ---- stores: rows [0, nt) of the tile, 16-byte chunks, consecutive threads on consecutive
+    //      chunks of the contiguous output ----
+    {
+      const int t_e = tid - W_EPI * 32;
+      copy_rows<KB>(s.kst, 16 * KB + 4, a.k_codes + row0 * (16 * KB), nt, t_e);
+      copy_rows<VB>(s.vst, 16 * VB + 4, a.v_codes + row0 * (16 * VB), nt, t_e);
+      if (qjl) copy_rows<1>(s.sst, 20, a.k_signs + row0 * 16, nt, t_e);
+      if (t_e < nt) {
+        a.k_norm[row0 + t_e] = s.kn[t_e];
+        a.v_norm[row0 + t_e] = s.vn[t_e];
+        if (qjl)
+          a.k_rnorm[row0 + t_e] = s.kn[t_e] * sqrtf(s.rho2[0][t_e] + s.rho2[1][t_e]) * (1.0f / 11.313708498984761f);
+      }
+    }
+    if (leader) pend[it & 1] = *reinterpret_cast<volatile unsigned int*>(&s.q_tail);
+  }
+  // ---- end: everything stored; the fixup warps drain the queue ----
+  named_bar(1, EPI_THREADS);
+  if (leader) {
+    __threadfence_block();
+    st_rel(&s.q_pub, *reinterpret_cast<volatile unsigned int*>(&s.q_tail));
+    st_rel(&s.stored_seq, (unsigned)n_tiles + 1u);
+    st_rel(&s.main_done, 1u);
+  }
+}
+
+// ================================================================ fp64 fixups (warps 14-15)
+template <int KB, int VB>
+__device__ __noinline__ void role_fix(const PArgs& a) {
+  PSmem& s = smem();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)tid; (void)warp; (void)lane;
+  // ================================================================ fp64 fixups
+  const int w = warp - W_FIX;
+  unsigned int k = (unsigned)w, seen = 0, done_count = 0;
+  long long t_last = clock64();
+  while (true) {
+    const unsigned int pub = ld_acq(&s.q_pub);
+    if (k < pub) {
+      const FixEntry E = g_fix_ring[blockIdx.x][k % QCAP];
+      fix_entry<KB, VB>(s, a, E, w);
+      k += N_FIX;
+      ++done_count;
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        st_rel(&s.fix_done[w], done_count);
+      }
+      t_last = clock64();
+      continue;
+    }
+    if (ld_acq(&s.main_done)) {
+      if (k >= ld_acq(&s.q_pub)) break;
+      continue;
+    }
+    if (*reinterpret_cast<volatile unsigned int*>(&s.err)) break;
+    const unsigned int sq = ld_acq(&s.stored_seq);
+    if (sq != seen) {
+      seen = sq;
+      t_last = clock64();
+    } else if (clock64() - t_last > WAIT_LIMIT) {
+      atomicOr(&s.err, 1u);
+      break;
+    }
+    __nanosleep(500);
+  }
+}
+
+template <int KB, int VB>
+__global__ void __launch_bounds__(THREADS, 1)
+    quantize_pipe_kernel(const __grid_constant__ PArgs a, const __grid_constant__ CUtensorMap tmk,
+                         const __grid_constant__ CUtensorMap tmv) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PSmem& s = *reinterpret_cast<PSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  constexpr int LK = 1 << KB, LV = 1 << VB;
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (tid == 0) atomicOr(&g_pipe_error, 2u);
+    return;
+  }
+  const int n_tiles = (int)((a.total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+
+  // ---- prologue ----
+  if (warp == W_MMA) {
+    tmem_alloc(&s.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < SLOTS; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.conv[i], N_CONV_WARPS);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.yfull[i], 1);
+      s.rho_cnt[i] = 0;
+      mbar_init(&s.sfull[i], 1);
+      mbar_init(&s.tfree[i], N_EPI_WARPS);
+      mbar_init(&s.rinfo[i], N_CONV_WARPS);
+    }
+    s.err = 0;
+    s.q_tail = 0;
+    s.q_pub = 0;
+    s.stored_seq = 0;
+    s.main_done = 0;
+    s.ep_abort = 0;
+    for (int i = 0; i < N_FIX; ++i) s.fix_done[i] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+  if (tid < LK) s.kcent[tid] = a.kc[tid];
+  if (tid < LK - 1) s.kthr[tid] = a.kt[tid];
+  if (tid < LV) s.vcent[tid] = a.vc[tid];
+  if (tid < LV - 1) s.vthr[tid] = a.vt[tid];
+  if (warp == W_FIX) build_lut(a.kt, LK, s.klut, &s.alpha_k, &s.err);
+  if (warp == W_FIX + 1) build_lut(a.vt, LV, s.vlut, &s.alpha_v, &s.err);
+  // Pi enters as 2^8 Pi so that its fp16 lo part stays clear of the subnormal range; the 2^-8 is
+  // folded into the scale of u.
+  load_matrix(a.Pi, PI_SCALE, s.pih, s.pil);
+  if (a.qjl) load_matrix(a.S, 1.0f, s.sm, nullptr);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (s.err & 4u) {  // no usable cell width for this codebook (never for Lloyd-Max grids of 2..4 bits)
+    if (tid == 0) atomicOr(&g_pipe_error, 4u);
+    if (warp == W_MMA) tmem_dealloc(s.tmem_base, TMEM_COLS);
+    return;
+  }
+  const uint32_t tmem = s.tmem_base;
+
+
+  if (warp == W_TMA) role_tma(a, &tmk, &tmv, n_tiles);
+  else if (warp == W_MMA) role_mma(a, tmem, n_tiles);
+  else if (warp < N_CONV_WARPS) role_conv(a, n_tiles);
+  else if (warp >= W_EPI && warp < W_EPI + N_EPI_WARPS) role_epi<KB, VB>(a, tmem, n_tiles);
+  else if (warp >= W_FIX && warp < W_FIX + N_FIX) role_fix<KB, VB>(a);
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0 && s.err) atomicOr(&g_pipe_error, s.err);
+  if (warp == W_MMA) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B, Hkv, T_new, 128] bf16 with element strides (sb, sh, st): boxes of 64 x 128 (one 16 KB
+// K atom of a tile), 128-byte swizzle, rows past T_new read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int B, int Hkv, int T_new, int64_t sb, int64_t sh, int64_t st) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int64_t e = 2;
+  int64_t s1 = st * e, s2 = sh * e, s3 = sb * e;
+  if (Hkv == 1) s2 = s1 * T_new;
+  if (B == 1) s3 = s2 * Hkv;
+  if (s1 <= 0 || s2 <= 0 || s3 <= 0 || s1 % 16 || s2 % 16 || s3 % 16) return false;
+  if (s1 >= (1LL << 40) || s2 >= (1LL << 40) || s3 >= (1LL << 40)) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)T_new, (cuuint64_t)Hkv, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)s1, (cuuint64_t)s2, (cuuint64_t)s3};
+  cuuint32_t box[4] = {64, TM, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KB, int VB>
+tq_status launch_kv(const PArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, int grid, cudaStream_t stream) {
+  const size_t smem = sizeof(PSmem);
+  cudaError_t err = cudaFuncSetAttribute(quantize_pipe_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(err));
+  quantize_pipe_kernel<KB, VB><<<grid, THREADS, smem, stream>>>(a, mk, mv);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "quantize launch: %s", cudaGetErrorString(err));
+  return TQ_OK;
+}
+
+}  // namespace
+
+// bf16 pipeline; returns TQ_OK with *handled = false when the inputs cannot be described by a
+// TMA tensor map (the caller then uses the general kernel).
+tq_status quantize_bf16_pipeline(const tq_params* p, const void* k, const void* v, int64_t sb, int64_t sh,
+                                 int64_t st, int T_new, int t_offset, const tq_cache* c, int sms,
+                                 cudaStream_t stream, bool* handled) {
+  *handled = false;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, k, c->B, c->Hkv, T_new, sb, sh, st) || !make_map(&mv, v, c->B, c->Hkv, T_new, sb, sh, st))
+    return TQ_OK;
+  PArgs a;
+  a.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.sb = sb;
+  a.sh = sh;
+  a.st = st;
+  a.T_new = T_new;
+  a.t_offset = t_offset;
+  a.B = c->B;
+  a.Hkv = c->Hkv;
+  a.T_cap = c->T_cap;
+  a.qjl = c->qjl_m ? 1 : 0;
+  a.tiles_per_bh = (T_new + TM - 1) / TM;
+  a.total_tiles = (int64_t)c->B * c->Hkv * a.tiles_per_bh;
+  if (a.total_tiles >= (1LL << 32)) return TQ_OK;
+  a.k_codes = c->k_codes;
+  a.k_signs = c->k_signs;
+  a.k_norm = c->k_norm;
+  a.k_rnorm = c->k_rnorm;
+  a.v_codes = c->v_codes;
+  a.v_norm = c->v_norm;
+  a.Pi = p->Pi;
+  a.S = p->S;
+  a.kc = p->k_centroids;
+  a.kt = p->k_thresholds;
+  a.vc = p->v_centroids;
+  a.vt = p->v_thresholds;
+  // Fast-path error bound in u: MMA with Pi as fp16 hi + lo (<= 7e-7 measured), the fp32 norm
+  // (<= 7e-7 relative at |u| <= 2.5) and fp16-subnormal elements (<= 1e-6): < 2.5e-6.  Signs:
+  // |S rho| error <= 8e-6 measured.  The bands are wider.
+  a.band_code = 4e-6f;
+  a.band_sign = 3e-5f;
+  const int grid = (int)std::min<int64_t>(a.total_tiles, std::min(sms, MAX_CTAS));
+  *handled = true;
+  const int kb = c->k_bits, vb = c->v_bits;
+#define TQ_PV(KB)                                                   \
+  switch (vb) {                                                     \
+    case 2: return launch_kv<KB, 2>(a, mk, mv, grid, stream);       \
+    case 3: return launch_kv<KB, 3>(a, mk, mv, grid, stream);       \
+    default: return launch_kv<KB, 4>(a, mk, mv, grid, stream);      \
+  }
+  switch (kb) {
+    case 2: TQ_PV(2)
+    case 3: TQ_PV(3)
+    default: TQ_PV(4)
+  }
+#undef TQ_PV
+}
+
+unsigned int pipe_device_errors() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pipe_error, sizeof(v)) != cudaSuccess) return 0xffffffffu;
+  return v;
+}
+long long pipe_vector_fixups() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pipe_vector_fixups, sizeof(v)) != cudaSuccess) return -1;
+  return v;
+}
+long long pipe_code_fixups() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pipe_code_fixups, sizeof(v)) != cudaSuccess) return -1;
+  return v;
+}
+
+}  // namespace tq
