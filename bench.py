@@ -104,18 +104,23 @@ class ClockSampler:
             get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
                 nv.nvmlDeviceGetCurrentClocksThrottleReasons
 
+            started = threading.Event()
+
             def run():
                 smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-                while not self._stop.is_set():
+                while True:
                     try:
                         self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax,
                                              int(get_reasons(h)), nv.nvmlDeviceGetPowerUsage(h) / 1e3))
                     except Exception:
                         pass
-                    self._stop.wait(0.001)
+                    started.set()
+                    if self._stop.is_set():
+                        break  # one last sample after the region ends
 
             self._thread = threading.Thread(target=run, daemon=True)
             self._thread.start()
+            started.wait(timeout=5)
         else:
             try:
                 self._smi = subprocess.Popen(

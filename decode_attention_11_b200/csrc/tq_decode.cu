@@ -29,10 +29,19 @@ namespace tq {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int WARPS = 4;
-constexpr int THREADS = 32 * WARPS;
-constexpr int STAGE_TOK = 16 * WARPS;  // 64 tokens per pipeline stage
-constexpr int NSTAGE = 4;
+// CTA shape per code widths.  With 4-bit keys and values the pair tables take 64 KB, so two CTAs
+// share an SM: six warps and three stages each (12 warps per SM).  Smaller tables leave room for
+// three four-warp CTAs with four stages (register-bound).
+template <int KB, int VB>
+struct Cfg {
+  static constexpr bool kPacked = KB == 4 && VB == 4;
+  static constexpr int W = kPacked ? 6 : 4;
+  static constexpr int THREADS = 32 * W;
+  static constexpr int STAGE_TOK = 16 * W;  // 16 tokens per warp per stage
+  static constexpr int NSTAGE = kPacked ? 3 : 4;
+  static constexpr int MIN_BLOCKS = kPacked ? 2 : 3;
+};
+inline int stage_tokens(int kb, int vb) { return (kb == 4 && vb == 4) ? 96 : 64; }
 constexpr int HG = 8;                  // query heads per MMA row block (hi rows 0-7, lo rows 8-15)
 constexpr int PART = 2 + D;            // (max, sum, o'[128]) per partial
 constexpr unsigned FULL = 0xffffffffu;
@@ -245,10 +254,12 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const QT* __restrict
 
 template <int KB, int VB, bool QJL>
 struct Layout {
+  static constexpr int W = Cfg<KB, VB>::W;
+  static constexpr int STAGE_TOK = Cfg<KB, VB>::STAGE_TOK;
+  static constexpr int NSTAGE = Cfg<KB, VB>::NSTAGE;
   static constexpr int K_ROW = 16 * KB;
   static constexpr int V_ROW = 16 * VB;
-  static constexpr int LUT_K = (1 << (2 * KB)) * 32;  // uint32 entries
-  static constexpr int LUT_V = (1 << (2 * VB)) * 32;
+  static constexpr bool kPackedLut = KB == 4 && VB == 4;
   static constexpr int OFF_KC = 0;
   static constexpr int OFF_SG = OFF_KC + STAGE_TOK * K_ROW;
   static constexpr int OFF_VC = OFF_SG + (QJL ? STAGE_TOK * 16 : 0);
@@ -256,10 +267,10 @@ struct Layout {
   static constexpr int OFF_RN = OFF_NK + STAGE_TOK * 4;
   static constexpr int OFF_NV = OFF_RN + (QJL ? STAGE_TOK * 4 : 0);
   static constexpr int STAGE_BYTES = OFF_NV + STAGE_TOK * 4;
-  static constexpr int LUT_BYTES = 4 * (LUT_K + LUT_V);
+  static constexpr int LUT_BYTES = kPackedLut ? 256 * 256 : ((1 << (2 * KB)) + (1 << (2 * VB))) * 128;
   // scratch after the pipeline: the CTA's own warp merge, then (last CTA) the split merge
-  static constexpr int MERGE_BYTES = 4 * (2 * HG + HG * D + 4 * HG * D + 4 * HG);
-  static_assert(MERGE_BYTES >= 4 * (WARPS * HG * 2 + WARPS * HG * D), "warp merge scratch");
+  static constexpr int MERGE_BYTES = 4 * (2 * HG + HG * D + W * HG * D + W * HG);
+  static_assert(MERGE_BYTES >= 4 * (W * HG * 2 + W * HG * D), "warp merge scratch");
   static constexpr int PIPE_BYTES = NSTAGE * STAGE_BYTES;
   static constexpr int SMEM = LUT_BYTES + (PIPE_BYTES > MERGE_BYTES ? PIPE_BYTES : MERGE_BYTES);
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
@@ -269,6 +280,7 @@ template <int KB, int VB, bool QJL>
 __device__ __forceinline__ void load_stage(const DArgs& a, unsigned char* stage, int64_t row0,
                                            int count) {
   using Lay = Layout<KB, VB, QJL>;
+  constexpr int THREADS = Cfg<KB, VB>::THREADS, STAGE_TOK = Cfg<KB, VB>::STAGE_TOK;
   const int tid = threadIdx.x;
   // key codes: KB 16-byte chunks per token
   {
@@ -318,31 +330,33 @@ __device__ __forceinline__ uint64_t load_v_chunk(const unsigned char* row, int g
 }
 
 // Log-sum-exp merge of the split partials of heads h0 .. h0+nh-1 of batch b, then o = Pi^T o'.
-// Run by the last CTA to finish; partials are read from L2 (written by other CTAs).
+// Run by the last CTA to finish (W warps); partials are read from L2 (written by other CTAs).
+template <int W>
 __device__ void merge_splits(const DArgs& a, int b, int h0, int nh, unsigned char* scratch) {
+  constexpr int T = 32 * W;
   const int tid = threadIdx.x;
   const int S = a.splits;
   float* Mr = reinterpret_cast<float*>(scratch);  // [HG]
   float* Lr = Mr + HG;                             // [HG]
   float* ob = Lr + HG;                             // [HG][D]
-  float* part4 = ob + HG * D;                      // [4][HG][D] partial sums over split groups
-  float* ls4 = part4 + 4 * HG * D;                 // [4][HG]
+  float* partw = ob + HG * D;                      // [W][HG][D] partial sums over split groups
+  float* lsw = partw + W * HG * D;                 // [W][HG]
   for (int r = 0; r < nh; ++r) {
     const float* p = a.part + ((int64_t)b * a.Hq + h0 + r) * S * PART;
     float m = -INFINITY;
-    for (int s2 = tid; s2 < S; s2 += THREADS) m = fmaxf(m, __ldcg(p + (int64_t)s2 * PART));
+    for (int s2 = tid; s2 < S; s2 += T) m = fmaxf(m, __ldcg(p + (int64_t)s2 * PART));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
     if ((tid & 31) == 0) ob[tid >> 5] = m;
     __syncthreads();
     if (tid == 0) {
       float M = -INFINITY;
-      for (int w = 0; w < WARPS; ++w) M = fmaxf(M, ob[w]);
+      for (int w = 0; w < W; ++w) M = fmaxf(M, ob[w]);
       Mr[r] = M;
     }
     __syncthreads();
   }
-  // thread = (split group g, 4-dim slice j4): sum over splits s = g (mod 4)
+  // thread = (split group g, 4-dim slice j4): sum over splits s = g (mod W)
   const int g = tid >> 5, j4 = tid & 31;
   for (int r = 0; r < nh; ++r) {
     const float M = Mr[r];
@@ -351,7 +365,7 @@ __device__ void merge_splits(const DArgs& a, int b, int h0, int nh, unsigned cha
     float lsum = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll 8
-      for (int s2 = g; s2 < S; s2 += 4) {
+      for (int s2 = g; s2 < S; s2 += W) {
         const float* ps = p + (int64_t)s2 * PART;
         const float ms = __ldcg(ps);
         const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
@@ -364,26 +378,28 @@ __device__ void merge_splits(const DArgs& a, int b, int h0, int nh, unsigned cha
         if (j4 == 0) lsum = fmaf(f, __ldcg(ps + 1), lsum);
       }
     }
-    float* dstp = part4 + (g * HG + r) * D + 4 * j4;
+    float* dstp = partw + (g * HG + r) * D + 4 * j4;
     dstp[0] = acc.x;
     dstp[1] = acc.y;
     dstp[2] = acc.z;
     dstp[3] = acc.w;
-    if (j4 == 0) ls4[g * HG + r] = lsum;
+    if (j4 == 0) lsw[g * HG + r] = lsum;
   }
   __syncthreads();
   if (tid < nh) {
     float L = 0.0f;
-    for (int gg = 0; gg < 4; ++gg) L += ls4[gg * HG + tid];
+    for (int gg = 0; gg < W; ++gg) L += lsw[gg * HG + tid];
     Lr[tid] = L;
   }
   __syncthreads();
-  for (int r = 0; r < nh; ++r) {
-    const float O = part4[(0 * HG + r) * D + tid] + part4[(1 * HG + r) * D + tid] +
-                    part4[(2 * HG + r) * D + tid] + part4[(3 * HG + r) * D + tid];
-    ob[r * D + tid] = Lr[r] > 0.0f ? O / Lr[r] : 0.0f;
-  }
+  for (int r = 0; r < nh; ++r)
+    for (int d = tid; d < D; d += T) {
+      float O = 0.0f;
+      for (int gg = 0; gg < W; ++gg) O += partw[(gg * HG + r) * D + d];
+      ob[r * D + d] = Lr[r] > 0.0f ? O / Lr[r] : 0.0f;
+    }
   __syncthreads();
+  if (tid >= D) return;
   // o_i = sum_j Pi[j][i] o'_j  (thread i; rows of Pi are read coalesced across threads)
   float acc[HG];
 #pragma unroll
@@ -401,16 +417,82 @@ __device__ void merge_splits(const DArgs& a, int b, int h0, int nh, unsigned cha
   for (int r = 0; r < nh; ++r) a.out[((int64_t)b * a.Hq + h0 + r) * D + tid] = acc[r];
 }
 
-template <int KB, int VB, bool QJL>
-__global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
+// Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (m8n8 fragment layout).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Pair-table lookups.  With 4-bit keys and values the K and V pair tables share 256-byte entry
+// slots (K replicas at +0, V replicas at +128): one byte permute turns a code byte e and the lane
+// offset into the byte address (e << 8) | 4 lane, so a pair costs one PRMT and one LDS.  Other bit
+// widths use separate tables with 128-byte entries (lane-replicated, bank = lane).
+template <int KB, int VB>
+struct PairLut {
+  static constexpr bool kPacked = KB == 4 && VB == 4;
+  static constexpr int K_BYTES = kPacked ? 0 : (1 << (2 * KB)) * 128;
+  static constexpr int V_BYTES = kPacked ? 0 : (1 << (2 * VB)) * 128;
+  static constexpr int BYTES = kPacked ? 256 * 256 : K_BYTES + V_BYTES;
+  uint32_t base;   // shared-window address of the tables
+  uint32_t lane4;  // 4 * lane
+  __device__ __forceinline__ static uint32_t lds(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+    return v;
+  }
+  __device__ __forceinline__ uint32_t k(uint32_t e) const { return lds(base + ((e << 7) | lane4)); }
+  __device__ __forceinline__ uint32_t v(uint32_t e) const { return lds(base + K_BYTES + ((e << 7) | lane4)); }
+  // byte `Bt` of word w as the pair index (packed layout only)
+  template <int Bt>
+  __device__ __forceinline__ uint32_t k_byte(uint32_t w) const {
+    return lds(base + __byte_perm(w, lane4, 0x5504u | (Bt << 4)));
+  }
+  template <int Bt>
+  __device__ __forceinline__ uint32_t v_byte(uint32_t w) const {
+    return lds(base + 128 + __byte_perm(w, lane4, 0x5504u | (Bt << 4)));
+  }
+};
+
+// Key pair P (0..15) of a thread's code chunk, as a half2 of centroids.
+template <int KB, int VB, int P>
+__device__ __forceinline__ uint32_t k_pair(const PairLut<KB, VB>& L, const uint32_t (&c)[KB]) {
+  if constexpr (PairLut<KB, VB>::kPacked) {
+    return L.template k_byte<P & 3>(c[P >> 2]);
+  } else {
+    return L.k(k_pair_index<KB, P>(c));
+  }
+}
+// Value pair NU of a token pair, as a half2 of centroids.
+template <int KB, int VB, int NU>
+__device__ __forceinline__ uint32_t v_pair(const PairLut<KB, VB>& L, const VPairs<VB>& p) {
+  if constexpr (PairLut<KB, VB>::kPacked) {
+    return L.template v_byte<((NU & 7) >> 1)>(p.w[2 * (NU >> 3) + (NU & 1)]);
+  } else {
+    return L.v(p.template index<NU>());
+  }
+}
+
+// Split-K decode over one token range.  Transposed MMAs: tokens are the M dimension and the
+// columns are (head, part) pairs, part 0 = fp16 hi and part 1 = fp16 lo of the query-side operand,
+// so one m16n8k16 covers 16 tokens of four heads:
+//   scores   D[tok x (h,p)] += Khat[tok x dim] . Q'[dim x (h,p)]        (A from the pair tables)
+//   QJL      D[tok x (h,p)] += sign[tok x row] . SQ'[row x (h,p)]        (A = +-0.5 from the bits)
+//   values   O'[dim x (h,p)] += Vhat^T[dim x tok] . P~[tok x (h,p)]      (B = P~ transposed in
+//                                                                          registers by movmatrix)
+// NB = 1 (up to 4 heads per kv-head) or 2 (up to 8): n-blocks of four heads share the A operands.
+template <int KB, int VB, bool QJL, int NB>
+__global__ void __launch_bounds__(Cfg<KB, VB>::THREADS, Cfg<KB, VB>::MIN_BLOCKS) split_kernel(DArgs a) {
   using Lay = Layout<KB, VB, QJL>;
+  using Lut = PairLut<KB, VB>;
+  constexpr int THREADS = Cfg<KB, VB>::THREADS, STAGE_TOK = Cfg<KB, VB>::STAGE_TOK;
+  constexpr int NSTAGE = Cfg<KB, VB>::NSTAGE, WARPS = Cfg<KB, VB>::W;
+  static_assert(Lay::LUT_BYTES == Lut::BYTES && Lut::K_BYTES + Lut::V_BYTES <= Lut::BYTES, "pair tables");
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* lutK = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* lutV = lutK + Lay::LUT_K;
   unsigned char* pipe = smem + Lay::LUT_BYTES;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, t = lane & 3;
+  const int gq = lane >> 2, t = lane & 3;
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / a.hgroups, hg = blockIdx.y % a.hgroups;
   const int b = blockIdx.z;
@@ -432,54 +514,72 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
   }
 
   // Pair tables: entry e = lo | hi << B  ->  half2(c[lo], c[hi]), replicated per lane (bank = lane).
-  for (int i = tid; i < Lay::LUT_K; i += THREADS) {
-    const int e = i >> 5;
-    lutK[i] = pack_half2(a.kc[e & ((1 << KB) - 1)], a.kc[e >> KB]);
+  if constexpr (Lut::kPacked) {
+    for (int i = tid; i < 256 * 64; i += THREADS) {
+      const int e = i >> 6, half = (i >> 5) & 1, ln = i & 31;
+      const float* c = half ? a.vc : a.kc;
+      *reinterpret_cast<uint32_t*>(smem + e * 256 + half * 128 + 4 * ln) = pack_half2(c[e & 15], c[e >> 4]);
+    }
+  } else {
+    for (int i = tid; i < Lut::K_BYTES / 4; i += THREADS) {
+      const int e = i >> 5;
+      reinterpret_cast<uint32_t*>(smem)[i] = pack_half2(a.kc[e & ((1 << KB) - 1)], a.kc[e >> KB]);
+    }
+    for (int i = tid; i < Lut::V_BYTES / 4; i += THREADS) {
+      const int e = i >> 5;
+      reinterpret_cast<uint32_t*>(smem + Lut::K_BYTES)[i] = pack_half2(a.vc[e & ((1 << VB) - 1)], a.vc[e >> VB]);
+    }
   }
-  for (int i = tid; i < Lay::LUT_V; i += THREADS) {
-    const int e = i >> 5;
-    lutV[i] = pack_half2(a.vc[e & ((1 << VB) - 1)], a.vc[e >> VB]);
-  }
+  Lut L;
+  L.base = smem_u32(smem);
+  L.lane4 = 4u * (uint32_t)lane;
 
   // Everything above reads only the cache; the rotated queries come from the prep kernel.
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
-  // A fragments: rows 0-7 = hi parts of the group's heads, rows 8-15 = lo parts (q' and S q').
-  uint32_t aq[8][4], asq[8][4];
-  {
-    const bool live = gid < nh;
-    const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? gid : 0)) * D;
-    const float* sp = a.sq + ((int64_t)b * a.Hq + h0 + (live ? gid : 0)) * D;
+  // B operands: column gq of n-block nb = head 4 nb + gq/2, part gq%2 (0: fp16 hi, 1: fp16 lo);
+  // k-step kk: dims 16kk + 2t, +1 (reg 0) and 16kk + 8 + 2t, +1 (reg 1).
+  uint32_t bq[NB][8][2], bsq[NB][8][2];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int hh = 4 * nb + (gq >> 1);
+    const bool live = hh < nh;
+    const bool lo = gq & 1;
+    const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
+    const float* sp = a.sq + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int c0 = 16 * kk + 8 * half + 2 * t;
-        float x0 = live ? qp[c0] : 0.0f, x1 = live ? qp[c0 + 1] : 0.0f;
-        float h0f, l0f, h1f, l1f;
-        split_half(x0, h0f, l0f);
-        split_half(x1, h1f, l1f);
-        aq[kk][2 * half + 0] = pack_half2(h0f, h1f);
-        aq[kk][2 * half + 1] = pack_half2(l0f, l1f);
+      for (int r = 0; r < 2; ++r) {
+        const int c0 = 16 * kk + 8 * r + 2 * t;
+        float hx, lx, hy, ly;
+        split_half(live ? qp[c0] : 0.0f, hx, lx);
+        split_half(live ? qp[c0 + 1] : 0.0f, hy, ly);
+        bq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
         if constexpr (QJL) {
-          const float s0 = live ? sp[c0] : 0.0f, s1 = live ? sp[c0 + 1] : 0.0f;
-          split_half(s0, h0f, l0f);
-          split_half(s1, h1f, l1f);
-          asq[kk][2 * half + 0] = pack_half2(h0f, h1f);
-          asq[kk][2 * half + 1] = pack_half2(l0f, l1f);
+          split_half(live ? sp[c0] : 0.0f, hx, lx);
+          split_half(live ? sp[c0 + 1] : 0.0f, hy, ly);
+          bsq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
         } else {
-          asq[kk][2 * half + 0] = asq[kk][2 * half + 1] = 0u;
+          bsq[nb][kk][r] = 0u;
         }
       }
     }
   }
 
-  float oacc[16][4];
+  // Output accumulators: n-block nb, dim block db: (dim 16db + gq, head 4nb + t) hi/lo in [0]/[1],
+  // (dim 16db + 8 + gq) in [2]/[3].
+  float oacc[NB][8][4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
-  float m_run = -INFINITY, l_run = 0.0f;
-  const uint32_t* lutK_lane = lutK + lane;  // replica of this lane: bank = lane
-  const uint32_t* lutV_lane = lutV + lane;
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) oacc[nb][i][0] = oacc[nb][i][1] = oacc[nb][i][2] = oacc[nb][i][3] = 0.0f;
+  float m_run[NB], l_run[NB];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    m_run[nb] = -INFINITY;
+    l_run[nb] = 0.0f;
+  }
 
   for (int st = 0; st < nstages; ++st) {
     cp_wait<NSTAGE - 2>();
@@ -495,100 +595,116 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
     const int wtok0 = st * STAGE_TOK + 16 * warp;  // first token of this warp, relative to range
     if (wtok0 >= ntok) continue;                    // warp-uniform
     const unsigned char* stage = pipe + (st % NSTAGE) * Lay::STAGE_BYTES;
+    const int r0 = 16 * warp + gq, r1 = r0 + 8;    // this lane's token rows in the stage
 
-    // ---- scores: S = Q' Khat^T (16 rows x 8 tokens per n-block) ----
-    float kacc[2][4], qacc[2][4];
+    // ---- scores for tokens r0, r1 and heads 4nb + t ----
+    float kacc[NB][4], qacc[NB][4];
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
+    for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
       for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = 0.0f;
-      const int r = 16 * warp + 8 * nb + gid;
-      uint32_t ck[KB];
-      const uint32_t* kw = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r * Lay::K_ROW + 4 * KB * t);
+    {
+      uint32_t c0[KB], c1[KB];
+      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r0 * Lay::K_ROW + 4 * KB * t);
+      const uint32_t* k1 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r1 * Lay::K_ROW + 4 * KB * t);
 #pragma unroll
-      for (int i = 0; i < KB; ++i) ck[i] = kw[i];
-#define TQ_KSTEP(KK)                                                                      \
-      mma16816(kacc[nb], aq[KK], lutK_lane[k_pair_index<KB, 2 * (KK)>(ck) * 32],          \
-               lutK_lane[k_pair_index<KB, 2 * (KK) + 1>(ck) * 32]);
+      for (int i = 0; i < KB; ++i) {
+        c0[i] = k0[i];
+        c1[i] = k1[i];
+      }
+#define TQ_KSTEP(KK)                                                                         \
+      {                                                                                      \
+        const uint32_t A[4] = {k_pair<KB, VB, 2 * (KK)>(L, c0), k_pair<KB, VB, 2 * (KK)>(L, c1), \
+                               k_pair<KB, VB, 2 * (KK) + 1>(L, c0),                          \
+                               k_pair<KB, VB, 2 * (KK) + 1>(L, c1)};                         \
+        _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                    \
+            mma16816(kacc[nb], A, bq[nb][KK][0], bq[nb][KK][1]);                              \
+      }
       TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
 #undef TQ_KSTEP
-      if constexpr (QJL) {
-        const uint32_t sw = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r * 16 + 4 * t);
-#define TQ_SSTEP(KK) \
-        mma16816(qacc[nb], asq[KK], sign_pair<2 * (KK)>(sw), sign_pair<2 * (KK) + 1>(sw));
-        TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
+    }
+    if constexpr (QJL) {
+      const uint32_t s0 = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r0 * 16 + 4 * t);
+      const uint32_t s1 = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r1 * 16 + 4 * t);
+#define TQ_SSTEP(KK)                                                                         \
+      {                                                                                      \
+        const uint32_t A[4] = {sign_pair<2 * (KK)>(s0), sign_pair<2 * (KK)>(s1),             \
+                               sign_pair<2 * (KK) + 1>(s0), sign_pair<2 * (KK) + 1>(s1)};    \
+        _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                    \
+            mma16816(qacc[nb], A, bsq[nb][KK][0], bsq[nb][KK][1]);                            \
+      }
+      TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
 #undef TQ_SSTEP
-      }
     }
 
-    // ---- online softmax (log2 units); this lane owns head gid, tokens 2t, 2t+1 (+8) ----
-    float sc[2][2], pv[2][2];
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      const int tl = 16 * warp + 8 * nb + 2 * t;  // token within the stage
-      const float2 nk = *reinterpret_cast<const float2*>(stage + Lay::OFF_NK + 4 * tl);
-      float2 rn = make_float2(0.f, 0.f);
-      if constexpr (QJL) rn = *reinterpret_cast<const float2*>(stage + Lay::OFF_RN + 4 * tl);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float n = e ? nk.y : nk.x;
-        const float rr = e ? rn.y : rn.x;
-        float s = (kacc[nb][e] + kacc[nb][2 + e]) * (n * a.sK);
-        if constexpr (QJL) s = fmaf(qacc[nb][e] + qacc[nb][2 + e], rr * a.sQ, s);
-        const bool valid = (st * STAGE_TOK + tl + e) < ntok;
-        sc[nb][e] = valid ? s : -INFINITY;
-      }
+    // ---- online softmax (log2 units) per head 4nb + t over this warp's 16 tokens ----
+    const float nk0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r0);
+    const float nk1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r1);
+    float rn0 = 0.0f, rn1 = 0.0f;
+    if constexpr (QJL) {
+      rn0 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r0);
+      rn1 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r1);
     }
-    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const bool grow = m_new > m_run;
-    if (__any_sync(FULL, grow)) {
-      const float alpha = grow ? ex2(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
+    const float nv0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r0) * 0.08838834764831845f;
+    const float nv1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r1) * 0.08838834764831845f;
+    const bool v0ok = wtok0 + gq < ntok, v1ok = wtok0 + 8 + gq < ntok;
+    uint32_t bp[NB][2];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        oacc[i][0] *= alpha;
-        oacc[i][1] *= alpha;
-        oacc[i][2] *= alpha;
-        oacc[i][3] *= alpha;
+    for (int nb = 0; nb < NB; ++nb) {
+      float s0 = (kacc[nb][0] + kacc[nb][1]) * (nk0 * a.sK);
+      float s1 = (kacc[nb][2] + kacc[nb][3]) * (nk1 * a.sK);
+      if constexpr (QJL) {
+        s0 = fmaf(qacc[nb][0] + qacc[nb][1], rn0 * a.sQ, s0);
+        s1 = fmaf(qacc[nb][2] + qacc[nb][3], rn1 * a.sQ, s1);
       }
-      l_run *= alpha;
-      m_run = m_new;
-    }
-    uint32_t ap[4];
+      s0 = v0ok ? s0 : -INFINITY;
+      s1 = v1ok ? s1 : -INFINITY;
+      float mx = fmaxf(s0, s1);
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+      const float m_new = fmaxf(m_run[nb], mx);
+      if (m_new > m_run[nb]) {  // uniform over the 8 lanes of head 4nb + t
+        const float alpha = ex2(m_run[nb] - m_new);  // ex2(-inf) = 0
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      const int tl = 16 * warp + 8 * nb + 2 * t;
-      const float2 nv = *reinterpret_cast<const float2*>(stage + Lay::OFF_NV + 4 * tl);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float p = (m_run == -INFINITY) ? 0.0f : ex2(sc[nb][e] - m_run);
-        l_run += p;
-        pv[nb][e] = p * (e ? nv.y : nv.x) * 0.08838834764831845f;  // p * nV / sqrt(128)
+        for (int i = 0; i < 8; ++i) {
+          oacc[nb][i][0] *= alpha;
+          oacc[nb][i][1] *= alpha;
+          oacc[nb][i][2] *= alpha;
+          oacc[nb][i][3] *= alpha;
+        }
+        l_run[nb] *= alpha;
+        m_run[nb] = m_new;
       }
-      float h0f, l0f, h1f, l1f;
-      split_half(pv[nb][0], h0f, l0f);
-      split_half(pv[nb][1], h1f, l1f);
-      ap[2 * nb + 0] = pack_half2(h0f, h1f);  // rows gid   : hi
-      ap[2 * nb + 1] = pack_half2(l0f, l1f);  // rows gid+8 : lo
+      const float p0 = m_run[nb] == -INFINITY ? 0.0f : ex2(s0 - m_run[nb]);
+      const float p1 = m_run[nb] == -INFINITY ? 0.0f : ex2(s1 - m_run[nb]);
+      l_run[nb] += p0 + p1;
+      // P~ = p nV / sqrt(d) as fp16 hi + lo: row token, columns (head t, hi) and (head t, lo)
+      float hx, lx, hy, ly;
+      split_half(p0 * nv0, hx, lx);
+      split_half(p1 * nv1, hy, ly);
+      bp[nb][0] = movmatrix_trans(pack_half2(hx, lx));  // tokens 2t, 2t+1 of column gq
+      bp[nb][1] = movmatrix_trans(pack_half2(hy, ly));  // tokens 2t+8, 2t+9
     }
 
-    // ---- O' += P Vhat: 16 n-blocks of 8 dims; B holds token pairs (2t,2t+1), (2t+8,2t+9) ----
+    // ---- O'^T += Vhat^T P~: dim blocks of 16; A holds token pairs (2t,2t+1), (2t+8,2t+9) ----
     {
       const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
-      const uint64_t cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gid);
-      const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gid);
-      const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gid);
-      const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gid);
+      const uint64_t cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
+      const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
+      const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
+      const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
       VPairs<VB> p01, p89;
       p01.build(cv0, cv1);
       p89.build(cv2, cv3);
-#define TQ_VSTEP(NU)                                                                        \
-      mma16816(oacc[NU], ap, lutV_lane[p01.template index<NU>() * 32],                      \
-               lutV_lane[p89.template index<NU>() * 32]);
+#define TQ_VSTEP(DB)                                                                          \
+      {                                                                                       \
+        const uint32_t A[4] = {v_pair<KB, VB, 2 * (DB)>(L, p01), v_pair<KB, VB, 2 * (DB) + 1>(L, p01), \
+                               v_pair<KB, VB, 2 * (DB)>(L, p89), v_pair<KB, VB, 2 * (DB) + 1>(L, p89)}; \
+        _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                     \
+            mma16816(oacc[nb][DB], A, bp[nb][0], bp[nb][1]);                                   \
+      }
       TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3) TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
-      TQ_VSTEP(8) TQ_VSTEP(9) TQ_VSTEP(10) TQ_VSTEP(11) TQ_VSTEP(12) TQ_VSTEP(13) TQ_VSTEP(14) TQ_VSTEP(15)
 #undef TQ_VSTEP
     }
   }
@@ -599,37 +715,42 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
   float* mw = reinterpret_cast<float*>(pipe);  // [WARPS][HG]
   float* lw = mw + WARPS * HG;                 // [WARPS][HG]
   float* ow = lw + WARPS * HG;                 // [WARPS][HG][D]
-  float lq = l_run;
-  lq += __shfl_xor_sync(FULL, lq, 1);
-  lq += __shfl_xor_sync(FULL, lq, 2);
-  if (t == 0) {
-    mw[warp * HG + gid] = m_run;
-    lw[warp * HG + gid] = lq;
-  }
 #pragma unroll
-  for (int nu = 0; nu < 16; ++nu) {
-    float* o = ow + (warp * HG + gid) * D + 8 * nu + 2 * t;
-    o[0] = oacc[nu][0] + oacc[nu][2];
-    o[1] = oacc[nu][1] + oacc[nu][3];
+  for (int nb = 0; nb < NB; ++nb) {
+    const int hh = 4 * nb + t;
+    float lq = l_run[nb];
+    lq += __shfl_xor_sync(FULL, lq, 4);
+    lq += __shfl_xor_sync(FULL, lq, 8);
+    lq += __shfl_xor_sync(FULL, lq, 16);
+    if (gq == 0) {
+      mw[warp * HG + hh] = m_run[nb];
+      lw[warp * HG + hh] = lq;
+    }
+    float* o = ow + (warp * HG + hh) * D;
+#pragma unroll
+    for (int db = 0; db < 8; ++db) {
+      o[16 * db + gq] = oacc[nb][db][0] + oacc[nb][db][1];
+      o[16 * db + 8 + gq] = oacc[nb][db][2] + oacc[nb][db][3];
+    }
   }
   __syncthreads();
-  for (int r = 0; r < nh; ++r) {
+  for (int r = 0; r < nh && tid < D; ++r) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) M = fmaxf(M, mw[w * HG + r]);
-    float L = 0.0f, O = 0.0f;
+    float Ls = 0.0f, O = 0.0f;
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) {
       const float mwr = mw[w * HG + r];
       const float f = (mwr == -INFINITY) ? 0.0f : ex2(mwr - M);
-      L += f * lw[w * HG + r];
+      Ls += f * lw[w * HG + r];
       O += f * ow[(w * HG + r) * D + tid];
     }
     float* dst = a.part + (((int64_t)b * a.Hq + h0 + r) * a.splits + split) * PART;
     dst[2 + tid] = O;
     if (tid == 0) {
       dst[0] = M;
-      dst[1] = L;
+      dst[1] = Ls;
     }
   }
 
@@ -644,7 +765,7 @@ __global__ void __launch_bounds__(THREADS, 2) split_kernel(DArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  merge_splits(a, b, h0, nh, pipe);
+  merge_splits<WARPS>(a, b, h0, nh, pipe);
 }
 
 // ------------------------------------------------------------------------------------------ host
@@ -666,7 +787,13 @@ int device_sms() {
   return sms;
 }
 
-Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
+// Resident split CTAs per SM: the 4-bit pair tables (64 KB) allow two, the smaller ones three
+// (register-bound, see split_kernel's launch bounds).
+int resident_ctas(int kb, int vb) { return (kb == 4 && vb == 4) ? 2 : 3; }
+// (two six-warp CTAs with the 4-bit tables, three four-warp CTAs otherwise)
+
+Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms, int resident, int stage_tok) {
+  const int STAGE_TOK = stage_tok;
   Plan p;
   const int g = Hq / Hkv;
   p.hgroups = (g + HG - 1) / HG;
@@ -676,8 +803,8 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
     p.tps = STAGE_TOK;
     return p;
   }
-  // One wave of 2 resident CTAs per SM: the largest split count whose grid still fits it.
-  const int64_t slots = 2LL * sms;
+  // One wave of resident CTAs: the largest split count whose grid still fits it.
+  const int64_t slots = (int64_t)resident * sms;
   int64_t splits = slots / units;
   const int64_t max_splits = (seq_len + 4 * STAGE_TOK - 1) / (4 * STAGE_TOK);  // >= 4 stages each
   if (splits > max_splits) splits = max_splits;
@@ -696,16 +823,16 @@ size_t workspace_bytes(int B, int Hq, int Hkv, const Plan& p) {
          sizeof(int) * (size_t)B * Hkv * p.hgroups;
 }
 
-template <int KB, int VB, bool QJL>
-tq_status launch_split(const DArgs& a, dim3 grid, cudaStream_t stream) {
+template <int KB, int VB, bool QJL, int NB>
+tq_status launch_split_nb(const DArgs& a, dim3 grid, cudaStream_t stream) {
   using Lay = Layout<KB, VB, QJL>;
-  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL>,
+  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
   // programmatic dependent launch: the prologue (tables, first cache stages) overlaps prep
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(THREADS);
+  cfg.blockDim = dim3(Cfg<KB, VB>::THREADS);
   cfg.dynamicSmemBytes = Lay::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -713,9 +840,15 @@ tq_status launch_split(const DArgs& a, dim3 grid, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL>, a);
+  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL, NB>, a);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "split launch: %s", cudaGetErrorString(e));
   return TQ_OK;
+}
+
+// One n-block of four heads when a group has at most four query heads, else two.
+template <int KB, int VB, bool QJL>
+tq_status launch_split(const DArgs& a, dim3 grid, cudaStream_t stream) {
+  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1>(a, grid, stream) : launch_split_nb<KB, VB, QJL, 2>(a, grid, stream);
 }
 
 template <int KB, bool QJL>
@@ -742,7 +875,8 @@ tq_status dispatch(int kb, int vb, const DArgs& a, dim3 grid, cudaStream_t s) {
 extern "C" size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_len) {
   using namespace tq;
   if (!cache || B < 1 || Hq < 1 || cache->Hkv < 1 || Hq % cache->Hkv || seq_len < 0) return 0;
-  const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
+  const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms(),
+                           resident_ctas(cache->k_bits, cache->v_bits), stage_tokens(cache->k_bits, cache->v_bits));
   return workspace_bytes(B, Hq, cache->Hkv, p);
 }
 
@@ -763,7 +897,8 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
     return fail(TQ_ERR_INVALID_ARG, "q / out / workspace must be 16-byte aligned");
   const int B = cache->B;
-  const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
+  const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms(),
+                              resident_ctas(cache->k_bits, cache->v_bits), stage_tokens(cache->k_bits, cache->v_bits));
   const size_t need = workspace_bytes(B, Hq, cache->Hkv, plan);
   if (ws_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
