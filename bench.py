@@ -30,8 +30,6 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
-KERNEL_SOURCES = {"tq_quantize": "decode_attention_11_b200/csrc/tq_quantize.cu",
-                  "tq_decode_attn": "decode_attention_11_b200/csrc/tq_decode.cu"}
 
 
 def source_digest(rel: str) -> str:
@@ -52,7 +50,7 @@ def dram_traffic(kernel: str, workload: str, batch, context):
     for e in table.get("captures", []):
         if e["api"] != kernel or e["workload"] != workload or context is not None:
             continue
-        if source_digest(KERNEL_SOURCES[kernel]) != e["source_sha256"]:
+        if source_digest(e["source"]) != e["source_sha256"]:
             return None, "kernel changed since the capture"
         full_b = W.CONFIGS[workload].B
         b = batch if batch is not None else full_b
