@@ -300,6 +300,9 @@ def run_gpu(args, w):
     t_all0 = torch.cuda.Event(enable_timing=True)
     t_all1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        # a short device-side delay ahead of the timed region lets the host queue the first steps,
+        # so that no host launch latency lands between a step's events
+        torch.cuda._sleep(2_000_000)
         t_all0.record(stream)
         for i in range(args.steps):
             step(evs[i])

@@ -37,7 +37,7 @@ EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codeboo
             "tq_quantize", "tq_quantize_device_errors", "tq_quantize_vector_fixups",
             "tq_quantize_code_fixups",
             "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
-            "tq_decode_static_workspace_limit")
+            "tq_decode_static_workspace_limit", "tq_sketch_rotation")
 
 
 class TqError(RuntimeError):
@@ -58,7 +58,8 @@ class _Cache(ctypes.Structure):
 class _Params(ctypes.Structure):
     _fields_ = [("Pi", ctypes.c_void_p), ("S", ctypes.c_void_p),
                 ("k_centroids", ctypes.c_void_p), ("k_thresholds", ctypes.c_void_p),
-                ("v_centroids", ctypes.c_void_p), ("v_thresholds", ctypes.c_void_p)]
+                ("v_centroids", ctypes.c_void_p), ("v_thresholds", ctypes.c_void_p),
+                ("S_Pi", ctypes.c_void_p)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -104,6 +105,9 @@ def lib() -> ctypes.CDLL:
                                         ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
     L.tq_decode_static_workspace_limit.restype = ctypes.c_size_t
     L.tq_decode_static_workspace_limit.argtypes = []
+    L.tq_sketch_rotation.restype = ctypes.c_int
+    L.tq_sketch_rotation.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                     ctypes.c_void_p]
     _lib = L
     return L
 
@@ -149,6 +153,17 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream if stream.cuda_stream else None
 
 
+def sketch_rotation_product(Pi: torch.Tensor, S: torch.Tensor, stream=None) -> torch.Tensor:
+    """S Pi in fp64 on the device of Pi (tq_sketch_rotation), for Params.S_Pi."""
+    assert Pi.is_cuda and S.is_cuda and Pi.dtype == torch.float32 and S.dtype == torch.float32
+    Pi = Pi.contiguous()
+    S = S.contiguous()
+    out = torch.empty(S.shape[0], 128, dtype=torch.float64, device=Pi.device)
+    _check(lib().tq_sketch_rotation(Pi.data_ptr(), S.data_ptr(), int(S.shape[0]), out.data_ptr(),
+                                    _stream_ptr(stream)))
+    return out
+
+
 @dataclasses.dataclass
 class Params:
     """Per-layer constants on the device (fp32): rotation, sketch, codebooks."""
@@ -159,17 +174,24 @@ class Params:
     k_thresholds: torch.Tensor
     v_centroids: torch.Tensor
     v_thresholds: torch.Tensor
+    S_Pi: Optional[torch.Tensor] = None
 
     @classmethod
-    def create(cls, Pi, S, k_bits: int, v_bits: int, device="cuda") -> "Params":
+    def create(cls, Pi, S, k_bits: int, v_bits: int, device="cuda", sketch_rotation=True) -> "Params":
+        """Upload the constants; with a sketch, also S Pi in fp64 (tq_sketch_rotation) unless
+        `sketch_rotation` is False."""
         kc, kt, _ = build_codebook(k_bits)
         vc, vt, _ = build_codebook(v_bits)
         f = lambda x: torch.as_tensor(np.ascontiguousarray(x, dtype=np.float32)).to(device)
-        return cls(f(Pi), None if S is None else f(S), f(kc), f(kt), f(vc), f(vt))
+        p = cls(f(Pi), None if S is None else f(S), f(kc), f(kt), f(vc), f(vt))
+        if p.S is not None and sketch_rotation and p.Pi.is_cuda:
+            p.S_Pi = sketch_rotation_product(p.Pi, p.S)
+        return p
 
     def as_c(self) -> _Params:
         return _Params(_ptr(self.Pi), _ptr(self.S), _ptr(self.k_centroids),
-                       _ptr(self.k_thresholds), _ptr(self.v_centroids), _ptr(self.v_thresholds))
+                       _ptr(self.k_thresholds), _ptr(self.v_centroids), _ptr(self.v_thresholds),
+                       _ptr(self.S_Pi))
 
 
 @dataclasses.dataclass

@@ -51,8 +51,8 @@ tq_status check_params(const tq_params* p, const tq_cache* c) {
   if (!p->Pi || !p->k_centroids || !p->k_thresholds || !p->v_centroids || !p->v_thresholds)
     return fail(TQ_ERR_INVALID_ARG, "params array is NULL");
   if (c->qjl_m && !p->S) return fail(TQ_ERR_INVALID_ARG, "S is NULL with qjl_m=%d", c->qjl_m);
-  if (!aligned16(p->Pi) || (c->qjl_m && !aligned16(p->S)))
-    return fail(TQ_ERR_INVALID_ARG, "Pi / S must be 16-byte aligned");
+  if (!aligned16(p->Pi) || (c->qjl_m && !aligned16(p->S)) || !aligned16(p->S_Pi))
+    return fail(TQ_ERR_INVALID_ARG, "Pi / S / S_Pi must be 16-byte aligned");
   return TQ_OK;
 }
 

@@ -787,8 +787,37 @@ tq_status launch(int kb, int vb, const QArgs& a, int sms, cudaStream_t s) {
 #undef TQ_V
 }
 
+// S_Pi = S Pi in fp64: block l, thread j; products of fp32 values are exact in fp64 and are
+// summed in ascending i.
+__global__ void __launch_bounds__(kHeadDim) sketch_rotation_kernel(const float* __restrict__ Pi,
+                                                                   const float* __restrict__ S,
+                                                                   double* __restrict__ S_Pi) {
+  __shared__ double srow[kHeadDim];
+  const int l = blockIdx.x, j = threadIdx.x;
+  srow[j] = (double)S[(int64_t)l * kHeadDim + j];
+  __syncthreads();
+  double acc = 0.0;
+#pragma unroll 8
+  for (int i = 0; i < kHeadDim; ++i) acc = fma(srow[i], (double)Pi[i * kHeadDim + j], acc);
+  S_Pi[(int64_t)l * kHeadDim + j] = acc;
+}
+
 }  // namespace
 }  // namespace tq
+
+extern "C" tq_status tq_sketch_rotation(const float* Pi, const float* S, int qjl_m, double* S_Pi,
+                                        void* stream) {
+  using namespace tq;
+  clear_error();
+  if (!Pi || !S || !S_Pi) return fail(TQ_ERR_INVALID_ARG, "Pi / S / S_Pi is NULL");
+  if (!aligned16(Pi) || !aligned16(S) || !aligned16(S_Pi))
+    return fail(TQ_ERR_INVALID_ARG, "Pi / S / S_Pi must be 16-byte aligned");
+  if (qjl_m < 1) return fail(TQ_ERR_INVALID_ARG, "qjl_m %d < 1", qjl_m);
+  sketch_rotation_kernel<<<qjl_m, kHeadDim, 0, reinterpret_cast<cudaStream_t>(stream)>>>(Pi, S, S_Pi);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "sketch rotation launch: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}
 
 extern "C" tq_status tq_quantize(const tq_params* params, const void* k, const void* v, int dtype,
                                  int64_t stride_b, int64_t stride_h, int64_t stride_t, int T_new,

@@ -101,12 +101,17 @@ typedef struct {
   float* v_norm;
 } tq_cache;
 
-/* Per-layer constants (device pointers, caller-owned, fp32).
+/* Per-layer constants (device pointers, caller-owned, fp32 unless stated).
  *   Pi            [128 x 128] row-major orthogonal rotation (u = sqrt(128) Pi x / ||x||)
  *   S             [qjl_m x 128] row-major Gaussian sketch, entries exactly representable in fp16
  *                 (may be NULL when qjl_m == 0)
  *   k_centroids   [1 << k_bits], k_thresholds [(1 << k_bits) - 1]  from tq_build_codebook
- *   v_centroids   [1 << v_bits], v_thresholds [(1 << v_bits) - 1] */
+ *   v_centroids   [1 << v_bits], v_thresholds [(1 << v_bits) - 1]
+ *   S_Pi          optional float64 [qjl_m x 128] row-major product S Pi, as written by
+ *                 tq_sketch_rotation for these S and Pi; NULL is allowed.  It changes no output:
+ *                 with it, tq_quantize settles a sketch value that lies near 0 with one
+ *                 length-128 dot product (S r = sqrt(128)/||x|| (S Pi) x - S c[idx]) instead of
+ *                 re-rotating the whole key in fp64. */
 typedef struct {
   const float* Pi;
   const float* S;
@@ -114,7 +119,17 @@ typedef struct {
   const float* k_thresholds;
   const float* v_centroids;
   const float* v_thresholds;
+  const double* S_Pi;
 } tq_params;
+
+/*
+ * S_Pi[l][j] = sum_i S[l][i] Pi[i][j] in float64 (device; every product of two fp32 values is
+ * exact in fp64, summed in ascending i), for tq_params.S_Pi.  Enqueued on `stream`.
+ *   Pi      device fp32 [128 x 128];  S  device fp32 [qjl_m x 128];  S_Pi  device fp64 [qjl_m x 128]
+ *   qjl_m   >= 1
+ * Errors: TQ_ERR_INVALID_ARG (NULL or misaligned pointer, qjl_m < 1), TQ_ERR_CUDA.
+ */
+tq_status tq_sketch_rotation(const float* Pi, const float* S, int qjl_m, double* S_Pi, void* stream);
 
 /*
  * Compress T_new new tokens of K and V into cache rows [t_offset, t_offset + T_new).
@@ -127,6 +142,9 @@ typedef struct {
  *   T_new       >= 0 (0 enqueues nothing);  0 <= t_offset, t_offset + T_new <= cache->T_cap
  * Output bits are those of the float64 definition except where a rotated coordinate lies within
  * about 1e-15 of a threshold (the kernel re-derives near-boundary cases in fp64).
+ * TQ_BF16 calls on one device share a file-scope device queue of those fp64 re-derivations:
+ * calls whose device work may overlap (different streams without ordering, or host threads
+ * racing on one device) corrupt each other's results; order them on one stream.
  * Errors: TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA.
  */
 tq_status tq_quantize(const tq_params* params, const void* k, const void* v, int dtype,

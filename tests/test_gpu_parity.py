@@ -107,6 +107,41 @@ def test_quantize_strided_input():
     compare_quantized(w, cache, Kh, Vh, 0)
 
 
+def test_sketch_rotation_product():
+    """tq_sketch_rotation against the float64 matrix product of the same fp32 S and Pi."""
+    w = small("llama3_8b_32k")
+    Pi, S = W.rotation_for(w), W.qjl_for(w)
+    got = tq.sketch_rotation_product(torch.as_tensor(Pi, dtype=torch.float32).cuda(),
+                                     torch.as_tensor(S, dtype=torch.float32).cuda()).cpu().numpy()
+    want = np.asarray(S, np.float32).astype(np.float64) @ np.asarray(Pi, np.float32).astype(np.float64)
+    assert got.dtype == np.float64 and got.shape == want.shape
+    assert np.max(np.abs(got - want)) <= 1e-13 * np.max(np.abs(want))
+
+
+def test_quantize_sign_fixups_with_and_without_sketch_rotation():
+    """Signs near 0 settled through S Pi (params.S_Pi) or by re-rotating the key give the same
+    cache, and both match the oracle; enough rows that both paths run."""
+    w = W.CONFIGS["llama3_8b_128k_b4"].scaled(T=8192, B=1, Hkv=2, Hq=8)
+    K, V, Kh, Vh = gpu_inputs(w)
+    caches = []
+    for with_spi in (True, False):
+        params = tq.Params.create(W.rotation_for(w), W.qjl_for(w), w.k_bits, w.v_bits,
+                                  sketch_rotation=with_spi)
+        assert (params.S_Pi is not None) == with_spi
+        cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+        v0 = tq.quantize_vector_fixups()
+        tq.quantize(params, K, V, cache)
+        torch.cuda.synchronize()
+        assert tq.quantize_device_errors() == 0
+        assert tq.quantize_vector_fixups() > v0
+        caches.append(cache)
+    a, b = caches
+    for x, y in zip((a.k_codes, a.k_signs, a.k_norm, a.k_rnorm, a.v_codes, a.v_norm),
+                    (b.k_codes, b.k_signs, b.k_norm, b.k_rnorm, b.v_codes, b.v_norm)):
+        assert torch.equal(x, y)
+    compare_quantized(w, a, Kh, Vh, 0)
+
+
 def decode_on_oracle_cache(w, seq_lens, scale=None, q_dtype=torch.float32):
     K, V, Kh, Vh = gpu_inputs(w)
     q = W.make_queries(w)
