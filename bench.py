@@ -115,6 +115,7 @@ class ClockSampler:
                     started.set()
                     if self._stop.is_set():
                         break  # one last sample after the region ends
+                    time.sleep(0.0005)  # releases the interpreter lock for the launching thread
 
             self._thread = threading.Thread(target=run, daemon=True)
             self._thread.start()
@@ -280,14 +281,35 @@ def run_gpu(args, w):
         for s in range(0, w.T, w.chunk):
             tq.quantize(params, K[:, :, s:s + w.chunk], V[:, :, s:s + w.chunk], cache, t_offset=s)
 
+    def decode():
+        tq.decode_attn(params, q, cache, w.T, out=out, workspace=ws)
+
+    # Each op is captured once into a CUDA graph and replayed per step, so that host launch
+    # latency (the moe workload makes 128 quantize calls per step) stays out of the device timing.
+    run_q, run_d = quantize_all, decode
+    if not args.no_graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):  # warm-up outside capture (function attributes, tensor maps)
+            quantize_all()
+            decode()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        gq, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gq):
+            quantize_all()
+        with torch.cuda.graph(gd):
+            decode()
+        run_q, run_d = gq.replay, gd.replay
+
     def step(ev):
         flush.zero_()
         ev[0].record(stream)
-        quantize_all()
+        run_q()
         ev[1].record(stream)
         flush.zero_()
         ev[2].record(stream)
-        tq.decode_attn(params, q, cache, w.T, out=out, workspace=ws)
+        run_d()
         ev[3].record(stream)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -385,7 +407,8 @@ def run_gpu(args, w):
         "value": dec_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16 mma / f32 accumulate (decode); f32+f64 (quantize)",
-        "data": "synthetic", "config": workload_config(w, parallelism=f"replicas x{world}"),
+        "data": "synthetic", "config": workload_config(w, parallelism=f"replicas x{world}",
+                                                      launch="direct" if args.no_graph else "cuda graph per op"),
         "decode_hbm_frac": dec_frac, "decode_ms": sum(d_ms) / len(d_ms),
         "quantize_tokens_per_s": q_tok_s, "quantize_GBps": q_gbs, "quantize_hbm_frac": q_frac,
         "quantize_ms": sum(q_ms) / len(q_ms),
@@ -411,6 +434,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.CONFIG_ORDER)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every op directly in the timed steps")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--context", type=int, default=None, help="override the workload's context")
     args = ap.parse_args()

@@ -7,7 +7,8 @@
 // Softmax and the value sum also run in the rotated basis; one final o = Pi^T o' per head.
 //
 // Kernels (both on the caller's stream; the second is a programmatic dependent launch):
-//   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace.
+//   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace: clusters of
+//           eight CTAs, each CTA holding 16 rows of Pi and S for a batch of up to 16 heads.
 //   split   grid (splits, Hkv * head_groups, B).  A 4-warp CTA streams its token range through a
 //           4-stage cp.async pipeline (64 tokens per stage).  Each warp takes 16 tokens per stage:
 //           codes are turned into fp16 pairs by a lane-replicated shared-memory table (one load per
@@ -21,6 +22,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "tq_internal.h"
@@ -44,6 +46,7 @@ struct Cfg {
 inline int stage_tokens(int kb, int vb) { return (kb == 4 && vb == 4) ? 96 : 64; }
 constexpr int HG = 8;                  // query heads per MMA row block (hi rows 0-7, lo rows 8-15)
 constexpr int PART = 2 + D;            // (max, sum, o'[128]) per partial
+constexpr int SPLITS_MAX = 512;        // CTAs per (batch, kv-head, head group)
 constexpr unsigned FULL = 0xffffffffu;
 
 struct DArgs {
@@ -195,59 +198,90 @@ __device__ __forceinline__ uint32_t v_code(uint64_t c) {
 
 // ------------------------------------------------------------------------------------------ prep
 
-// One 512-thread block per (batch, query head): q' = Pi q and sq = S q'.  Thread (i, k) forms the
-// partial dot product of row i with elements 32k..32k+31 (eight independent 16-byte loads, so one
-// memory round trip per matrix); block 0 also zeroes the split-completion counters.  The split
-// kernel is launched as a programmatic dependent of this one and starts its prologue early.
-constexpr int PREP_THREADS = 4 * D;
+// Clusters of eight 128-thread CTAs; cluster k handles query heads hb*k .. hb*k + hb - 1 (flattened
+// over the batch; hb <= 16 is chosen on the host so that there are enough clusters to spread the
+// work) and CTA c of it rows 16c .. 16c+15 of q' = Pi q and of sq = S q', eight threads per row
+// with 16 columns each.  Each CTA loads its rows of Pi and S once (one memory round trip,
+// together with the query vectors) and reuses them for all its heads; the full q' of every head
+// reaches the other CTAs of the cluster through distributed shared memory.  CTA 0 also
+// zeroes the split counters.  The split kernel is launched as a programmatic dependent of this
+// one and starts its prologue early.
+constexpr int PREP_CLUSTER = 8, PREP_THREADS = 128, PREP_ROWS = D / PREP_CLUSTER, PREP_HB = 16;
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Shared-memory float at the same offset as `p` in CTA `rank` of this cluster.
+__device__ __forceinline__ float ld_cluster_f32(const float* p, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 template <typename QT>
-__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const QT* __restrict__ q,
-                                                           const float* __restrict__ Pi,
-                                                           const float* __restrict__ S, int qjl,
-                                                           float* __restrict__ qrot,
-                                                           float* __restrict__ sq,
-                                                           int* __restrict__ counters,
-                                                           int n_counters) {
+__global__ void __cluster_dims__(PREP_CLUSTER, 1, 1) __launch_bounds__(PREP_THREADS)
+    prep_kernel(const QT* __restrict__ q, int BH, int hb, const float* __restrict__ Pi, const float* __restrict__ S,
+                int qjl, float* __restrict__ qrot, float* __restrict__ sq, int* __restrict__ counters,
+                int n_counters) {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  __shared__ __align__(16) float qs[D];
-  __shared__ __align__(16) float qr[D];
-  const int tid = threadIdx.x, i = tid >> 2, k = tid & 3;
-  const int64_t bh = blockIdx.x;
+  __shared__ __align__(16) float qs[PREP_HB][D];           // query vectors, then q' of the cluster
+  __shared__ __align__(16) float qpart[PREP_HB][PREP_ROWS];  // this CTA's rows of q'
+  const int tid = threadIdx.x;
+  const uint32_t c = blockIdx.x % PREP_CLUSTER;  // rank in the cluster (clusters are consecutive CTAs)
+  const int h0 = (int)(blockIdx.x / PREP_CLUSTER) * hb;
+  const int nhb = min(hb, BH - h0);
+  const int rl = tid >> 3, part = tid & 7;
+  const int row = PREP_ROWS * (int)c + rl;
   if (blockIdx.x == 0)
-    for (int c = tid; c < n_counters; c += PREP_THREADS) counters[c] = 0;
-  if (tid < D) {
-    if constexpr (sizeof(QT) == 4) qs[tid] = (float)q[bh * D + tid];
-    else qs[tid] = __bfloat162float(q[bh * D + tid]);
+    for (int i = tid; i < n_counters; i += PREP_THREADS) counters[i] = 0;
+  float4 p[4], s4[4];
+  const float4* pr = reinterpret_cast<const float4*>(Pi + row * D + 16 * part);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = pr[i];
+  if (qjl) {
+    const float4* sr = reinterpret_cast<const float4*>(S + row * D + 16 * part);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s4[i] = sr[i];
+  }
+  for (int h = 0; h < nhb; ++h) {
+    if constexpr (sizeof(QT) == 4) qs[h][tid] = (float)q[(int64_t)(h0 + h) * D + tid];
+    else qs[h][tid] = __bfloat162float(q[(int64_t)(h0 + h) * D + tid]);
   }
   __syncthreads();
-  auto dot_row = [&](const float* M, const float* vec) {
-    const float4* row = reinterpret_cast<const float4*>(M + i * D + 32 * k);
-    const float4* v4 = reinterpret_cast<const float4*>(vec + 32 * k);
-    float4 p[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) p[c] = row[c];
+  auto dot16 = [&](const float4 (&m)[4], const float* vec) {
+    const float4* v4 = reinterpret_cast<const float4*>(vec + 16 * part);
     float acc = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float4 x = v4[c];
-      acc = fmaf(p[c].x, x.x, acc);
-      acc = fmaf(p[c].y, x.y, acc);
-      acc = fmaf(p[c].z, x.z, acc);
-      acc = fmaf(p[c].w, x.w, acc);
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = v4[i];
+      acc = fmaf(m[i].x, x.x, acc);
+      acc = fmaf(m[i].y, x.y, acc);
+      acc = fmaf(m[i].z, x.z, acc);
+      acc = fmaf(m[i].w, x.w, acc);
     }
     acc += __shfl_xor_sync(FULL, acc, 1);
     acc += __shfl_xor_sync(FULL, acc, 2);
+    acc += __shfl_xor_sync(FULL, acc, 4);
     return acc;
   };
-  const float v = dot_row(Pi, qs);
-  if (k == 0) {
-    qr[i] = v;
-    qrot[bh * D + i] = v;
+  for (int h = 0; h < nhb; ++h) {
+    const float v = dot16(p, qs[h]);
+    if (part == 0) {
+      qpart[h][rl] = v;
+      qrot[(int64_t)(h0 + h) * D + row] = v;
+    }
   }
-  if (!qjl) return;
-  __syncthreads();
-  const float w = dot_row(S, qr);
-  if (k == 0) sq[bh * D + i] = w;
+  if (!qjl) return;  // uniform over the cluster: no CTA waits at the barriers below
+  cluster_sync_all();
+  for (int h = 0; h < nhb; ++h)
+    qs[h][tid] = ld_cluster_f32(&qpart[h][tid % PREP_ROWS], (uint32_t)(tid / PREP_ROWS));
+  cluster_sync_all();  // every remote read is done before any CTA of the cluster exits
+  for (int h = 0; h < nhb; ++h) {
+    const float w = dot16(s4, qs[h]);
+    if (part == 0) sq[(int64_t)(h0 + h) * D + row] = w;
+  }
 }
 
 // ------------------------------------------------------------------------------------------ split
@@ -268,11 +302,13 @@ struct Layout {
   static constexpr int OFF_NV = OFF_RN + (QJL ? STAGE_TOK * 4 : 0);
   static constexpr int STAGE_BYTES = OFF_NV + STAGE_TOK * 4;
   static constexpr int LUT_BYTES = kPackedLut ? 256 * 256 : ((1 << (2 * KB)) + (1 << (2 * VB))) * 128;
-  // scratch after the pipeline: the CTA's own warp merge, then (last CTA) the split merge
-  static constexpr int MERGE_BYTES = 4 * (2 * HG + HG * D + W * HG * D + W * HG);
-  static_assert(MERGE_BYTES >= 4 * (W * HG * 2 + W * HG * D), "warp merge scratch");
+  // After the main loop the pipeline buffers hold the CTA's own warp merge; the last CTA then
+  // reuses all of shared memory (tables included) for the split merge.
+  static constexpr int WARP_MERGE_BYTES = 4 * (W * HG * 2 + W * HG * D);
+  static constexpr int MERGE_BYTES = 4 * (2 * HG * SPLITS_MAX + HG + W * HG * D + HG * D);
   static constexpr int PIPE_BYTES = NSTAGE * STAGE_BYTES;
-  static constexpr int SMEM = LUT_BYTES + (PIPE_BYTES > MERGE_BYTES ? PIPE_BYTES : MERGE_BYTES);
+  static constexpr int MAIN_BYTES = LUT_BYTES + (PIPE_BYTES > WARP_MERGE_BYTES ? PIPE_BYTES : WARP_MERGE_BYTES);
+  static constexpr int SMEM = MAIN_BYTES > MERGE_BYTES ? MAIN_BYTES : MERGE_BYTES;
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
 };
 
@@ -331,90 +367,105 @@ __device__ __forceinline__ uint64_t load_v_chunk(const unsigned char* row, int g
 
 // Log-sum-exp merge of the split partials of heads h0 .. h0+nh-1 of batch b, then o = Pi^T o'.
 // Run by the last CTA to finish (W warps); partials are read from L2 (written by other CTAs).
+// Every phase issues its loads for all heads and splits at once; the un-rotation keeps the next
+// rows of Pi in flight while the current ones are used.
 template <int W>
-__device__ void merge_splits(const DArgs& a, int b, int h0, int nh, unsigned char* scratch) {
+__device__ void merge_splits(const float* __restrict__ part, const float* __restrict__ Pi,
+                                          float* __restrict__ out, int Hq, int S, int b, int h0, int nh,
+                                          unsigned char* scratch) {
   constexpr int T = 32 * W;
-  const int tid = threadIdx.x;
-  const int S = a.splits;
-  float* Mr = reinterpret_cast<float*>(scratch);  // [HG]
-  float* Lr = Mr + HG;                             // [HG]
-  float* ob = Lr + HG;                             // [HG][D]
-  float* partw = ob + HG * D;                      // [W][HG][D] partial sums over split groups
-  float* lsw = partw + W * HG * D;                 // [W][HG]
-  for (int r = 0; r < nh; ++r) {
-    const float* p = a.part + ((int64_t)b * a.Hq + h0 + r) * S * PART;
-    float m = -INFINITY;
-    for (int s2 = tid; s2 < S; s2 += T) m = fmaxf(m, __ldcg(p + (int64_t)s2 * PART));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-    if ((tid & 31) == 0) ob[tid >> 5] = m;
-    __syncthreads();
-    if (tid == 0) {
-      float M = -INFINITY;
-      for (int w = 0; w < W; ++w) M = fmaxf(M, ob[w]);
-      Mr[r] = M;
-    }
-    __syncthreads();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* wt = reinterpret_cast<float*>(scratch);  // [nh][S]: partial max, then its weight
+  float* ls = wt + HG * SPLITS_MAX;                // [nh][S]: partial sum
+  float* Lr = ls + HG * SPLITS_MAX;                // [HG]
+  float* red = Lr + HG;                            // [W][HG][D]: per-warp sums over splits
+  float* ob = red + W * HG * D;                    // [HG][D]: merged, normalized o'
+  const float* part0 = part + ((int64_t)b * Hq + h0) * S * PART;  // heads are S partials apart
+
+  // phase 1: (max, sum) of every partial
+  for (int idx = tid; idx < nh * S; idx += T) {
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(part0 + (int64_t)idx * PART));
+    wt[idx] = ml.x;
+    ls[idx] = ml.y;
   }
-  // thread = (split group g, 4-dim slice j4): sum over splits s = g (mod W)
-  const int g = tid >> 5, j4 = tid & 31;
-  for (int r = 0; r < nh; ++r) {
-    const float M = Mr[r];
-    const float* p = a.part + ((int64_t)b * a.Hq + h0 + r) * S * PART;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lsum = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll 8
-      for (int s2 = g; s2 < S; s2 += W) {
-        const float* ps = p + (int64_t)s2 * PART;
-        const float ms = __ldcg(ps);
-        const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
-        const float2 lo = __ldcg(reinterpret_cast<const float2*>(ps + 2 + 4 * j4));
-        const float2 hi = __ldcg(reinterpret_cast<const float2*>(ps + 4 + 4 * j4));
-        acc.x = fmaf(f, lo.x, acc.x);
-        acc.y = fmaf(f, lo.y, acc.y);
-        acc.z = fmaf(f, hi.x, acc.z);
-        acc.w = fmaf(f, hi.y, acc.w);
-        if (j4 == 0) lsum = fmaf(f, __ldcg(ps + 1), lsum);
+  __syncthreads();
+  // phase 2: warp r (mod W) turns head r's maxima into weights 2^(m_s - M) and forms L
+  for (int r = warp; r < nh; r += W) {
+    float M = -INFINITY;
+    for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, wt[r * S + s2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
+    float L = 0.0f;
+    for (int s2 = lane; s2 < S; s2 += 32) {
+      const float m = wt[r * S + s2];
+      const float f = (m == -INFINITY) ? 0.0f : ex2(m - M);
+      wt[r * S + s2] = f;
+      L = fmaf(f, ls[r * S + s2], L);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
+    if (lane == 0) Lr[r] = L;
+  }
+  __syncthreads();
+  // phase 3: warp g sums splits s = g (mod W) for all heads; lane j4 owns dims 4 j4 .. 4 j4 + 3
+  {
+    float4 acc[HG];
+#pragma unroll
+    for (int r = 0; r < HG; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int s2 = warp; s2 < S; s2 += W) {
+#pragma unroll
+      for (int r = 0; r < HG; ++r) {
+        if (r < nh) {
+          const float f = wt[r * S + s2];
+          const float* ps = part0 + ((int64_t)r * S + s2) * PART + 2 + 4 * lane;
+          const float2 lo = __ldcg(reinterpret_cast<const float2*>(ps));
+          const float2 hi = __ldcg(reinterpret_cast<const float2*>(ps + 2));
+          acc[r].x = fmaf(f, lo.x, acc[r].x);
+          acc[r].y = fmaf(f, lo.y, acc[r].y);
+          acc[r].z = fmaf(f, hi.x, acc[r].z);
+          acc[r].w = fmaf(f, hi.y, acc[r].w);
+        }
       }
     }
-    float* dstp = partw + (g * HG + r) * D + 4 * j4;
-    dstp[0] = acc.x;
-    dstp[1] = acc.y;
-    dstp[2] = acc.z;
-    dstp[3] = acc.w;
-    if (j4 == 0) lsw[g * HG + r] = lsum;
+#pragma unroll
+    for (int r = 0; r < HG; ++r)
+      if (r < nh) *reinterpret_cast<float4*>(red + (warp * HG + r) * D + 4 * lane) = acc[r];
   }
   __syncthreads();
-  if (tid < nh) {
-    float L = 0.0f;
-    for (int gg = 0; gg < W; ++gg) L += lsw[gg * HG + tid];
-    Lr[tid] = L;
+  // phase 4: o' = (sum over warps) / L
+  for (int idx = tid; idx < nh * D; idx += T) {
+    const int r = idx / D, d = idx % D;
+    float O = 0.0f;
+#pragma unroll
+    for (int g = 0; g < W; ++g) O += red[(g * HG + r) * D + d];
+    ob[idx] = Lr[r] > 0.0f ? O / Lr[r] : 0.0f;
   }
-  __syncthreads();
-  for (int r = 0; r < nh; ++r)
-    for (int d = tid; d < D; d += T) {
-      float O = 0.0f;
-      for (int gg = 0; gg < W; ++gg) O += partw[(gg * HG + r) * D + d];
-      ob[r * D + d] = Lr[r] > 0.0f ? O / Lr[r] : 0.0f;
-    }
   __syncthreads();
   if (tid >= D) return;
-  // o_i = sum_j Pi[j][i] o'_j  (thread i; rows of Pi are read coalesced across threads)
-  float acc[HG];
+  // phase 5: o_i = sum_j Pi[j][i] o'_j (thread i; rows of Pi coalesced across threads), the next
+  // 16 rows loaded while the current ones are used
+  constexpr int JB = 16;
+  float acc[HG], pj[JB];
 #pragma unroll
   for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
+#pragma unroll
+  for (int jj = 0; jj < JB; ++jj) pj[jj] = __ldg(Pi + jj * D + tid);
 #pragma unroll 1
-  for (int j0 = 0; j0 < D; j0 += 32) {
-    float pj[32];
+  for (int j0 = 0; j0 < D; j0 += JB) {
+    float nx[JB];
+    if (j0 + JB < D) {
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) pj[jj] = __ldg(a.Pi + (j0 + jj) * D + tid);
+      for (int jj = 0; jj < JB; ++jj) nx[jj] = __ldg(Pi + (j0 + JB + jj) * D + tid);
+    }
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj)
+    for (int jj = 0; jj < JB; ++jj)
 #pragma unroll
       for (int r = 0; r < HG; ++r) acc[r] = fmaf(pj[jj], ob[r * D + j0 + jj], acc[r]);
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj) pj[jj] = nx[jj];
   }
-  for (int r = 0; r < nh; ++r) a.out[((int64_t)b * a.Hq + h0 + r) * D + tid] = acc[r];
+  for (int r = 0; r < nh; ++r) out[((int64_t)b * Hq + h0 + r) * D + tid] = acc[r];
 }
 
 // Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (m8n8 fragment layout).
@@ -765,7 +816,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::THREADS, Cfg<KB, VB>::MIN_BLOCKS)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  merge_splits<WARPS>(a, b, h0, nh, pipe);
+  merge_splits<WARPS>(a.part, a.Pi, a.out, a.Hq, a.splits, b, h0, nh, smem);
 }
 
 // ------------------------------------------------------------------------------------------ host
@@ -808,6 +859,7 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms, int resident, int s
   int64_t splits = slots / units;
   const int64_t max_splits = (seq_len + 4 * STAGE_TOK - 1) / (4 * STAGE_TOK);  // >= 4 stages each
   if (splits > max_splits) splits = max_splits;
+  if (splits > SPLITS_MAX) splits = SPLITS_MAX;
   if (splits < 1) splits = 1;
   int64_t tps = (seq_len + splits - 1) / splits;
   tps = (tps + STAGE_TOK - 1) / STAGE_TOK * STAGE_TOK;
@@ -936,14 +988,17 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   a.counters = reinterpret_cast<int*>(ws + (size_t)2 * BH * D + (size_t)BH * plan.splits * PART);
   a.Pi = params->Pi;
   a.out = out;
+  // heads per cluster: about 16 clusters at least (one CTA on each of 128 SMs), at most PREP_HB
+  const int hb = std::max(1, std::min(PREP_HB, BH / 16));
+  const int prep_ctas = (BH + hb - 1) / hb * PREP_CLUSTER;
   if (q_dtype == TQ_F32)
-    prep_kernel<float><<<BH, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), params->Pi, params->S,
-                                        cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D, a.counters,
-                                        n_counters);
+    prep_kernel<float><<<prep_ctas, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), BH, hb, params->Pi,
+                                                           params->S, cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D,
+                                                           a.counters, n_counters);
   else
-    prep_kernel<__nv_bfloat16><<<BH, PREP_THREADS, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(q), params->Pi,
-                                                params->S, cache->qjl_m ? 1 : 0, ws,
-                                                ws + (size_t)BH * D, a.counters, n_counters);
+    prep_kernel<__nv_bfloat16><<<prep_ctas, PREP_THREADS, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16*>(q), BH, hb, params->Pi, params->S, cache->qjl_m ? 1 : 0, ws,
+        ws + (size_t)BH * D, a.counters, n_counters);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
 

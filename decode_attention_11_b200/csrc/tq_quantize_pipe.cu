@@ -29,7 +29,6 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
-#include <atomic>
 #include <mutex>
 
 #include "tq_internal.h"
@@ -61,6 +60,19 @@ constexpr float C_SCALE = 0.04419417382415922f;   // sqrt(128) / 256 (u = y * C_
 __device__ unsigned int g_pipe_error;         // bit 0: a wait timed out; bit 1: smem misaligned; bit 2: no LUT
 __device__ unsigned int g_pipe_vector_fixups;
 __device__ unsigned int g_pipe_code_fixups;
+// Launch epoch of the fixup ring: read by every CTA at start, advanced by the last CTA to finish,
+// so consecutive launches on a stream (CUDA graph replays included) never share an epoch.
+__device__ unsigned int g_pipe_epoch;
+__device__ unsigned int g_pipe_ctas_done;
+
+// One thread per CTA, on every exit path.
+__device__ __forceinline__ void count_cta_done() {
+  __threadfence();
+  if (atomicAdd(&g_pipe_ctas_done, 1u) == gridDim.x - 1) {  // every CTA has read the epoch
+    g_pipe_ctas_done = 0;
+    atomicAdd(&g_pipe_epoch, 1u);
+  }
+}
 
 // One queued fixup for row r of global tile `tile` (CTA-local tile number seqt).  kind 0 / 1: half
 // e of the row (coordinates 64e..64e+63): m[0..1] key coordinates near a threshold (flags bit 0),
@@ -103,7 +115,6 @@ struct PArgs {
   const float* vc;
   const float* vt;
   float band_code, band_sign;
-  uint32_t epoch;  // distinguishes this launch's fixup entries from older ones in the ring
 };
 
 struct __align__(1024) PSmem {
@@ -139,6 +150,7 @@ struct __align__(1024) PSmem {
   unsigned int stored_seq;   // tiles in global memory (CTA-local count)
   unsigned int main_done;
   unsigned int fix_done[N_FIX];
+  uint32_t epoch;            // this launch's ring epoch
 };
 
 static_assert(sizeof(PSmem) <= 232448, "shared memory per CTA");
@@ -790,8 +802,8 @@ __device__ __noinline__ void role_mma(const PArgs& a, uint32_t tmem, int n_tiles
   __syncwarp();
 }
 
-__device__ __forceinline__ uint64_t fix_tag(const PArgs& a, unsigned int k) {
-  return ((uint64_t)a.epoch << 32) | (uint64_t)(k + 1u);
+__device__ __forceinline__ uint64_t fix_tag(const PSmem& s, unsigned int k) {
+  return ((uint64_t)s.epoch << 32) | (uint64_t)(k + 1u);
 }
 
 // Push one fixup entry (rare).  Tiles leave the CTA in order and every entry belongs to a tile
@@ -819,7 +831,7 @@ __device__ __forceinline__ void push_fix(PSmem& s, const PArgs& a, const FixEntr
   for (int i = 0; i < 4; ++i) dst->m[i] = E.m[i];
   dst->seqt = E.seqt;
   __threadfence_block();
-  *reinterpret_cast<volatile uint64_t*>(&dst->tag) = fix_tag(a, slot);  // valid from here on
+  *reinterpret_cast<volatile uint64_t*>(&dst->tag) = fix_tag(s, slot);  // valid from here on
 }
 
 // Once all four conversion warps have stored tile ut (its sfree phase), let fixups of tiles up to
@@ -1127,7 +1139,7 @@ __device__ __noinline__ void role_fix(const PArgs& a) {
   while (true) {
     const FixEntry* src = &g_fix_ring[blockIdx.x][k % QCAP];
     const unsigned int stored = ld_acq(&s.stored_seq);
-    if (*reinterpret_cast<const volatile uint64_t*>(&src->tag) == fix_tag(a, k)) {
+    if (*reinterpret_cast<const volatile uint64_t*>(&src->tag) == fix_tag(s, k)) {
       __threadfence_block();
       const FixEntry E = *src;
       if (E.seqt < stored) {  // its tile is in global memory: patch it
@@ -1166,7 +1178,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr int LK = 1 << KB, LV = 1 << VB;
   if ((smem_u32(smem_raw) & 1023u) != 0) {
-    if (tid == 0) atomicOr(&g_pipe_error, 2u);
+    if (tid == 0) {
+      atomicOr(&g_pipe_error, 2u);
+      count_cta_done();
+    }
     return;
   }
   const int n_tiles = (int)((a.total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
@@ -1195,6 +1210,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     s.q_tail = 0;
     s.stored_seq = 0;
     s.main_done = 0;
+    s.epoch = *reinterpret_cast<volatile unsigned int*>(&g_pipe_epoch);
     for (int i = 0; i < N_FIX; ++i) s.fix_done[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -1214,7 +1230,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (s.err & 4u) {  // no usable cell width for this codebook (never for Lloyd-Max grids of 2..4 bits)
-    if (tid == 0) atomicOr(&g_pipe_error, 4u);
+    if (tid == 0) {
+      atomicOr(&g_pipe_error, 4u);
+      count_cta_done();
+    }
     if (warp == W_MMA) tmem_dealloc(s.tmem_base, TMEM_COLS);
     return;
   }
@@ -1229,7 +1248,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0 && s.err) atomicOr(&g_pipe_error, s.err);
+  if (tid == 0) {
+    if (s.err) atomicOr(&g_pipe_error, s.err);
+    count_cta_done();
+  }
   if (warp == W_MMA) tmem_dealloc(tmem, TMEM_COLS);
 }
 
@@ -1327,8 +1349,6 @@ tq_status quantize_bf16_pipeline(const tq_params* p, const void* k, const void* 
   // |S rho| error <= 8e-6 measured.  The bands are wider.
   a.band_code = 4e-6f;
   a.band_sign = 3e-5f;
-  static std::atomic<uint32_t> launches{0};
-  a.epoch = launches.fetch_add(1u, std::memory_order_relaxed) + 1u;
   const int grid = (int)std::min<int64_t>(a.total_tiles, std::min(sms, MAX_CTAS));
   *handled = true;
   const int kb = c->k_bits, vb = c->v_bits;

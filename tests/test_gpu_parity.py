@@ -169,6 +169,74 @@ def test_decode_parity_small(name):
         assert_attention_close(got, ref)
 
 
+def test_decode_ignores_workspace_contents():
+    """The workspace's previous contents (counters included) never change the result: filled with
+    0x00, 0xFF and 0x5A bytes, and reused across back-to-back calls on one stream."""
+    w = small("llama3_8b_32k")
+    K, V, Kh, Vh = gpu_inputs(w)
+    q = W.make_queries(w).cuda()
+    params = params_for(w)
+    arrays, _ = oracle_cache_arrays(w, Kh, Vh, w.T)
+    cache = tq.Cache.from_arrays(arrays, w.k_bits, w.v_bits, w.qjl_m)
+    ref = O.decode_attention(q.double().cpu().numpy(), W.rotation_for(w), W.qjl_for(w), arrays,
+                             w.k_bits, w.v_bits, w.T)
+    ws = torch.empty(tq.decode_workspace_size(w.B, w.Hq, cache, w.T), dtype=torch.uint8, device="cuda")
+    outs = []
+    for fill in (0x00, 0xFF, 0x5A):
+        ws.fill_(fill)
+        for _ in range(3):
+            outs.append(tq.decode_attn(params, q, cache, w.T, workspace=ws))
+    torch.cuda.synchronize()
+    for out in outs:
+        assert_attention_close(out.cpu().numpy(), ref)
+
+
+def test_quantize_and_decode_replayed_from_cuda_graphs():
+    """Both ops captured once into CUDA graphs, then replayed on new inputs copied into the captured
+    buffers, match direct calls: the same cache bits, and attention within fp32 summation order
+    (the decode's chunk-to-CTA assignment is dynamic)."""
+    w = W.CONFIGS["llama3_8b_128k_b4"].scaled(T=4096, B=1, Hkv=2, Hq=8)
+    params = params_for(w)
+    K, V, _, _ = gpu_inputs(w)
+    q = W.make_queries(w).cuda()
+    Kb, Vb, qb = K.clone(), V.clone(), q.clone()
+    cache_g = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    ws = torch.empty(tq.decode_workspace_size(w.B, w.Hq, cache_g, w.T), dtype=torch.uint8, device="cuda")
+    out_g = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        tq.quantize(params, Kb, Vb, cache_g)
+        tq.decode_attn(params, qb, cache_g, w.T, out=out_g, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    gq, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gq):
+        tq.quantize(params, Kb, Vb, cache_g)
+    with torch.cuda.graph(gd):
+        tq.decode_attn(params, qb, cache_g, w.T, out=out_g, workspace=ws)
+    v0 = tq.quantize_vector_fixups()
+    for shift in (0, 1000, 2321):
+        Ki, Vi, qi = torch.roll(K, shift, 2), torch.roll(V, shift, 2), torch.roll(q, shift, 1)
+        Kb.copy_(Ki)
+        Vb.copy_(Vi)
+        qb.copy_(qi)
+        gq.replay()
+        gd.replay()
+        cache_d = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+        tq.quantize(params, Ki, Vi, cache_d)
+        out_d = tq.decode_attn(params, qi, cache_d, w.T)
+        torch.cuda.synchronize()
+        assert tq.quantize_device_errors() == 0
+        for x, y in zip((cache_g.k_codes, cache_g.k_signs, cache_g.k_norm, cache_g.k_rnorm, cache_g.v_codes,
+                         cache_g.v_norm),
+                        (cache_d.k_codes, cache_d.k_signs, cache_d.k_norm, cache_d.k_rnorm, cache_d.v_codes,
+                         cache_d.v_norm)):
+            assert torch.equal(x, y)
+        assert torch.allclose(out_g, out_d, rtol=0, atol=1e-5)
+    assert tq.quantize_vector_fixups() > v0  # the replays went through the fp64 fixup queue
+
+
 def test_decode_empty_context_is_zero():
     w = small("llama3_8b_32k")
     (got, ref), = decode_on_oracle_cache(w, [0])
