@@ -45,7 +45,7 @@ struct Cfg {
 };
 inline int stage_tokens(int kb, int vb) { return (kb == 4 && vb == 4) ? 96 : 64; }
 constexpr int HG = 8;                  // query heads per MMA row block (hi rows 0-7, lo rows 8-15)
-constexpr int PART = 2 + D;            // (max, sum, o'[128]) per partial
+constexpr int PART = 4 + D;            // (max, sum, pad, pad, o'[128]) per partial: o' 16-byte aligned
 constexpr int SPLITS_MAX = 512;        // CTAs per (batch, kv-head, head group)
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -418,13 +418,11 @@ __device__ void merge_splits(const float* __restrict__ part, const float* __rest
       for (int r = 0; r < HG; ++r) {
         if (r < nh) {
           const float f = wt[r * S + s2];
-          const float* ps = part0 + ((int64_t)r * S + s2) * PART + 2 + 4 * lane;
-          const float2 lo = __ldcg(reinterpret_cast<const float2*>(ps));
-          const float2 hi = __ldcg(reinterpret_cast<const float2*>(ps + 2));
-          acc[r].x = fmaf(f, lo.x, acc[r].x);
-          acc[r].y = fmaf(f, lo.y, acc[r].y);
-          acc[r].z = fmaf(f, hi.x, acc[r].z);
-          acc[r].w = fmaf(f, hi.y, acc[r].w);
+          const float4 o = __ldcg(reinterpret_cast<const float4*>(part0 + ((int64_t)r * S + s2) * PART + 4 + 4 * lane));
+          acc[r].x = fmaf(f, o.x, acc[r].x);
+          acc[r].y = fmaf(f, o.y, acc[r].y);
+          acc[r].z = fmaf(f, o.z, acc[r].z);
+          acc[r].w = fmaf(f, o.w, acc[r].w);
         }
       }
     }
@@ -798,7 +796,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::THREADS, Cfg<KB, VB>::MIN_BLOCKS)
       O += f * ow[(w * HG + r) * D + tid];
     }
     float* dst = a.part + (((int64_t)b * a.Hq + h0 + r) * a.splits + split) * PART;
-    dst[2 + tid] = O;
+    dst[4 + tid] = O;
     if (tid == 0) {
       dst[0] = M;
       dst[1] = Ls;
@@ -868,7 +866,7 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms, int resident, int s
   return p;
 }
 
-// Workspace: q' and S q' [B*Hq][128] fp32, split partials [B*Hq][splits][130] fp32, then one
+// Workspace: q' and S q' [B*Hq][128] fp32, split partials [B*Hq][splits][132] fp32, then one
 // completion counter per (batch, kv-head, head group).
 size_t workspace_bytes(int B, int Hq, int Hkv, const Plan& p) {
   return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART) +
