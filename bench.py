@@ -11,6 +11,7 @@ independent replica of the workload (the path has no exchange step), timing is t
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -246,7 +247,7 @@ def run_reference(args, w):
 def workload_config(w: W.Workload, **extra):
     c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.head_dim,
          "context": w.T, "k_bits": w.k_bits, "v_bits": w.v_bits, "qjl_m": w.qjl_m,
-         "input_dtype": w.in_dtype, "quantize_chunk": w.chunk,
+         "input_dtype": w.in_dtype, "quantize_chunk": w.chunk, "rotation": w.rotation,
          "l2": f"flushed before every kernel call ({L2_FLUSH_BYTES >> 20} MiB write)"}
     c.update(extra)
     return c
@@ -435,6 +436,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every op directly in the timed steps")
+    ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
+                    help="Pi: dense Haar-random (default) or the structured D1 H D2 H D3 / 128")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--context", type=int, default=None, help="override the workload's context")
     args = ap.parse_args()
@@ -443,6 +446,8 @@ def main():
     w = W.CONFIGS[args.workload]
     if args.batch is not None or args.context is not None:
         w = w.scaled(B=args.batch, T=args.context, name=w.name + "(resized)")
+    if args.rotation != w.rotation:
+        w = dataclasses.replace(w, rotation=args.rotation)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -37,7 +37,8 @@ EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codeboo
             "tq_quantize", "tq_quantize_device_errors", "tq_quantize_vector_fixups",
             "tq_quantize_code_fixups",
             "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
-            "tq_decode_static_workspace_limit", "tq_sketch_rotation")
+            "tq_decode_static_workspace_limit", "tq_sketch_rotation", "tq_build_hadamard_rotation",
+            "tq_decode_step")
 
 
 class TqError(RuntimeError):
@@ -105,6 +106,13 @@ def lib() -> ctypes.CDLL:
                                         ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
     L.tq_decode_static_workspace_limit.restype = ctypes.c_size_t
     L.tq_decode_static_workspace_limit.argtypes = []
+    L.tq_decode_step.restype = ctypes.c_int
+    L.tq_decode_step.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                 ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache),
+                                 ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                 ctypes.c_size_t, ctypes.c_void_p]
+    L.tq_build_hadamard_rotation.restype = ctypes.c_int
+    L.tq_build_hadamard_rotation.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_float)]
     L.tq_sketch_rotation.restype = ctypes.c_int
     L.tq_sketch_rotation.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                      ctypes.c_void_p]
@@ -141,6 +149,14 @@ def build_codebook(bits: int, max_iter: int = 100000, tol: float = 1e-13
                                    t.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
                                    ctypes.byref(dist)))
     return c[:L], t[:L - 1], float(dist.value)
+
+
+def build_hadamard_rotation(seed: int) -> np.ndarray:
+    """Structured orthogonal rotation D1 H D2 H D3 / 128 (tq_build_hadamard_rotation), fp32 [128, 128]."""
+    P = np.empty((128, 128), dtype=np.float32)
+    _check(lib().tq_build_hadamard_rotation(int(seed) & ((1 << 64) - 1),
+                                            P.ctypes.data_as(ctypes.POINTER(ctypes.c_float))))
+    return P
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -303,6 +319,33 @@ def decode_attn(params: Params, q: torch.Tensor, cache: Cache, seq_len: int,
                                 ctypes.byref(c), int(seq_len), float(scale), out.data_ptr(),
                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                 _stream_ptr(stream)))
+    return out
+
+
+def decode_step(params: Params, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, cache: Cache,
+                t: int, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                scale: float = 0.0, stream=None) -> torch.Tensor:
+    """One decode step: k_new, v_new [B, Hkv, 128] go to cache row t, then q [B, Hq, 128] attends
+    over rows [0, t] -> fp32 [B, Hq, 128] (tq_decode_step)."""
+    for x, n in ((k_new, "k_new"), (v_new, "v_new"), (q, "q")):
+        if x.dim() != 3 or x.shape[-1] != 128 or not x.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous [B, H, 128] tensor")
+    if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    if tuple(k_new.shape[:2]) != (cache.B, cache.Hkv):
+        raise ValueError("k_new must be [B, Hkv, 128] of the cache")
+    B, Hq, _ = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, 128, dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, Hq, cache, t + 1)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    c = cache.as_c()
+    p = params.as_c()
+    _check(lib().tq_decode_step(ctypes.byref(p), k_new.data_ptr(), v_new.data_ptr(), _dtype_code(k_new),
+                                q.data_ptr(), _dtype_code(q), int(Hq), ctypes.byref(c), int(t), float(scale),
+                                out.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
     return out
 
 

@@ -1007,6 +1007,34 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   return TQ_OK;
 }
 
+// One decode step: append the new token (tq_quantize with T_new = 1), then attend over t + 1
+// tokens.  The decode arguments are checked first so that an invalid call enqueues nothing.
+extern "C" tq_status tq_decode_step(const tq_params* params, const void* k_new, const void* v_new,
+                                    int kv_dtype, const void* q, int q_dtype, int Hq, const tq_cache* cache,
+                                    int t, float scale, float* out, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  using namespace tq;
+  clear_error();
+  tq_status st = check_cache(cache);
+  if (st != TQ_OK) return st;
+  st = check_params(params, cache);
+  if (st != TQ_OK) return st;
+  if (t < 0 || t >= cache->T_cap) return fail(TQ_ERR_INVALID_ARG, "t %d outside [0, %d)", t, cache->T_cap);
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, "q_dtype %d", q_dtype);
+  if (Hq < 1 || Hq % cache->Hkv) return fail(TQ_ERR_INVALID_ARG, "Hq %d vs Hkv %d", Hq, cache->Hkv);
+  if (!q || !out || !workspace) return fail(TQ_ERR_INVALID_ARG, "q / out / workspace is NULL");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
+    return fail(TQ_ERR_INVALID_ARG, "q / out / workspace must be 16-byte aligned");
+  const size_t need = tq_decode_workspace_size(cache->B, Hq, cache, t + 1);
+  if (workspace_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  const int64_t sh = kHeadDim, sb = (int64_t)cache->Hkv * kHeadDim;
+  st = tq_quantize(params, k_new, v_new, kv_dtype, sb, sh, kHeadDim, 1, t, cache, stream);
+  if (st != TQ_OK) return st;
+  return tq_decode_attn(params, q, q_dtype, Hq, cache, t + 1, scale, out, workspace, workspace_bytes,
+                        stream);
+}
+
 // ------------------------------------------------------------------------------------------------
 // Allocation-free decode: the same kernels, with the scratch space in a fixed device array.
 //

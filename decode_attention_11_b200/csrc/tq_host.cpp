@@ -166,4 +166,30 @@ tq_status tq_build_codebook(int bits, int max_iter, double tol, float* centroids
   return TQ_OK;
 }
 
+// Structured rotation D1 H D2 H D3 / 128 (see tq.h).  Signs from SplitMix64 (Steele, Lea and
+// Flood, OOPSLA 2014): output n of a generator started at `seed`.
+tq_status tq_build_hadamard_rotation(uint64_t seed, float* Pi) {
+  tq::clear_error();
+  if (!Pi) return tq::fail(TQ_ERR_INVALID_ARG, "Pi is NULL");
+  constexpr int d = tq::kHeadDim;
+  auto splitmix = [seed](uint64_t n) {
+    uint64_t z = seed + (n + 1) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  };
+  auto had = [](int i, int j) { return (__builtin_popcount((unsigned)(i & j)) & 1) ? -1 : 1; };
+  int sgn[3][d];
+  for (int k = 0; k < 3; ++k)
+    for (int i = 0; i < d; ++i) sgn[k][i] = (splitmix((uint64_t)(k * d + i)) & 1) ? -1 : 1;
+  // (D1 H D2 H D3)[i][j] = s1[i] s3[j] sum_m H[i][m] s2[m] H[m][j]: an integer, exact in fp32
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) {
+      int acc = 0;
+      for (int m = 0; m < d; ++m) acc += had(i, m) * sgn[1][m] * had(m, j);
+      Pi[i * d + j] = (float)(sgn[0][i] * sgn[2][j] * acc) / (float)d;
+    }
+  return TQ_OK;
+}
+
 }  // extern "C"

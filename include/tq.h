@@ -89,6 +89,20 @@ int tq_version(void);
 tq_status tq_build_codebook(int bits, int max_iter, double tol, float* centroids,
                             float* thresholds, double* distortion);
 
+/*
+ * Structured alternative to a dense Haar rotation for tq_params.Pi (host, no device work):
+ * Pi = D1 H D2 H D3 / 128, H the 128 x 128 Sylvester Hadamard matrix (H[i][j] = (-1)^popcount(i & j)),
+ * D_k = diag(s_k) with s_k[i] = +1 when output 128k + i of a SplitMix64 generator started at
+ * `seed` is even, else -1.  Orthogonal exactly; every entry is a multiple of 1/64, so it is exact
+ * in fp16 and the rotation MMA needs no lo part.
+ * Source: tproger.ru, section "TurboQuant in llama.cpp, MLX and PyTorch: who is already trying"
+ * (the dense rotation is the slow step; its authors turn to the Hadamard transform); ai-news.ru
+ * overview, paragraph on RotorQuant (the dense d x d rotation costs 16384 operations at d = 128).
+ *   Pi   host float[128 * 128] out, row-major.
+ * Errors: TQ_ERR_INVALID_ARG (Pi NULL).  Thread-safe.
+ */
+tq_status tq_build_hadamard_rotation(uint64_t seed, float* Pi);
+
 /* Caller-owned packed cache (device pointers; see the layout above).  k_signs and k_rnorm may
  * be NULL when qjl_m == 0. */
 typedef struct {
@@ -190,6 +204,26 @@ size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_le
 tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, int Hq,
                          const tq_cache* cache, int seq_len, float scale, float* out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One autoregressive decode step: compress the new token's K and V into cache row t of every
+ * (batch, kv-head), then attend q over rows [0, t].  Enqueues tq_quantize (T_new = 1) and
+ * tq_decode_attn (seq_len = t + 1) back to back on `stream`, so one CUDA graph can hold a whole
+ * step (the graph is specific to t).
+ * Source: ai-manual.ru MLX port, section "who needs this right now" (the method serves text
+ * generation with autoregressive decoding); ai-news.ru overview, paragraph on the speed figures
+ * (quantization is paid per token on top of attention).
+ *   k_new, v_new  device [B, Hkv, 128] of kv_dtype (TQ_F32 or TQ_BF16), contiguous
+ *   q             device [B, Hq, 128] of q_dtype (TQ_F32 or TQ_BF16), contiguous
+ *   t             0 <= t < cache->T_cap;  rows [0, t) must already hold the earlier tokens
+ *   scale, out    as tq_decode_attn
+ *   workspace     device, at least tq_decode_workspace_size(B, Hq, cache, t + 1) bytes
+ * Errors: as tq_quantize and tq_decode_attn; every argument is checked before anything is
+ * enqueued.
+ */
+tq_status tq_decode_step(const tq_params* params, const void* k_new, const void* v_new, int kv_dtype,
+                         const void* q, int q_dtype, int Hq, const tq_cache* cache, int t, float scale,
+                         float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * tq_decode_attn_static -- decode attention that allocates nothing and takes no workspace.

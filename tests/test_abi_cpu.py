@@ -120,3 +120,35 @@ def test_workspace_size():
     assert L.tq_decode_workspace_size(1, 8, None, 64) == 0
     big = L.tq_decode_workspace_size(4, 32, ctypes.byref(fake_cache(B=4, Hkv=8, T_cap=131072)), 131072)
     assert big < 64 << 20
+
+
+def step_status(cache=None, params=None, k=FAKE, v=FAKE, kv_dtype=tq.TQ_BF16, q=FAKE, Hq=8, t=10,
+                out=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    L = tq.lib()
+    return L.tq_decode_step(ctypes.byref(params or fake_params()), k, v, kv_dtype, q, tq.TQ_F32, Hq,
+                            ctypes.byref(cache or fake_cache()), t, 0.0, out, ws, ws_bytes, None)
+
+
+def test_decode_step_argument_errors():
+    """Every argument of tq_decode_step is checked before anything is enqueued."""
+    assert step_status(t=64) == tq.TQ_ERR_INVALID_ARG  # T_cap = 64: the new row must exist
+    assert step_status(t=-1) == tq.TQ_ERR_INVALID_ARG
+    assert step_status(Hq=7) == tq.TQ_ERR_INVALID_ARG
+    assert step_status(out=None) == tq.TQ_ERR_INVALID_ARG
+    assert step_status(q=FAKE + 8) == tq.TQ_ERR_INVALID_ARG
+    assert step_status(ws_bytes=16) == tq.TQ_ERR_WORKSPACE
+    assert "need" in tq.last_error()
+    assert step_status(kv_dtype=7) == tq.TQ_ERR_UNSUPPORTED
+    assert step_status(k=None) == tq.TQ_ERR_INVALID_ARG
+    assert step_status(v=FAKE + 4) == tq.TQ_ERR_INVALID_ARG
+    assert step_status(cache=fake_cache(k_bits=5)) == tq.TQ_ERR_UNSUPPORTED
+    assert step_status(params=fake_params(S_Pi=FAKE + 8)) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_sketch_rotation_and_hadamard_builder_argument_errors():
+    L = tq.lib()
+    assert L.tq_sketch_rotation(None, FAKE, 128, FAKE, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_sketch_rotation(FAKE, FAKE + 4, 128, FAKE, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_sketch_rotation(FAKE, FAKE, 0, FAKE, None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_build_hadamard_rotation(1, None) == tq.TQ_ERR_INVALID_ARG
+    assert quantize_status(params=fake_params(S_Pi=FAKE + 8)) == tq.TQ_ERR_INVALID_ARG

@@ -2,6 +2,7 @@
 
 Small cases are compared element by element (several tiles plus a ragged tail); the full-size
 workloads are compared on sampled rows / heads that the oracle computes one by one."""
+import dataclasses
 import math
 
 import numpy as np
@@ -237,6 +238,22 @@ def test_quantize_and_decode_replayed_from_cuda_graphs():
     assert tq.quantize_vector_fixups() > v0  # the replays went through the fp64 fixup queue
 
 
+def test_hadamard_rotation_quantize_and_decode_parity():
+    """The structured rotation D1 H D2 H D3 / 128 (tq_build_hadamard_rotation) as Pi: both kernels
+    against the oracle given the same Pi (fp16-exact entries, so the rotation's lo part is 0)."""
+    w = dataclasses.replace(small("llama3_8b_128k_b4"), rotation="hadamard")
+    assert np.array_equal(W.rotation_for(w), tq.build_hadamard_rotation(1000 + w.seed))
+    params = params_for(w)
+    K, V, Kh, Vh = gpu_inputs(w)
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    tq.quantize(params, K, V, cache)
+    torch.cuda.synchronize()
+    assert tq.quantize_device_errors() == 0
+    compare_quantized(w, cache, Kh, Vh, 0)
+    for got, ref in decode_on_oracle_cache(w, [w.T, 100]):
+        assert_attention_close(got, ref)
+
+
 def test_decode_empty_context_is_zero():
     w = small("llama3_8b_32k")
     (got, ref), = decode_on_oracle_cache(w, [0])
@@ -281,6 +298,31 @@ def test_quantize_then_decode_end_to_end():
     rel_mse = np.linalg.norm(no_qjl - exact) / np.linalg.norm(exact)
     print(f"attention rel-L2 vs exact: with QJL {rel_qjl:.3f}, without {rel_mse:.3f}")
     assert rel_qjl < 1.0 and rel_mse < 1.0
+
+
+def test_decode_step_appends_and_attends():
+    """Autoregressive use: the first tokens by one tq_quantize, then one tq_decode_step per new
+    token (bf16 K/V rows written at row t, then attention over rows 0..t).  Each step matches the
+    oracle over the tokens so far, and the whole cache matches the oracle's quantization."""
+    w = small("llama3_8b_32k")
+    params = params_for(w)
+    K, V, Kh, Vh = gpu_inputs(w)
+    T0 = w.T - 5
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    tq.quantize(params, K[:, :, :T0], V[:, :, :T0], cache)
+    q0 = W.make_queries(w)
+    _, oc = oracle_cache_arrays(w, Kh, Vh)
+    ex = O.code_exempt(oc["k_u"], w.k_bits).sum() + O.code_exempt(oc["v_u"], w.v_bits).sum()
+    for t in range(T0, w.T):
+        q = q0 * (1.0 + 0.25 * (t - T0))
+        out = tq.decode_step(params, K[:, :, t].contiguous(), V[:, :, t].contiguous(), q.cuda(), cache, t)
+        torch.cuda.synchronize()
+        assert tq.quantize_device_errors() == 0
+        ref = O.decode_attention(q.double().numpy(), W.rotation_for(w), W.qjl_for(w), oc, w.k_bits,
+                                 w.v_bits, t + 1)
+        if ex == 0:
+            assert_attention_close(out.cpu().numpy(), ref)
+    compare_quantized(w, cache, Kh, Vh, 0)
 
 
 # ------------------------------------------------------------------------------- full size

@@ -59,6 +59,7 @@ class Workload:
     t3_prob: float  # probability an entry is Student-t(3)
     chunk: int  # streaming-quantize chunk length (tokens); T = one chunk
     head_dim: int = HEAD_DIM
+    rotation: str = "haar"  # "haar" (dense Haar-random) | "hadamard" (D1 H D2 H D3 / d)
 
     @property
     def group(self) -> int:
@@ -151,7 +152,37 @@ def make_qjl_matrix(seed: int, m: int = 128, d: int = HEAD_DIM) -> np.ndarray:
     return S.to(torch.float16).to(torch.float32).numpy().copy()
 
 
+_U64 = (1 << 64) - 1
+
+
+def splitmix64(seed: int, n: int) -> int:
+    """Output n (0, 1, ...) of the SplitMix64 generator started at state `seed` (Steele, Lea and
+    Flood, "Fast splittable pseudorandom number generators", OOPSLA 2014): the state advances by
+    0x9E3779B97F4A7C15 and each output is the state after two xor-shift-multiply rounds."""
+    z = (int(seed) + (int(n) + 1) * 0x9E3779B97F4A7C15) & _U64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _U64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _U64
+    return z ^ (z >> 31)
+
+
+def make_hadamard_rotation(seed: int, d: int = HEAD_DIM) -> np.ndarray:
+    """Structured orthogonal d x d matrix D1 H D2 H D3 / d (fp32, every entry a multiple of 2/d).
+
+    H is the Sylvester Hadamard matrix (H[i][j] = (-1)^popcount(i & j)); D_k = diag(s_k) with
+    s_k[i] = +1 if SplitMix64 output k*d + i of `seed` is even, else -1.
+    """
+    assert d & (d - 1) == 0
+    idx = np.arange(d)
+    H = np.array([[(-1) ** bin(i & j).count("1") for j in idx] for i in idx], dtype=np.float64)
+    s = np.array([[1.0 if splitmix64(seed, k * d + i) % 2 == 0 else -1.0 for i in idx] for k in range(3)])
+    P = (s[0][:, None] * H) @ (s[1][:, None] * H) * s[2][None, :] / d
+    return P.astype(np.float32)
+
+
 def rotation_for(w: Workload) -> np.ndarray:
+    if w.rotation == "hadamard":
+        return make_hadamard_rotation(1000 + w.seed, w.head_dim)
+    assert w.rotation == "haar", w.rotation
     return make_rotation(1000 + w.seed, w.head_dim)
 
 
@@ -234,7 +265,8 @@ def nbytes_human(n: int) -> str:
 
 
 __all__ = [
-    "HEAD_DIM", "Workload", "CONFIGS", "CONFIG_ORDER", "make_rotation", "make_qjl_matrix",
+    "HEAD_DIM", "Workload", "CONFIGS", "CONFIG_ORDER", "make_rotation", "make_hadamard_rotation",
+    "splitmix64", "make_qjl_matrix",
     "rotation_for", "qjl_for", "make_kv", "make_queries", "gqa_kv_head", "shard_units",
     "nbytes_human",
 ]
