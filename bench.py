@@ -34,9 +34,16 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 def source_digest(rel: str) -> str:
+    """Digest of a kernel source with comments and blank lines removed, so that a change to the
+    comments alone keeps a capture valid."""
     import hashlib
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    import re
+    with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def dram_traffic(kernel: str, workload: str, batch, context):

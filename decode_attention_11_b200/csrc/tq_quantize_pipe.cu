@@ -10,19 +10,21 @@
 //   warp 12      TMA producer: bf16 K and V tiles into a 3-slot ring (128-byte swizzle, the
 //                UMMA operand layout), completion on mbarriers.
 //   warps 0-3    conversion: each thread turns one row of a slot into fp16 in place (exact for
-//                bf16) and sums its squares (the stored norm, and the scale of u).
+//                bf16) and sums its squares (the stored norm, and the scale of u).  The same
+//                warps then finish the previous tile: the 128 sign bits of each row from the
+//                sketch in tensor memory, and the copy of the staged tile to global memory.
 //   warp 13      MMA issuer: Y = X (Pi_hi + Pi_lo)^T for K and V into one of two tensor-memory
-//                buffers; later S (rho_hi + rho_lo) for the QJL signs, A read from tensor memory.
+//                buffers.
 //   warps 4-11   epilogue: two warpgroups split the 128 coordinates of every row.  Codes come
 //                from a uniform-cell lookup table (one fma gives the cell, one compare against
 //                the cell's threshold gives the code); the key residual rho goes back into
-//                tensor memory as fp16 hi + lo over Y_K; the sketch lands over Y_V.  Rows are
-//                staged in shared memory and leave by bulk copies.
+//                tensor memory as fp16 hi + lo over Y_K, and the last warp to finish issues the
+//                sketch S (rho_hi + rho_lo) over Y_V.  Codes are staged in shared memory.
 //   warps 14-15  fixups: coordinates whose fast value lies within a guard band of a decision
 //                boundary (a threshold; 0 for a sign) are re-derived in fp64 from the original
-//                inputs after the tile has been stored, and patched in place.
+//                inputs once their tile is in global memory, and patched in place.
 // Exactness: codes and sign bits equal those of the float64 definition except where the exact
-// value lies within ~1e-15 of a boundary.
+// value lies within ~1e-13 of a boundary.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
