@@ -175,8 +175,9 @@ def sketch_rotation_product(Pi: torch.Tensor, S: torch.Tensor, stream=None) -> t
     Pi = Pi.contiguous()
     S = S.contiguous()
     out = torch.empty(S.shape[0], 128, dtype=torch.float64, device=Pi.device)
-    _check(lib().tq_sketch_rotation(Pi.data_ptr(), S.data_ptr(), int(S.shape[0]), out.data_ptr(),
-                                    _stream_ptr(stream)))
+    with torch.cuda.device(Pi.device):
+        _check(lib().tq_sketch_rotation(Pi.data_ptr(), S.data_ptr(), int(S.shape[0]), out.data_ptr(),
+                                        _stream_ptr(stream)))
     return out
 
 
