@@ -171,7 +171,11 @@ def _stream_ptr(stream) -> Optional[int]:
 
 def sketch_rotation_product(Pi: torch.Tensor, S: torch.Tensor, stream=None) -> torch.Tensor:
     """S Pi in fp64 on the device of Pi (tq_sketch_rotation), for Params.S_Pi."""
-    assert Pi.is_cuda and S.is_cuda and Pi.dtype == torch.float32 and S.dtype == torch.float32
+    if not (Pi.is_cuda and S.is_cuda and Pi.device == S.device):
+        raise ValueError("Pi and S must be on the same CUDA device")
+    if Pi.dtype != torch.float32 or S.dtype != torch.float32 or tuple(Pi.shape) != (128, 128) \
+            or S.dim() != 2 or S.shape[1] != 128:
+        raise ValueError("Pi must be fp32 [128, 128] and S fp32 [m, 128]")
     Pi = Pi.contiguous()
     S = S.contiguous()
     out = torch.empty(S.shape[0], 128, dtype=torch.float64, device=Pi.device)
