@@ -1,6 +1,6 @@
 // tq_decode_attn: single-token decode attention directly over the packed cache.
 //
-// Scores follow the QJL-corrected estimator of the method statement,
+// Scores follow the QJL-corrected inner-product estimator,
 //   est_i = <q', khat'_i> + ||r_i|| sqrt(pi/2)/m <S q', 2 sign_i - 1>,  q' = Pi q,
 // with khat'_i = (n_i / sqrt(d)) c_K[idx_i] in the rotated basis (ai-news.ru overview, first and
 // second ideas plus the third, QJL, component; tproger.ru "Step 1: PolarQuant", "Step 2: QJL").

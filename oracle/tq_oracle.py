@@ -22,11 +22,12 @@ Sources (all page citations name the page and the passage):
   one extra bit to make the residual error unbiased.  Section "Benchmarks --
   from independent implementations": TQ3 MSE 0.034, TQ4 MSE 0.009, a TQ3
   block is 52 bytes per 128 values.
-* The estimator of the inner product, in the method statement this build
-  follows: <q,k> ~= <q,k_mse> + ||r|| sqrt(pi/2)/m <S q, sign(S r)> with a
-  Gaussian S of m rows, storing sign(S r) and ||r||.
+* The QJL estimator of the inner product (the unbiased 1-bit residual
+  correction of tproger.ru "Step 2: QJL" and the ai-news.ru third component):
+  <q,k> ~= <q,k_mse> + ||r|| sqrt(pi/2)/m <S q, sign(S r)> with a Gaussian S
+  of m rows, storing sign(S r) and ||r||.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * the Lloyd-Max density is the standard normal (rotated, rescaled
   coordinates u = sqrt(d) * Pi x / ||x||);
@@ -176,7 +177,7 @@ def quantize_vectors(X: np.ndarray, Pi: np.ndarray, k_bits: int,
 
 
 # ---------------------------------------------------------------------------
-# Packed row layouts (pages silent: this build's reading, stated in the design doc)
+# Packed row layouts (the pages give none; the layout below is a reading)
 # ---------------------------------------------------------------------------
 
 def k_slot_of_coord(j: int) -> int:
