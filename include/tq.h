@@ -7,6 +7,10 @@
  *   tq_quantize        device   rotate -> scalar-quantize -> pack -> 1-bit QJL sketch of K/V.
  *   tq_decode_attn     device   single-token attention directly over the packed cache.
  *
+ * Around them: tq_decode_attn_static (decode without a caller workspace), tq_decode_step (append
+ * one token, then attend), tq_sketch_rotation (the optional fp64 constant S Pi),
+ * tq_build_hadamard_rotation (a structured Pi), and the tq_quantize diagnostics.
+ *
  * Method sources (page and passage):
  *   - ai-news.ru TurboQuant overview, paragraphs on the first and second ideas: multiply each
  *     vector by a random orthogonal matrix so the coordinates become near-Gaussian, then apply a
