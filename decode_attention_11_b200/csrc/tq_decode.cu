@@ -6,7 +6,7 @@
 // second ideas plus the third, QJL, component; tproger.ru "Step 1: PolarQuant", "Step 2: QJL").
 // Softmax and the value sum also run in the rotated basis; one final o = Pi^T o' per head.
 //
-// Kernels (both on the caller's stream; the second is a programmatic dependent launch):
+// Kernels (all on the caller's stream; split and merge are programmatic dependent launches):
 //   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace: clusters of
 //           eight CTAs, each CTA holding 16 rows of Pi and S for a batch of up to 16 heads.
 //   split   grid (splits, Hkv * head_groups, B).  A 4-warp CTA streams its token range through a
@@ -15,9 +15,9 @@
 //           two coordinates, no bank conflicts), and m16n8k16 tensor-core MMAs compute q'.khat,
 //           the QJL sign dot (q' and S q' split into fp16 hi + lo rows; signs -> +-0.5 by one
 //           half2 FMA) and P.vhat (P split into hi + lo rows).  Online softmax runs in log2 units.
-//           The CTA merges its 4 warps and writes one (max, sum, o'[128]) partial per head.
-//           The last CTA of each (batch, kv-head, head group) to finish (completion counter)
-//           merges the split partials by log-sum-exp and writes o = Pi^T o'.
+//           The CTA merges its warps and writes one (max, sum, o'[128]) partial per head.
+//   merge   one CTA per (batch, query head), a programmatic dependent of split: log-sum-exp
+//           merge of the head's split partials, then o = Pi^T o'.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -64,9 +64,6 @@ struct DArgs {
   const float* qrot;
   const float* sq;
   float* part;
-  int* counters;    // one per (batch, kv-head, head group); zeroed by prep
-  const float* Pi;  // final un-rotation
-  float* out;
 };
 
 // ------------------------------------------------------------------------------------------ PTX
@@ -203,9 +200,8 @@ __device__ __forceinline__ uint32_t v_code(uint64_t c) {
 // work) and CTA c of it rows 16c .. 16c+15 of q' = Pi q and of sq = S q', eight threads per row
 // with 16 columns each.  Each CTA loads its rows of Pi and S once (one memory round trip,
 // together with the query vectors) and reuses them for all its heads; the full q' of every head
-// reaches the other CTAs of the cluster through distributed shared memory.  CTA 0 also
-// zeroes the split counters.  The split kernel is launched as a programmatic dependent of this
-// one and starts its prologue early.
+// reaches the other CTAs of the cluster through distributed shared memory.  The split kernel is
+// launched as a programmatic dependent of this one and starts its prologue early.
 constexpr int PREP_CLUSTER = 8, PREP_THREADS = 128, PREP_ROWS = D / PREP_CLUSTER, PREP_HB = 16;
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -223,8 +219,7 @@ __device__ __forceinline__ float ld_cluster_f32(const float* p, uint32_t rank) {
 template <typename QT>
 __global__ void __cluster_dims__(PREP_CLUSTER, 1, 1) __launch_bounds__(PREP_THREADS)
     prep_kernel(const QT* __restrict__ q, int BH, int hb, const float* __restrict__ Pi, const float* __restrict__ S,
-                int qjl, float* __restrict__ qrot, float* __restrict__ sq, int* __restrict__ counters,
-                int n_counters) {
+                int qjl, float* __restrict__ qrot, float* __restrict__ sq) {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   __shared__ __align__(16) float qs[PREP_HB][D];           // query vectors, then q' of the cluster
   __shared__ __align__(16) float qpart[PREP_HB][PREP_ROWS];  // this CTA's rows of q'
@@ -234,8 +229,6 @@ __global__ void __cluster_dims__(PREP_CLUSTER, 1, 1) __launch_bounds__(PREP_THRE
   const int nhb = min(hb, BH - h0);
   const int rl = tid >> 3, part = tid & 7;
   const int row = PREP_ROWS * (int)c + rl;
-  if (blockIdx.x == 0)
-    for (int i = tid; i < n_counters; i += PREP_THREADS) counters[i] = 0;
   float4 p[4], s4[4];
   const float4* pr = reinterpret_cast<const float4*>(Pi + row * D + 16 * part);
 #pragma unroll
@@ -302,13 +295,10 @@ struct Layout {
   static constexpr int OFF_NV = OFF_RN + (QJL ? STAGE_TOK * 4 : 0);
   static constexpr int STAGE_BYTES = OFF_NV + STAGE_TOK * 4;
   static constexpr int LUT_BYTES = kPackedLut ? 256 * 256 : ((1 << (2 * KB)) + (1 << (2 * VB))) * 128;
-  // After the main loop the pipeline buffers hold the CTA's own warp merge; the last CTA then
-  // reuses all of shared memory (tables included) for the split merge.
+  // After the main loop the pipeline buffers hold the CTA's own warp merge.
   static constexpr int WARP_MERGE_BYTES = 4 * (W * HG * 2 + W * HG * D);
-  static constexpr int MERGE_BYTES = 4 * (2 * HG * SPLITS_MAX + HG + W * HG * D + HG * D);
   static constexpr int PIPE_BYTES = NSTAGE * STAGE_BYTES;
-  static constexpr int MAIN_BYTES = LUT_BYTES + (PIPE_BYTES > WARP_MERGE_BYTES ? PIPE_BYTES : WARP_MERGE_BYTES);
-  static constexpr int SMEM = MAIN_BYTES > MERGE_BYTES ? MAIN_BYTES : MERGE_BYTES;
+  static constexpr int SMEM = LUT_BYTES + (PIPE_BYTES > WARP_MERGE_BYTES ? PIPE_BYTES : WARP_MERGE_BYTES);
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
 };
 
@@ -365,106 +355,92 @@ __device__ __forceinline__ uint64_t load_v_chunk(const unsigned char* row, int g
   }
 }
 
-// Log-sum-exp merge of the split partials of heads h0 .. h0+nh-1 of batch b, then o = Pi^T o'.
-// Run by the last CTA to finish (W warps); partials are read from L2 (written by other CTAs).
-// Every phase issues its loads for all heads and splits at once; the un-rotation keeps the next
-// rows of Pi in flight while the current ones are used.
-template <int W>
-__device__ void merge_splits(const float* __restrict__ part, const float* __restrict__ Pi,
-                                          float* __restrict__ out, int Hq, int S, int b, int h0, int nh,
-                                          unsigned char* scratch) {
-  constexpr int T = 32 * W;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* wt = reinterpret_cast<float*>(scratch);  // [nh][S]: partial max, then its weight
-  float* ls = wt + HG * SPLITS_MAX;                // [nh][S]: partial sum
-  float* Lr = ls + HG * SPLITS_MAX;                // [HG]
-  float* red = Lr + HG;                            // [W][HG][D]: per-warp sums over splits
-  float* ob = red + W * HG * D;                    // [HG][D]: merged, normalized o'
-  const float* part0 = part + ((int64_t)b * Hq + h0) * S * PART;  // heads are S partials apart
+// ------------------------------------------------------------------------------------------ merge
 
-  // phase 1: (max, sum) of every partial
-  for (int idx = tid; idx < nh * S; idx += T) {
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(part0 + (int64_t)idx * PART));
-    wt[idx] = ml.x;
-    ls[idx] = ml.y;
+// One 512-thread CTA per (batch, query head), a programmatic dependent of the split kernel: it
+// waits for the split grid, merges the head's split partials by log-sum-exp and writes
+// o = Pi^T o'.  Thread (d, q), d = tid % 128 and q = tid / 128, sums the splits s = q (mod 4) of
+// dimension d; the un-rotation gives thread (i, q) the rows 32q .. 32q + 31 of Pi.  Each phase
+// issues its loads at once (one L2 round trip each).
+constexpr int MERGE_THREADS = 4 * D;
+
+__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(FULL, v, o);
+    v = is_max ? fmaxf(v, x) : v + x;
   }
+  if (lane == 0) red[warp] = v;
   __syncthreads();
-  // phase 2: warp r (mod W) turns head r's maxima into weights 2^(m_s - M) and forms L
-  for (int r = warp; r < nh; r += W) {
-    float M = -INFINITY;
-    for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, wt[r * S + s2]);
+  v = red[lane < MERGE_THREADS / 32 ? lane : 0];
+  if (lane >= MERGE_THREADS / 32) v = is_max ? -INFINITY : 0.0f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
-    float L = 0.0f;
-    for (int s2 = lane; s2 < S; s2 += 32) {
-      const float m = wt[r * S + s2];
-      const float f = (m == -INFINITY) ? 0.0f : ex2(m - M);
-      wt[r * S + s2] = f;
-      L = fmaf(f, ls[r * S + s2], L);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
-    if (lane == 0) Lr[r] = L;
+  for (int o = 16; o > 0; o >>= 1) {  // every lane ends with the full result
+    const float x = __shfl_xor_sync(FULL, v, o);
+    v = is_max ? fmaxf(v, x) : v + x;
   }
-  __syncthreads();
-  // phase 3: warp g sums splits s = g (mod W) for all heads; lane j4 owns dims 4 j4 .. 4 j4 + 3
-  {
-    float4 acc[HG];
-#pragma unroll
-    for (int r = 0; r < HG; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-    for (int s2 = warp; s2 < S; s2 += W) {
-#pragma unroll
-      for (int r = 0; r < HG; ++r) {
-        if (r < nh) {
-          const float f = wt[r * S + s2];
-          const float4 o = __ldcg(reinterpret_cast<const float4*>(part0 + ((int64_t)r * S + s2) * PART + 4 + 4 * lane));
-          acc[r].x = fmaf(f, o.x, acc[r].x);
-          acc[r].y = fmaf(f, o.y, acc[r].y);
-          acc[r].z = fmaf(f, o.z, acc[r].z);
-          acc[r].w = fmaf(f, o.w, acc[r].w);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < HG; ++r)
-      if (r < nh) *reinterpret_cast<float4*>(red + (warp * HG + r) * D + 4 * lane) = acc[r];
-  }
-  __syncthreads();
-  // phase 4: o' = (sum over warps) / L
-  for (int idx = tid; idx < nh * D; idx += T) {
-    const int r = idx / D, d = idx % D;
-    float O = 0.0f;
-#pragma unroll
-    for (int g = 0; g < W; ++g) O += red[(g * HG + r) * D + d];
-    ob[idx] = Lr[r] > 0.0f ? O / Lr[r] : 0.0f;
-  }
-  __syncthreads();
-  if (tid >= D) return;
-  // phase 5: o_i = sum_j Pi[j][i] o'_j (thread i; rows of Pi coalesced across threads), the next
-  // 16 rows loaded while the current ones are used
-  constexpr int JB = 16;
-  float acc[HG], pj[JB];
-#pragma unroll
-  for (int r = 0; r < HG; ++r) acc[r] = 0.0f;
-#pragma unroll
-  for (int jj = 0; jj < JB; ++jj) pj[jj] = __ldg(Pi + jj * D + tid);
-#pragma unroll 1
-  for (int j0 = 0; j0 < D; j0 += JB) {
-    float nx[JB];
-    if (j0 + JB < D) {
-#pragma unroll
-      for (int jj = 0; jj < JB; ++jj) nx[jj] = __ldg(Pi + (j0 + JB + jj) * D + tid);
-    }
-#pragma unroll
-    for (int jj = 0; jj < JB; ++jj)
-#pragma unroll
-      for (int r = 0; r < HG; ++r) acc[r] = fmaf(pj[jj], ob[r * D + j0 + jj], acc[r]);
-#pragma unroll
-    for (int jj = 0; jj < JB; ++jj) pj[jj] = nx[jj];
-  }
-  for (int r = 0; r < nh; ++r) out[((int64_t)b * Hq + h0 + r) * D + tid] = acc[r];
+  __syncthreads();  // red is reused by the next reduction
+  return v;
 }
+
+__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* __restrict__ part,
+                                                              const float* __restrict__ Pi,
+                                                              float* __restrict__ out, int S) {
+  extern __shared__ __align__(16) float msm[];  // [S] weights, [S] sums, [4][D] partial o', [D] o', [4][D]
+  __shared__ float red[32];
+  const int tid = threadIdx.x, d = tid % D, q = tid / D;
+  // Pi is an input, not an output of split: its rows load while the split grid finishes
+  float pj[32];
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) pj[jj] = __ldg(Pi + (32 * q + jj) * D + d);
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  const int64_t bh = blockIdx.x;
+  const float* p = part + bh * S * PART;
+  float* wts = msm;
+  float* ls = wts + S;
+  float* osum = ls + ((S + 3) & ~3);
+  float* ob = osum + 4 * D;
+  float* rsum = ob + D;
+  // phase 1: (max, sum) of every partial
+  float m = -INFINITY;
+  for (int s2 = tid; s2 < S; s2 += MERGE_THREADS) {
+    const float2 ml = *reinterpret_cast<const float2*>(p + (int64_t)s2 * PART);
+    wts[s2] = ml.x;
+    ls[s2] = ml.y;
+    m = fmaxf(m, ml.x);
+  }
+  const float M = block_reduce(m, red, true);
+  // phase 2: weights 2^(m_s - M) and L = sum_s w_s l_s
+  float l = 0.0f;
+  for (int s2 = tid; s2 < S; s2 += MERGE_THREADS) {
+    const float ms = wts[s2];
+    const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
+    wts[s2] = f;
+    l = fmaf(f, ls[s2], l);
+  }
+  const float L = block_reduce(l, red, false);  // also makes the weights visible
+  // phase 3: thread (d, q) sums splits q, q + 4, ...
+  float acc = 0.0f;
+#pragma unroll 16
+  for (int s2 = q; s2 < S; s2 += 4) acc = fmaf(wts[s2], p[(int64_t)s2 * PART + 4 + d], acc);
+  osum[q * D + d] = acc;
+  __syncthreads();
+  if (tid < D) {
+    const float o = osum[d] + osum[D + d] + osum[2 * D + d] + osum[3 * D + d];
+    ob[d] = L > 0.0f ? o / L : 0.0f;
+  }
+  __syncthreads();
+  // phase 4: o_i = sum_j Pi[j][i] o'_j, thread (i = d, q) over rows 32q .. 32q + 31
+  float r = 0.0f;
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) r = fmaf(pj[jj], ob[32 * q + jj], r);
+  rsum[q * D + d] = r;
+  __syncthreads();
+  if (tid < D) out[bh * D + d] = rsum[d] + rsum[D + d] + rsum[2 * D + d] + rsum[3 * D + d];
+}
+
+inline size_t merge_smem_bytes(int S) { return sizeof(float) * ((size_t)S + ((S + 3) & ~3) + 9 * D); }
 
 // Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (m8n8 fragment layout).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -585,6 +561,8 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::THREADS, Cfg<KB, VB>::MIN_BLOCKS)
 
   // Everything above reads only the cache; the rotated queries come from the prep kernel.
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // the merge kernel may launch now; its CTAs wait for this grid to finish before reading
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   // B operands: column gq of n-block nb = head 4 nb + gq/2, part gq%2 (0: fp16 hi, 1: fp16 lo);
   // k-step kk: dims 16kk + 2t, +1 (reg 0) and 16kk + 8 + 2t, +1 (reg 1).
@@ -803,18 +781,6 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::THREADS, Cfg<KB, VB>::MIN_BLOCKS)
     }
   }
 
-  // ---- the last CTA of this (batch, kv-head, head group) merges all splits and un-rotates ----
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int unit = (b * a.Hkv + kvh) * a.hgroups + hg;
-    s_last = atomicAdd(&a.counters[unit], 1) == a.splits - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  merge_splits<WARPS>(a.part, a.Pi, a.out, a.Hq, a.splits, b, h0, nh, smem);
 }
 
 // ------------------------------------------------------------------------------------------ host
@@ -866,11 +832,10 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms, int resident, int s
   return p;
 }
 
-// Workspace: q' and S q' [B*Hq][128] fp32, split partials [B*Hq][splits][132] fp32, then one
-// completion counter per (batch, kv-head, head group).
+// Workspace: q' and S q' [B*Hq][128] fp32, then the split partials [B*Hq][splits][132] fp32.
 size_t workspace_bytes(int B, int Hq, int Hkv, const Plan& p) {
-  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART) +
-         sizeof(int) * (size_t)B * Hkv * p.hgroups;
+  (void)Hkv;
+  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART);
 }
 
 template <int KB, int VB, bool QJL, int NB>
@@ -982,21 +947,16 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   const int BH = B * Hq;
-  const int n_counters = B * cache->Hkv * plan.hgroups;
-  a.counters = reinterpret_cast<int*>(ws + (size_t)2 * BH * D + (size_t)BH * plan.splits * PART);
-  a.Pi = params->Pi;
-  a.out = out;
   // heads per cluster: about 16 clusters at least (one CTA on each of 128 SMs), at most PREP_HB
   const int hb = std::max(1, std::min(PREP_HB, BH / 16));
   const int prep_ctas = (BH + hb - 1) / hb * PREP_CLUSTER;
   if (q_dtype == TQ_F32)
     prep_kernel<float><<<prep_ctas, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), BH, hb, params->Pi,
-                                                           params->S, cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D,
-                                                           a.counters, n_counters);
+                                                           params->S, cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D);
   else
     prep_kernel<__nv_bfloat16><<<prep_ctas, PREP_THREADS, 0, s>>>(
         reinterpret_cast<const __nv_bfloat16*>(q), BH, hb, params->Pi, params->S, cache->qjl_m ? 1 : 0, ws,
-        ws + (size_t)BH * D, a.counters, n_counters);
+        ws + (size_t)BH * D);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
 
@@ -1004,6 +964,19 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, a, grid, s)
                     : dispatch<false>(cache->k_bits, cache->v_bits, a, grid, s);
   if (st != TQ_OK) return st;
+  // merge: programmatic dependent of split (its CTAs wait for the split grid before reading)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(BH);
+  cfg.blockDim = dim3(MERGE_THREADS);
+  cfg.dynamicSmemBytes = merge_smem_bytes(plan.splits);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, merge_kernel, (const float*)a.part, params->Pi, out, plan.splits);
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
 
