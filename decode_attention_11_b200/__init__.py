@@ -35,7 +35,7 @@ TQ_BF16 = 1
 # Functions declared in include/tq.h (checked by the test-suite against the header).
 EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codebook",
             "tq_quantize", "tq_quantize_device_errors", "tq_quantize_vector_fixups",
-            "tq_quantize_code_fixups",
+            "tq_quantize_code_fixups", "tq_quantize_exempt_codes", "tq_quantize_exempt_signs",
             "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
             "tq_decode_static_workspace_limit", "tq_sketch_rotation", "tq_build_hadamard_rotation",
             "tq_decode_step")
@@ -93,6 +93,10 @@ def lib() -> ctypes.CDLL:
     L.tq_quantize_vector_fixups.argtypes = []
     L.tq_quantize_code_fixups.restype = ctypes.c_longlong
     L.tq_quantize_code_fixups.argtypes = []
+    L.tq_quantize_exempt_codes.restype = ctypes.c_longlong
+    L.tq_quantize_exempt_codes.argtypes = []
+    L.tq_quantize_exempt_signs.restype = ctypes.c_longlong
+    L.tq_quantize_exempt_signs.argtypes = []
     L.tq_decode_workspace_size.restype = ctypes.c_size_t
     L.tq_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache),
                                            ctypes.c_int]
@@ -301,6 +305,17 @@ def quantize_code_fixups() -> int:
     return int(lib().tq_quantize_code_fixups())
 
 
+def quantize_exempt_codes() -> int:
+    """Coordinates so far whose exact rotated value lay within 1e-6 of a threshold (the cases the
+    parity rule exempts; divide by 256 per quantized (token, kv-head) for the fraction)."""
+    return int(lib().tq_quantize_exempt_codes())
+
+
+def quantize_exempt_signs() -> int:
+    """QJL sketch values so far that were flagged near 0 and lay within 1e-5 of 0 exactly."""
+    return int(lib().tq_quantize_exempt_signs())
+
+
 def decode_workspace_size(B: int, Hq: int, cache: Cache, seq_len: int) -> int:
     c = cache.as_c()
     return int(lib().tq_decode_workspace_size(int(B), int(Hq), ctypes.byref(c), int(seq_len)))
@@ -383,7 +398,8 @@ __all__ = [
     "LIB_PATH", "EXPORTED", "TqError", "lib", "status_string", "last_error", "version",
     "build_codebook", "Params", "Cache", "quantize", "quantize_device_errors",
     "decode_attn_static", "decode_static_workspace_limit",
-    "quantize_vector_fixups", "quantize_code_fixups", "decode_workspace_size", "decode_attn",
+    "quantize_vector_fixups", "quantize_code_fixups", "quantize_exempt_codes", "quantize_exempt_signs",
+    "decode_workspace_size", "decode_attn",
     "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
     "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16",
 ]

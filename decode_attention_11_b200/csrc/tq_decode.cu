@@ -384,7 +384,9 @@ __device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) 
   return v;
 }
 
-__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* __restrict__ part,
+// (The partials are written by the still-running split grid: they are read with ld.global.cg,
+// through L2 only, never through the non-coherent read-only path.)
+__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
                                                               const float* __restrict__ Pi,
                                                               float* __restrict__ out, int S) {
   extern __shared__ __align__(16) float msm[];  // [S] weights, [S] sums, [4][D] partial o', [D] o', [4][D]
@@ -405,7 +407,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* __res
   // phase 1: (max, sum) of every partial
   float m = -INFINITY;
   for (int s2 = tid; s2 < S; s2 += MERGE_THREADS) {
-    const float2 ml = *reinterpret_cast<const float2*>(p + (int64_t)s2 * PART);
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p + (int64_t)s2 * PART));
     wts[s2] = ml.x;
     ls[s2] = ml.y;
     m = fmaxf(m, ml.x);
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* __res
   // phase 3: thread (d, q) sums splits q, q + 4, ...
   float acc = 0.0f;
 #pragma unroll 16
-  for (int s2 = q; s2 < S; s2 += 4) acc = fmaf(wts[s2], p[(int64_t)s2 * PART + 4 + d], acc);
+  for (int s2 = q; s2 < S; s2 += 4) acc = fmaf(wts[s2], __ldcg(p + (int64_t)s2 * PART + 4 + d), acc);
   osum[q * D + d] = acc;
   __syncthreads();
   if (tid < D) {

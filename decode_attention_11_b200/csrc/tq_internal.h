@@ -16,6 +16,11 @@ namespace tq {
 
 constexpr int kHeadDim = 128;
 constexpr int kQjlRows = 128;
+// Comparison bands of the parity rules: a coordinate within kExemptCodeBand of a threshold (in u
+// units), or a sketch value within kExemptSignBand of 0, is decided by rounding; the quantize
+// kernels count such cases (tq_quantize_exempt_codes / _signs).
+constexpr double kExemptCodeBand = 1e-6;
+constexpr double kExemptSignBand = 1e-5;
 
 // Thread-local error detail; returns `st` so callers can `return fail(...)`.
 tq_status fail(tq_status st, const char* fmt, ...);
@@ -48,6 +53,8 @@ tq_status quantize_bf16_pipeline(const tq_params* p, const void* k, const void* 
 unsigned int pipe_device_errors();
 long long pipe_vector_fixups();
 long long pipe_code_fixups();
+long long pipe_exempt_codes();
+long long pipe_exempt_signs();
 
 // Validation shared by tq_quantize / tq_decode_attn.
 tq_status check_params(const tq_params* p, const tq_cache* c);

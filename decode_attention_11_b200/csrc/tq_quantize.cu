@@ -56,6 +56,8 @@ struct Guards {
 __device__ unsigned int g_quantize_error;          // bit 0: a wait timed out; bit 1: misaligned smem
 __device__ unsigned int g_quantize_vector_fixups;  // key vectors re-derived in fp64 (diagnostic)
 __device__ unsigned int g_quantize_code_fixups;    // coordinates re-derived in fp64 (diagnostic)
+__device__ unsigned int g_quantize_exempt_codes;   // exact u within kExemptCodeBand of a threshold
+__device__ unsigned int g_quantize_exempt_signs;   // exact sketch value within kExemptSignBand of 0
 
 struct QArgs {
   const void* k;
@@ -105,6 +107,7 @@ struct __align__(1024) Smem {
   uint8_t fcode[D];
   uint8_t fsign[D];
   int nfl, nvfl;
+  unsigned int nexc, nexs;  // exempt codes / signs found by this tile's fp64 fixups
   uint64_t bar_kv, bar_s;
   uint32_t tmem_base;
   unsigned int err;
@@ -219,6 +222,12 @@ __device__ __forceinline__ int code_exact(double u, const float* thr, int nthr) 
   int idx = 0;
   for (int i = 0; i < nthr; ++i) idx += (u >= (double)thr[i]) ? 1 : 0;
   return idx;
+}
+// Whether an exact coordinate lies within kExemptCodeBand of one of the nthr thresholds.
+__device__ __forceinline__ bool code_exempt_exact(double u, const float* thr, int nthr) {
+  bool near = false;
+  for (int i = 0; i < nthr; ++i) near = near || fabs(u - (double)thr[i]) <= kExemptCodeBand;
+  return near;
 }
 
 // Read / replace the b-bit code at slot `slot` of a staged row (32-bit shared words).
@@ -418,6 +427,8 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
     if (tid == 0) {
       s.nfl = 0;
       s.nvfl = 0;
+      s.nexc = 0;
+      s.nexs = 0;
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -589,6 +600,7 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
         if (!have || (tid & 3)) continue;
         const double nn = val ? s.nrmv[rr] : s.nrmk[rr];
         const double ud = sqrt((double)D) * dot / nn;
+        if (code_exempt_exact(ud, val ? s.vthr : s.kthr, (val ? LV : LK) - 1)) atomicAdd(&s.nexc, 1u);
         if (val) {
           const uint32_t idx = (uint32_t)code_exact(ud, s.vthr, LV - 1);
           uint8_t* row = s.vst + rr * (16 * VB);
@@ -654,6 +666,8 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
             const double dot = quad_sum(exact_dot_part<InT>(a.Pi, vx, j, tid & 3));
             if ((tid & 3) == 0) {
               const int idx = nv > 0.0 ? code_exact(sqrt((double)D) * dot / nv, s.vthr, LV - 1) : LV / 2;
+              // (a row whose near-threshold list overflowed: its coordinates are counted here)
+              if (nv > 0.0 && code_exempt_exact(sqrt((double)D) * dot / nv, s.vthr, LV - 1)) atomicAdd(&s.nexc, 1u);
               s.fcode[v_slot_of_coord(j)] = (uint8_t)idx;
             }
           }
@@ -680,6 +694,7 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
             if (nk > 0.0) {
               const double ud = sqrt((double)D) * dot / nk;
               idx = code_exact(ud, s.kthr, LK - 1);
+              if ((fl & 2) && code_exempt_exact(ud, s.kthr, LK - 1)) atomicAdd(&s.nexc, 1u);
               rho = ud - (double)s.kcent[idx];
             } else {
               idx = LK / 2;
@@ -703,7 +718,10 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
             sp1 = fma((double)__half2float(*reinterpret_cast<const __half*>(s.sm + sw_off(l, j + 1))), s.fx64[j + 1], sp1);
           }
           const double sp = quad_sum(sp0 + sp1);
-          if (q == 0) s.fsign[sign_bit_of_row(l)] = sp >= 0.0 ? 1 : 0;
+          if (q == 0) {
+            s.fsign[sign_bit_of_row(l)] = sp >= 0.0 ? 1 : 0;
+            if (fabs(sp) <= kExemptSignBand) atomicAdd(&s.nexs, 1u);
+          }
         }
         __syncthreads();
         if (tid < 4 * KB) {
@@ -727,6 +745,8 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
       }
       if (tid < TM) s.vflag[tid] = 0;
       if (tid == 0 && nvf) atomicAdd(&g_quantize_vector_fixups, (unsigned)nvf);
+      if (tid == 0 && s.nexc) atomicAdd(&g_quantize_exempt_codes, s.nexc);
+      if (tid == 0 && s.nexs) atomicAdd(&g_quantize_exempt_signs, s.nexs);
     }
 
     // ---- 6. coalesced stores of the tile's rows ----
@@ -904,5 +924,19 @@ extern "C" long long tq_quantize_code_fixups(void) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, tq::g_quantize_code_fixups, sizeof(v)) != cudaSuccess) return -1;
   const long long p = tq::pipe_code_fixups();
+  return p < 0 ? -1 : (long long)v + p;
+}
+
+extern "C" long long tq_quantize_exempt_codes(void) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tq::g_quantize_exempt_codes, sizeof(v)) != cudaSuccess) return -1;
+  const long long p = tq::pipe_exempt_codes();
+  return p < 0 ? -1 : (long long)v + p;
+}
+
+extern "C" long long tq_quantize_exempt_signs(void) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tq::g_quantize_exempt_signs, sizeof(v)) != cudaSuccess) return -1;
+  const long long p = tq::pipe_exempt_signs();
   return p < 0 ? -1 : (long long)v + p;
 }

@@ -62,6 +62,11 @@ constexpr float C_SCALE = 0.04419417382415922f;   // sqrt(128) / 256 (u = y * C_
 __device__ unsigned int g_pipe_error;         // bit 0: a wait timed out; bit 1: smem misaligned; bit 2: no LUT
 __device__ unsigned int g_pipe_vector_fixups;
 __device__ unsigned int g_pipe_code_fixups;
+// Coordinates whose exact (fp64) u lies within kExemptCodeBand of a threshold, and sketch values
+// flagged near 0 whose exact value lies within kExemptSignBand of 0 (both counted once, in the
+// fp64 fixups, which every such case reaches: the fast path's error is far inside its guard bands).
+__device__ unsigned int g_pipe_exempt_codes;
+__device__ unsigned int g_pipe_exempt_signs;
 // Launch epoch of the fixup ring: read by every CTA at start, advanced by the last CTA to finish,
 // so consecutive launches on a stream (CUDA graph replays included) never share an epoch.
 __device__ unsigned int g_pipe_epoch;
@@ -479,6 +484,12 @@ __device__ __forceinline__ uint32_t code_lut(double u, const uint32_t* lut, floa
   const uint32_t L = lut[__float_as_uint(fmaf((float)u, alpha, CELL_MAGIC)) & (LUT_N - 1)];
   return (L & 15u) + (u >= (double)__uint_as_float(L & ~15u) ? 1u : 0u);
 }
+// Whether an exact coordinate lies within kExemptCodeBand of a threshold.  A value that close to a
+// threshold always falls in that threshold's cell (thresholds sit at least 0.05 cells from an edge).
+__device__ __forceinline__ bool code_exempt(double u, const uint32_t* lut, float alpha) {
+  const uint32_t L = lut[__float_as_uint(fmaf((float)u, alpha, CELL_MAGIC)) & (LUT_N - 1)];
+  return fabs(u - (double)__uint_as_float(L & ~15u)) <= kExemptCodeBand;
+}
 // Lane holds x[4 lane .. 4 lane + 3]; returns the exact dot product of Pi row j with x.
 __device__ __forceinline__ double pi_dot(const float* __restrict__ Pi, int j, const double (&x)[4]) {
   const int lane = threadIdx.x & 31;
@@ -576,7 +587,7 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
   const int64_t in_off = (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)t * a.st;
   const int64_t row = ((int64_t)b * a.Hkv + h) * a.T_cap + a.t_offset + t;
   const double sqd = sqrt((double)D);
-  unsigned int ncodes = 0;
+  unsigned int ncodes = 0, nexempt = 0;
   if (E.flags & 2) {
     double x[4];
     load_row(a.v + in_off, x);
@@ -590,12 +601,15 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
         const double dot = pi_dot(a.Pi, j, x);
         const uint32_t code = n > 0.0 ? code_lut(sqd * dot / n, s.vlut, s.alpha_v) : (uint32_t)(LV / 2);
         if (lane == 0 && get_code(vrow, VB, v_slot_of_coord(j)) != code) set_code(vrow, VB, v_slot_of_coord(j), code);
+        if (n > 0.0 && code_exempt(sqd * dot / n, s.vlut, s.alpha_v)) ++nexempt;
         ++ncodes;
       }
     }
   }
   if (lane == 0 && ncodes) atomicAdd(&g_pipe_code_fixups, ncodes);
+  if (lane == 0 && nexempt) atomicAdd(&g_pipe_exempt_codes, nexempt);
   ncodes = 0;
+  nexempt = 0;
   bool vec = false;  // a key code changed: every sign and ||r|| are re-derived
   if (!(E.flags & 5)) return;
   double x[4];
@@ -610,6 +624,7 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
         m &= m - 1;
         const double dot = pi_dot(a.Pi, j, x);
         const uint32_t code = nk > 0.0 ? code_lut(sqd * dot / nk, s.klut, s.alpha_k) : (uint32_t)(LK / 2);
+        if (nk > 0.0 && code_exempt(sqd * dot / nk, s.klut, s.alpha_k)) ++nexempt;
         const uint32_t old = __shfl_sync(0xffffffffu, lane == 0 ? get_code(krow, KB, k_slot_of_coord(j)) : 0u, 0);
         if (old != code) {
           if (lane == 0) set_code(krow, KB, k_slot_of_coord(j), code);
@@ -620,6 +635,8 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
     }
   }
   if (lane == 0 && ncodes) atomicAdd(&g_pipe_code_fixups, ncodes);
+  if (lane == 0 && nexempt) atomicAdd(&g_pipe_exempt_codes, nexempt);
+  nexempt = 0;
   if (!a.qjl || (!vec && !(E.flags & 4))) return;
   if (!vec && !(E.flags & 8) && a.SPi != nullptr && nk > 0.0 && nk <= 1e300) {
     // The stored codes are final: (S rho)_l = sqrt(128)/||x|| ((S Pi) x)_l - (S c[idx])_l.
@@ -650,9 +667,13 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
           if (sp >= 0.0) atomicOr(&srow[bit >> 5], 1u << (bit & 31));
           else atomicAnd(&srow[bit >> 5], ~(1u << (bit & 31)));
         }
+        if (fabs(sp) <= kExemptSignBand) ++nexempt;
       }
     }
-    if (lane == 0) atomicAdd(&g_pipe_vector_fixups, 1u);
+    if (lane == 0) {
+      atomicAdd(&g_pipe_vector_fixups, 1u);
+      if (nexempt) atomicAdd(&g_pipe_exempt_signs, nexempt);
+    }
     return;
   }
   // Exact residual of the whole key vector (fp64): u, codes, rho.
@@ -689,9 +710,13 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
           if (sp >= 0.0) atomicOr(&srow[bit >> 5], 1u << (bit & 31));
           else atomicAnd(&srow[bit >> 5], ~(1u << (bit & 31)));
         }
+        if (fabs(sp) <= kExemptSignBand) ++nexempt;
       }
     }
-    if (lane == 0) atomicAdd(&g_pipe_vector_fixups, 1u);
+    if (lane == 0) {
+      atomicAdd(&g_pipe_vector_fixups, 1u);
+      if (nexempt) atomicAdd(&g_pipe_exempt_signs, nexempt);
+    }
     return;
   }
   matvec8(a.S, rl, [&](int l, double sp) { s.fsign[w][sign_bit_of_row(l)] = sp >= 0.0 ? 1 : 0; });
@@ -1381,6 +1406,16 @@ long long pipe_vector_fixups() {
 long long pipe_code_fixups() {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_pipe_code_fixups, sizeof(v)) != cudaSuccess) return -1;
+  return v;
+}
+long long pipe_exempt_codes() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pipe_exempt_codes, sizeof(v)) != cudaSuccess) return -1;
+  return v;
+}
+long long pipe_exempt_signs() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pipe_exempt_signs, sizeof(v)) != cudaSuccess) return -1;
   return v;
 }
 

@@ -183,6 +183,21 @@ int tq_quantize_device_errors(void);
 long long tq_quantize_vector_fixups(void);
 /* Number of single coordinates whose code was re-derived in fp64 (value near a threshold). */
 long long tq_quantize_code_fixups(void);
+/*
+ * Exemption counts of the comparison rule for codes and signs (cumulative since the library was
+ * loaded; host, synchronizes with the device; -1 if the device could not be queried).  The
+ * method's parity rule lets a code differ from the float64 definition only where the rotated
+ * coordinate u lies within 1e-6 of a decision threshold, and asks for the fraction of such
+ * cases to be reported.  The fast path's error is far inside its fp64 guard bands, so every such
+ * coordinate is re-derived in fp64, where it is counted:
+ *   tq_quantize_exempt_codes   coordinates (keys and values) whose exact u lies within 1e-6 of a
+ *                              threshold.  Divide by 256 per (token, kv-head) quantized for the
+ *                              fraction.
+ *   tq_quantize_exempt_signs   QJL sketch values that the fast path flagged near 0 and whose exact
+ *                              value lies within 1e-5 of 0 (normalized units).
+ */
+long long tq_quantize_exempt_codes(void);
+long long tq_quantize_exempt_signs(void);
 
 /*
  * Bytes of device workspace tq_decode_attn needs for these sizes on the current device
@@ -256,6 +271,9 @@ tq_status tq_decode_attn_static(const tq_params* params, const void* q, int q_dt
                                 const tq_cache* cache, int seq_len, float scale, float* out,
                                 void* stream);
 
+/* The device address of the array is looked up once per device and kept for the life of the
+ * process: after a cudaDeviceReset (or any reset of the primary context) this entry point must not
+ * be called again in the same process. */
 /* Size in bytes of the static scratch array used by tq_decode_attn_static. */
 size_t tq_decode_static_workspace_limit(void);
 

@@ -31,69 +31,148 @@ def params_for(w: W.Workload, device="cuda") -> tq.Params:
     return tq.Params.create(W.rotation_for(w), W.qjl_for(w), w.k_bits, w.v_bits, device=device)
 
 
-def compare_quantized(w: W.Workload, cache: tq.Cache, Kh, Vh, t_offset: int, rows=None) -> dict:
-    """Compare GPU cache rows with the oracle's quantization of the exact inputs.
-
-    Kh, Vh: float64 [B, H, T, 128] inputs written at cache rows [t_offset, t_offset + T); or, with
-    rows = [(b, h, t), ...], float64 [len(rows), 128] input vectors for exactly those rows.
-    Returns counts; asserts the comparison rules."""
+def compare_rows(w: W.Workload, cache: tq.Cache, kx, vx, bi, hi, ti) -> dict:
+    """Compare the GPU cache rows (bi, hi, ti) (index arrays) with the oracle's quantization of
+    the exact float64 input vectors kx, vx ([n, 128]) under the comparison rules; asserts them and
+    returns counts (coordinates, exempt cases, in-band differences)."""
     Pi, S = W.rotation_for(w), W.qjl_for(w)
-    if rows is None:
-        B, H, T, _ = Kh.shape
-        rows = [(b, h, t) for b in range(B) for h in range(H) for t in range(T)]
-        bi = np.array([r[0] for r in rows])
-        hi = np.array([r[1] for r in rows])
-        ti = np.array([r[2] for r in rows])
-        kx = Kh[bi, hi, ti]
-        vx = Vh[bi, hi, ti]
-    else:
-        bi = np.array([r[0] for r in rows])
-        hi = np.array([r[1] for r in rows])
-        ti = np.array([r[2] for r in rows])
-        kx, vx = np.asarray(Kh, np.float64), np.asarray(Vh, np.float64)
+    kx, vx = np.asarray(kx, np.float64), np.asarray(vx, np.float64)
     kq = O.quantize_vectors(kx, Pi, w.k_bits, S)
     vq = O.quantize_vectors(vx, Pi, w.v_bits, None)
-    tc = ti + t_offset
     dev = cache.k_codes.device
-    ib, ih, it = (torch.as_tensor(x, device=dev) for x in (bi, hi, tc))
+    ib, ih, it = (torch.as_tensor(np.asarray(x), device=dev) for x in (bi, hi, ti))
     g = lambda t: t[ib, ih, it].cpu().numpy()
     k_codes, v_codes = g(cache.k_codes), g(cache.v_codes)
     k_norm, v_norm = g(cache.k_norm), g(cache.v_norm)
-    k_idx = O.unpack_codes(k_codes, w.k_bits, O.k_slot_of_coord)
-    v_idx = O.unpack_codes(v_codes, w.v_bits, O.v_slot_of_coord)
     k_ex = O.code_exempt(kq["u"], w.k_bits)
     v_ex = O.code_exempt(vq["u"], w.v_bits)
-    k_bad = (k_idx != kq["idx"]) & ~k_ex
-    v_bad = (v_idx != vq["idx"]) & ~v_ex
-    assert not k_bad.any(), f"key codes differ outside the exemption band at {np.argwhere(k_bad)[:5]}"
-    assert not v_bad.any(), f"value codes differ outside the exemption band at {np.argwhere(v_bad)[:5]}"
-    # rows with no exempt coordinate must be byte-identical to the oracle's packing
     k_rows_clean = ~k_ex.any(1)
     v_rows_clean = ~v_ex.any(1)
-    assert np.array_equal(k_codes[k_rows_clean], O.pack_codes(kq["idx"], w.k_bits, O.k_slot_of_coord)[k_rows_clean])
-    assert np.array_equal(v_codes[v_rows_clean], O.pack_codes(vq["idx"], w.v_bits, O.v_slot_of_coord)[v_rows_clean])
+    # rows with no exempt coordinate must be byte-identical to the oracle's packing
+    k_want = O.pack_codes(kq["idx"], w.k_bits, O.k_slot_of_coord)
+    v_want = O.pack_codes(vq["idx"], w.v_bits, O.v_slot_of_coord)
+    kb = np.flatnonzero(~np.all(k_codes == k_want, axis=1) & k_rows_clean)
+    vb = np.flatnonzero(~np.all(v_codes == v_want, axis=1) & v_rows_clean)
+    assert kb.size == 0, f"key code rows differ from the oracle at {kb[:5]}"
+    assert vb.size == 0, f"value code rows differ from the oracle at {vb[:5]}"
+    # rows with an exempt coordinate: every other coordinate must match
+    k_in_band = v_in_band = 0
+    if (~k_rows_clean).any():
+        r = ~k_rows_clean
+        got = O.unpack_codes(k_codes[r], w.k_bits, O.k_slot_of_coord)
+        diff = got != kq["idx"][r]
+        assert not (diff & ~k_ex[r]).any(), "key codes differ outside the exemption band"
+        k_in_band = int(diff.sum())
+    if (~v_rows_clean).any():
+        r = ~v_rows_clean
+        got = O.unpack_codes(v_codes[r], w.v_bits, O.v_slot_of_coord)
+        diff = got != vq["idx"][r]
+        assert not (diff & ~v_ex[r]).any(), "value codes differ outside the exemption band"
+        v_in_band = int(diff.sum())
     # Stored norms: the bf16 path sums the 128 exact squares in fp32 (chains of 8 fmas, then a
     # 4-level tree: relative error <= 11 * 2^-24 on ||x||^2, 5.5 * 2^-24 on ||x||), takes a
     # correctly rounded sqrt (<= 2^-24) and is compared with the oracle's fp32 rounding of the exact
     # norm (<= 2^-24): |diff| <= 7.5 * 2^-24 * ||x|| <= 7.5 ulp.
     assert ulp_distance_f32(k_norm, kq["n"].astype(np.float32)).max() <= NORM_ULP
     assert ulp_distance_f32(v_norm, vq["n"].astype(np.float32)).max() <= NORM_ULP
-    out = {"coords": k_idx.size + v_idx.size,
+    out = {"vectors": int(kx.shape[0]), "coords": int(kq["idx"].size + vq["idx"].size),
            "exempt_codes": int(k_ex.sum() + v_ex.sum()),
-           "code_mismatch_in_band": int(((k_idx != kq["idx"]) & k_ex).sum() + ((v_idx != vq["idx"]) & v_ex).sum())}
+           "code_mismatch_in_band": k_in_band + v_in_band}
     if w.qjl_m:
-        signs = O.unpack_signs(g(cache.k_signs))
+        k_signs = g(cache.k_signs)
         s_ex = O.sign_exempt(kq["sproj"], k_ex)
-        s_bad = (signs != kq["signs"]) & ~s_ex
-        assert not s_bad.any(), f"sign bits differ outside the exemption band at {np.argwhere(s_bad)[:5]}"
+        s_rows_clean = ~s_ex.any(1)
+        s_want = O.pack_signs(kq["signs"])
+        sb = np.flatnonzero(~np.all(k_signs == s_want, axis=1) & s_rows_clean)
+        assert sb.size == 0, f"sign rows differ from the oracle at {sb[:5]}"
+        s_in_band = 0
+        if (~s_rows_clean).any():
+            r = ~s_rows_clean
+            diff = O.unpack_signs(k_signs[r]) != kq["signs"][r]
+            assert not (diff & ~s_ex[r]).any(), "sign bits differ outside the exemption band"
+            s_in_band = int(diff.sum())
         rn = g(cache.k_rnorm).astype(np.float64)
         ref = kq["rnorm"]
-        clean = ~k_ex.any(1)
+        clean = k_rows_clean
         err = np.abs(rn - ref)[clean]
         assert (err <= 1e-5 * ref[clean] + 1e-30).all(), (err / np.maximum(ref[clean], 1e-30)).max()
+        out["sign_bits"] = int(kq["signs"].size)
         out["exempt_signs"] = int(s_ex.sum())
-        out["sign_mismatch_in_band"] = int(((signs != kq["signs"]) & s_ex).sum())
+        out["near_zero_signs"] = int((np.abs(kq["sproj"]) <= O.SIGN_BAND).sum())
+        out["sign_mismatch_in_band"] = s_in_band
     return out
+
+
+def merge_counts(total: dict, part: dict) -> dict:
+    for k, v in part.items():
+        total[k] = total.get(k, 0) + v
+    return total
+
+
+def compare_quantized(w: W.Workload, cache: tq.Cache, Kh, Vh, t_offset: int, rows=None) -> dict:
+    """Compare GPU cache rows with the oracle's quantization of the exact inputs.
+
+    Kh, Vh: float64 [B, H, T, 128] inputs written at cache rows [t_offset, t_offset + T); or, with
+    rows = [(b, h, t), ...], float64 [len(rows), 128] input vectors for exactly those rows.
+    Returns counts; asserts the comparison rules."""
+    if rows is None:
+        B, H, T, _ = Kh.shape
+        bi, hi, ti = (a.reshape(-1) for a in np.meshgrid(np.arange(B), np.arange(H), np.arange(T),
+                                                         indexing="ij"))
+        kx = np.asarray(Kh, np.float64).reshape(-1, Kh.shape[-1])
+        vx = np.asarray(Vh, np.float64).reshape(-1, Vh.shape[-1])
+    else:
+        bi = np.array([r[0] for r in rows])
+        hi = np.array([r[1] for r in rows])
+        ti = np.array([r[2] for r in rows])
+        kx, vx = np.asarray(Kh, np.float64), np.asarray(Vh, np.float64)
+    return compare_rows(w, cache, kx, vx, bi, hi, ti + t_offset)
+
+
+def compare_full_cache(w: W.Workload, cache: tq.Cache, K: torch.Tensor, V: torch.Tensor,
+                       chunk_rows: int = 1 << 16) -> dict:
+    """Every row of a cache quantized from the device tensors K, V ([B, Hkv, T, 128], written at
+    rows 0..T-1) against the oracle, in chunks of rows; returns the summed counts."""
+    B, H, T, d = K.shape
+    Kf = K.reshape(B * H * T, d)
+    Vf = V.reshape(B * H * T, d)
+    total: dict = {}
+    for r0 in range(0, B * H * T, chunk_rows):
+        r1 = min(B * H * T, r0 + chunk_rows)
+        flat = np.arange(r0, r1)
+        bi, rem = np.divmod(flat, H * T)
+        hi, ti = np.divmod(rem, T)
+        kx = Kf[r0:r1].double().cpu().numpy()
+        vx = Vf[r0:r1].double().cpu().numpy()
+        merge_counts(total, compare_rows(w, cache, kx, vx, bi, hi, ti))
+    return total
+
+
+def exemption_free_inputs(w: W.Workload, spare: int = 64):
+    """K, V of the workload's recipe ([B, Hkv, T, 128], input dtype, CPU) in which no vector has a
+    coordinate within the code band of a threshold or a sketch value within the sign band of 0:
+    the recipe is drawn with T + spare tokens and, per (batch, kv-head), the first T vectors whose
+    K and V are both free of exempt cases are kept (about 0.3% of vectors are skipped).  On such
+    inputs the cache has exactly one correct value, so a GPU-written cache and the decode over it
+    can be compared with the oracle without exceptions."""
+    big = w.scaled(T=w.T + spare)
+    K = W.make_kv(big, "k")
+    V = W.make_kv(big, "v")
+    Pi, S = W.rotation_for(w), W.qjl_for(w)
+    Ko = torch.empty((w.B, w.Hkv, w.T, w.head_dim), dtype=K.dtype)
+    Vo = torch.empty_like(Ko)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            kq = O.quantize_vectors(K[b, h].double().numpy(), Pi, w.k_bits, S)
+            vq = O.quantize_vectors(V[b, h].double().numpy(), Pi, w.v_bits, None)
+            bad = O.code_exempt(kq["u"], w.k_bits).any(1) | O.code_exempt(vq["u"], w.v_bits).any(1)
+            if S is not None:
+                bad |= (np.abs(kq["sproj"]) <= O.SIGN_BAND).any(1)
+            keep = np.flatnonzero(~bad)[: w.T]
+            assert keep.size == w.T, "too few exemption-free vectors in the spare draw"
+            Ko[b, h] = K[b, h, torch.as_tensor(keep)]
+            Vo[b, h] = V[b, h, torch.as_tensor(keep)]
+    return Ko, Vo
 
 
 def attention_errors(got: np.ndarray, ref: np.ndarray):
@@ -122,5 +201,6 @@ def oracle_cache_arrays(w: W.Workload, Kh, Vh, T_cap=None):
 
 
 __all__ = ["ATTN_MAX_ABS", "ATTN_REL_L2", "EXEMPT_FRACTION_MAX", "ulp_distance_f32", "gpu_inputs",
-           "params_for", "compare_quantized", "attention_errors", "assert_attention_close",
+           "params_for", "compare_rows", "compare_quantized", "compare_full_cache", "merge_counts",
+           "exemption_free_inputs", "attention_errors", "assert_attention_close",
            "oracle_cache_arrays", "math", "torch"]

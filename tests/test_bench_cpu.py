@@ -25,7 +25,7 @@ def test_reference_arm_json_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
-    assert d["config"]["workload"] == "llama3_8b_32k"
+    assert d["config"]["workload"] == "llama3_8b_128k_b4"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -1,7 +1,10 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 CPU oracle.
 
-Small cases are compared element by element (several tiles plus a ragged tail); the full-size
-workloads are compared on sampled rows / heads that the oracle computes one by one."""
+Small cases are compared element by element (several tiles plus a ragged tail).  At full size,
+every quantized row of all five workloads is compared with the oracle, and decode is compared on
+the query heads of one (batch, kv-head) slice whose cache the oracle wrote.  Where a GPU-written
+cache feeds the decode, the inputs are drawn free of exempt cases so that the cache has exactly
+one correct value."""
 import dataclasses
 import math
 
@@ -13,8 +16,9 @@ import decode_attention_11_b200 as tq
 import workloads as W
 from oracle import tq_oracle as O
 
-from _parity import (EXEMPT_FRACTION_MAX, assert_attention_close, compare_quantized, gpu_inputs,
-                     oracle_cache_arrays, params_for)
+from _parity import (EXEMPT_FRACTION_MAX, assert_attention_close, compare_full_cache,
+                     compare_quantized, exemption_free_inputs, gpu_inputs, oracle_cache_arrays,
+                     params_for)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +52,10 @@ def test_quantize_parity_small(name):
     quantize_chunked(params, K, V, cache, t_off, w.chunk)
     torch.cuda.synchronize()
     stats = compare_quantized(w, cache, Kh, Vh, t_off)
-    assert stats["exempt_codes"] / stats["coords"] <= 10 * EXEMPT_FRACTION_MAX
+    # The fraction of exempt coordinates is a property of the data; on a few hundred vectors it is
+    # a count of a handful, so it is reported here and gated at full size (test_full_size_quantize).
+    print(f"{name}: {stats['exempt_codes']} exempt coordinates of {stats['coords']}, "
+          f"{stats['code_mismatch_in_band']} of them differ")
     # rows outside the written range are untouched
     for arr in (cache.k_codes, cache.v_codes, cache.k_norm, cache.v_norm):
         a = arr.cpu()
@@ -171,8 +178,8 @@ def test_decode_parity_small(name):
 
 
 def test_decode_ignores_workspace_contents():
-    """The workspace's previous contents (counters included) never change the result: filled with
-    0x00, 0xFF and 0x5A bytes, and reused across back-to-back calls on one stream."""
+    """The workspace's previous contents never change the result: filled with 0x00, 0xFF and 0x5A
+    bytes, and reused across back-to-back calls on one stream."""
     w = small("llama3_8b_32k")
     K, V, Kh, Vh = gpu_inputs(w)
     q = W.make_queries(w).cuda()
@@ -273,20 +280,29 @@ def test_decode_without_qjl():
         assert_attention_close(got, ref)
 
 
+def _clean_gpu_inputs(w):
+    K, V = exemption_free_inputs(w)
+    return K.cuda(), V.cuda(), K.double().numpy(), V.double().numpy()
+
+
 def test_quantize_then_decode_end_to_end():
+    """GPU quantize, then GPU decode over the GPU-written cache, against the oracle's quantize and
+    decode of the same inputs.  The inputs have no vector with an exempt code or sign, so the
+    cache has a single correct value: it is compared first, then the attention output."""
     w = small("llama3_8b_128k_b4")
     params = params_for(w)
-    K, V, Kh, Vh = gpu_inputs(w)
+    K, V, Kh, Vh = _clean_gpu_inputs(w)
     cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
     tq.quantize(params, K, V, cache)
     q = W.make_queries(w)
     out = tq.decode_attn(params, q.cuda(), cache, w.T).cpu().numpy()
+    torch.cuda.synchronize()
+    stats = compare_quantized(w, cache, Kh, Vh, 0)
+    assert stats["exempt_codes"] == 0 and stats["exempt_signs"] == 0
     _, oc = oracle_cache_arrays(w, Kh, Vh)
-    ex = O.code_exempt(oc["k_u"], w.k_bits).sum() + O.code_exempt(oc["v_u"], w.v_bits).sum()
     ref = O.decode_attention(q.double().numpy(), W.rotation_for(w), W.qjl_for(w), oc, w.k_bits,
                              w.v_bits, w.T)
-    if ex == 0:
-        assert_attention_close(out, ref)
+    assert_attention_close(out, ref)
     # Context, not a gate: error against exact attention on the uncompressed K/V.  The QJL term
     # makes the score unbiased but adds variance that the softmax amplifies (ai-news.ru overview,
     # paragraph on the third component), so on this outlier-heavy data the QJL-on error exceeds
@@ -300,19 +316,20 @@ def test_quantize_then_decode_end_to_end():
     assert rel_qjl < 1.0 and rel_mse < 1.0
 
 
-def test_decode_step_appends_and_attends():
+@pytest.mark.parametrize("name", ["llama3_8b_32k", "moe_1m"])
+def test_decode_step_appends_and_attends(name):
     """Autoregressive use: the first tokens by one tq_quantize, then one tq_decode_step per new
-    token (bf16 K/V rows written at row t, then attention over rows 0..t).  Each step matches the
-    oracle over the tokens so far, and the whole cache matches the oracle's quantization."""
-    w = small("llama3_8b_32k")
+    token (bf16 K/V rows written at row t, then attention over rows 0..t).  Every step's output is
+    compared with the oracle's decode over the oracle's cache of the tokens so far, and the whole
+    GPU-written cache with the oracle's quantization (inputs free of exempt cases)."""
+    w = small(name)
     params = params_for(w)
-    K, V, Kh, Vh = gpu_inputs(w)
+    K, V, Kh, Vh = _clean_gpu_inputs(w)
     T0 = w.T - 5
     cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
     tq.quantize(params, K[:, :, :T0], V[:, :, :T0], cache)
     q0 = W.make_queries(w)
     _, oc = oracle_cache_arrays(w, Kh, Vh)
-    ex = O.code_exempt(oc["k_u"], w.k_bits).sum() + O.code_exempt(oc["v_u"], w.v_bits).sum()
     for t in range(T0, w.T):
         q = q0 * (1.0 + 0.25 * (t - T0))
         out = tq.decode_step(params, K[:, :, t].contiguous(), V[:, :, t].contiguous(), q.cuda(), cache, t)
@@ -320,14 +337,14 @@ def test_decode_step_appends_and_attends():
         assert tq.quantize_device_errors() == 0
         ref = O.decode_attention(q.double().numpy(), W.rotation_for(w), W.qjl_for(w), oc, w.k_bits,
                                  w.v_bits, t + 1)
-        if ex == 0:
-            assert_attention_close(out.cpu().numpy(), ref)
-    compare_quantized(w, cache, Kh, Vh, 0)
+        assert_attention_close(out.cpu().numpy(), ref)
+    stats = compare_quantized(w, cache, Kh, Vh, 0)
+    assert stats["exempt_codes"] == 0
 
 
 # ------------------------------------------------------------------------------- full size
 
-FULL = ["llama3_8b_32k", "llama3_8b_128k_b4", "llama3_70b_16k_b16", "moe_1m"]
+FULL = ["single_head_4k", "llama3_8b_32k", "llama3_8b_128k_b4", "llama3_70b_16k_b16", "moe_1m"]
 
 
 def full_inputs(w):
@@ -336,28 +353,29 @@ def full_inputs(w):
     return K, V
 
 
-def sample_rows(w, n, rng):
-    rows = {(0, 0, 0), (w.B - 1, w.Hkv - 1, w.T - 1), (0, w.Hkv - 1, w.T // 2)}
-    while len(rows) < n:
-        rows.add((int(rng.integers(w.B)), int(rng.integers(w.Hkv)), int(rng.integers(w.T))))
-    return sorted(rows)
-
-
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_quantize_sampled(name):
-    """Full-size quantize in the launch shape the benchmark times (config 5: 8192-token chunks);
-    sampled rows checked against the oracle on the exact inputs."""
+def test_full_size_quantize(name):
+    """Full-size quantize in the launch shape the benchmark times (1M case: 8192-token chunks),
+    every row compared with the oracle on the exact inputs.  The fraction of coordinates within
+    1e-6 of a threshold (the only place a code may differ) is gated at 1e-5, and the kernel's own
+    count of such coordinates must agree with the oracle's."""
     w = W.CONFIGS[name]
     params = params_for(w)
     K, V = full_inputs(w)
     cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m)
+    ex0 = tq.quantize_exempt_codes()
     quantize_chunked(params, K, V, cache, 0, w.chunk)
     torch.cuda.synchronize()
-    rows = sample_rows(w, 256, np.random.default_rng(11))
-    idx = torch.tensor(rows, device="cuda")
-    Ks = K[idx[:, 0], idx[:, 1], idx[:, 2]].double().cpu().numpy()
-    Vs = V[idx[:, 0], idx[:, 1], idx[:, 2]].double().cpu().numpy()
-    compare_quantized(w, cache, Ks, Vs, 0, rows=rows)
+    gpu_exempt = tq.quantize_exempt_codes() - ex0
+    st = compare_full_cache(w, cache, K, V)
+    frac = st["exempt_codes"] / st["coords"]
+    print(f"{name}: {st['vectors']} vectors, exempt codes {st['exempt_codes']} of {st['coords']} "
+          f"(fraction {frac:.3e}; kernel count {gpu_exempt}), {st['code_mismatch_in_band']} differ; "
+          f"sign values within 1e-5 of 0: {st.get('near_zero_signs', 0)} of {st.get('sign_bits', 0)}, "
+          f"{st.get('sign_mismatch_in_band', 0)} exempt signs differ")
+    assert st["vectors"] == w.B * w.Hkv * w.T
+    assert frac <= EXEMPT_FRACTION_MAX
+    assert abs(gpu_exempt - st["exempt_codes"]) <= 2
 
 
 @pytest.mark.parametrize("name", FULL)

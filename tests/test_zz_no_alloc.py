@@ -51,6 +51,9 @@ def test_static_decode_matches_workspace_decode_two_calls():
         assert np.isfinite(got).all()
         max_abs, rel = attention_errors(got, exp)
         assert max_abs <= ATTN_MAX_ABS and rel <= ATTN_REL_L2, (max_abs, rel)
+        # Both entry points run the same kernels with the same plan, so the results are the same
+        # bits: a wrong scratch offset or a stale scratch read would show up here.
+        assert torch.equal(out_static, ref)
 
 
 def test_static_decode_rejects_sizes_above_the_limit():
