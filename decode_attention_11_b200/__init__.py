@@ -38,7 +38,7 @@ EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codeboo
             "tq_quantize_code_fixups", "tq_quantize_exempt_codes", "tq_quantize_exempt_signs",
             "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
             "tq_decode_static_workspace_limit", "tq_sketch_rotation", "tq_build_hadamard_rotation",
-            "tq_decode_step")
+            "tq_decode_step", "tq_decode_device_errors")
 
 
 class TqError(RuntimeError):
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
     L.tq_quantize_exempt_codes.argtypes = []
     L.tq_quantize_exempt_signs.restype = ctypes.c_longlong
     L.tq_quantize_exempt_signs.argtypes = []
+    L.tq_decode_device_errors.restype = ctypes.c_int
+    L.tq_decode_device_errors.argtypes = []
     L.tq_decode_workspace_size.restype = ctypes.c_size_t
     L.tq_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache),
                                            ctypes.c_int]
@@ -316,6 +318,11 @@ def quantize_exempt_signs() -> int:
     return int(lib().tq_quantize_exempt_signs())
 
 
+def decode_device_errors() -> int:
+    """Device-side error bits recorded by tq_decode_attn (0 = none); synchronizes."""
+    return int(lib().tq_decode_device_errors())
+
+
 def decode_workspace_size(B: int, Hq: int, cache: Cache, seq_len: int) -> int:
     c = cache.as_c()
     return int(lib().tq_decode_workspace_size(int(B), int(Hq), ctypes.byref(c), int(seq_len)))
@@ -399,7 +406,7 @@ __all__ = [
     "build_codebook", "Params", "Cache", "quantize", "quantize_device_errors",
     "decode_attn_static", "decode_static_workspace_limit",
     "quantize_vector_fixups", "quantize_code_fixups", "quantize_exempt_codes", "quantize_exempt_signs",
-    "decode_workspace_size", "decode_attn",
+    "decode_workspace_size", "decode_attn", "decode_device_errors",
     "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
     "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16",
 ]

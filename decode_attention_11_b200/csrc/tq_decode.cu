@@ -9,15 +9,16 @@
 // Kernels (all on the caller's stream; split and merge are programmatic dependent launches):
 //   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace: clusters of
 //           eight CTAs, each CTA holding 16 rows of Pi and S for a batch of up to 16 heads.
-//   split   grid (splits, Hkv * head_groups, B).  A 4-warp CTA streams its token range through a
-//           4-stage cp.async pipeline (64 tokens per stage).  Each warp takes 16 tokens per stage:
-//           codes are turned into fp16 pairs by a lane-replicated shared-memory table (one load per
-//           two coordinates, no bank conflicts), and m16n8k16 tensor-core MMAs compute q'.khat,
-//           the QJL sign dot (q' and S q' split into fp16 hi + lo rows; signs -> +-0.5 by one
-//           half2 FMA) and P.vhat (P split into hi + lo rows).  Online softmax runs in log2 units.
-//           The CTA merges its warps and writes one (max, sum, o'[128]) partial per head.
+//   split   one persistent CTA per SM over an even share of all (unit, token) pairs.  A producer
+//           warp streams 128-token stages of the packed cache into a ring of shared-memory slots
+//           with bulk copies (mbarrier completion); 11 (7 for groups of 5-8 heads) consumer warps take 16 tokens each per
+//           stage: codes become fp16 pairs through a lane-replicated shared-memory table (one
+//           permute + one load per two coordinates), and m16n8k16 tensor-core MMAs compute q'.khat,
+//           the QJL sign dot (sign bits placed in fp16 mantissas by a shift and one logic op, B rows
+//           pre-scaled to match) and P.vhat (P split into fp16 hi + lo).  Online softmax runs in
+//           log2 units; each segment ends with one (max, sum, o'[128]) partial per head.
 //   merge   one CTA per (batch, query head), a programmatic dependent of split: log-sum-exp
-//           merge of the head's split partials, then o = Pi^T o'.
+//           merge of the head's partials, then o = Pi^T o'.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -31,40 +32,10 @@ namespace tq {
 namespace {
 
 constexpr int D = kHeadDim;
-// CTA shape per code widths.  With 4-bit keys and values the pair tables take 64 KB, so two CTAs
-// share an SM: six warps and three stages each (12 warps per SM).  Smaller tables leave room for
-// three four-warp CTAs with four stages (register-bound).
-template <int KB, int VB>
-struct Cfg {
-  static constexpr bool kPacked = KB == 4 && VB == 4;
-  static constexpr int W = kPacked ? 6 : 4;
-  static constexpr int THREADS = 32 * W;
-  static constexpr int STAGE_TOK = 16 * W;  // 16 tokens per warp per stage
-  static constexpr int NSTAGE = kPacked ? 3 : 4;
-  static constexpr int MIN_BLOCKS = kPacked ? 2 : 3;
-};
-inline int stage_tokens(int kb, int vb) { return (kb == 4 && vb == 4) ? 96 : 64; }
 constexpr int HG = 8;                  // query heads per MMA row block (hi rows 0-7, lo rows 8-15)
 constexpr int PART = 4 + D;            // (max, sum, pad, pad, o'[128]) per partial: o' 16-byte aligned
-constexpr int SPLITS_MAX = 512;        // CTAs per (batch, kv-head, head group)
 constexpr unsigned FULL = 0xffffffffu;
 
-struct DArgs {
-  int B, Hq, Hkv, g, hgroups, T_cap, seq_len, splits, tps;
-  float sK;   // scale*log2e/sqrt(d)                     (times n_i)
-  float sQ;   // scale*log2e*2*sqrt(pi/2)/m              (times ||r_i||; 2 undoes the +-0.5 signs)
-  const uint8_t* k_codes;
-  const uint8_t* k_signs;
-  const float* k_norm;
-  const float* k_rnorm;
-  const uint8_t* v_codes;
-  const float* v_norm;
-  const float* kc;
-  const float* vc;
-  const float* qrot;
-  const float* sq;
-  float* part;
-};
 
 // ------------------------------------------------------------------------------------------ PTX
 
@@ -87,21 +58,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// 16-byte async copy; src_bytes < 16 zero-fills the rest (src_bytes = 0: no global read).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes));
-}
+// 4-byte async copy (src_bytes = 0: no global read, zero fill).
 __device__ __forceinline__ void cp_async4(void* dst, const void* src, int src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
                "r"(src_bytes));
 }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
-}
-
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __halves2half2(__float2half_rn(lo), __float2half_rn(hi));
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -111,26 +72,6 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 __device__ __forceinline__ void split_half(float x, float& hi, float& lo) {
   hi = __half2float(__float2half_rn(x));
   lo = x - hi;
-}
-
-// Sign bits -> +-0.5 fp16 pair: bits q and q+16 of w (1 <= q <= 9) placed in the mantissa of 1.0
-// (fp16 0x3C00: mantissa bits 0-9 are zero, bit 10 is already an exponent bit), then one exact
-// half2 FMA maps 1 + b*2^(q-10) to b - 0.5.
-template <int Q>
-__device__ __forceinline__ uint32_t sign_half2(uint32_t w) {
-  static_assert(Q >= 1 && Q <= 9, "mantissa position");
-  const uint32_t x = (w & (0x00010001u << Q)) | 0x3C003C00u;
-  const __half2 hx = *reinterpret_cast<const __half2*>(&x);
-  const float m = (float)(1 << (10 - Q));
-  const __half2 r = __hfma2(hx, __float2half2_rn(m), __float2half2_rn(-(m + 0.5f)));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-// Pair p of a thread's 32-bit sign word (bits p and p+16).
-template <int P>
-__device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
-  if constexpr (P == 0) return sign_half2<1>(w << 1);
-  else if constexpr (P <= 9) return sign_half2<P>(w);
-  else return sign_half2<P - 9>(w >> 9);
 }
 
 // Pair p (0..15) of a thread's key-code chunk: 2*KB bits starting at bit 2*KB*p.
@@ -186,12 +127,6 @@ struct VPairs {
     }
   }
 };
-
-// Value code nu (0..15) of a thread's 16-code value chunk held in a 64-bit integer.
-template <int VB, int NU>
-__device__ __forceinline__ uint32_t v_code(uint64_t c) {
-  return (uint32_t)(c >> (VB * NU)) & ((1u << VB) - 1u);
-}
 
 // ------------------------------------------------------------------------------------------ prep
 
@@ -278,66 +213,163 @@ __global__ void __cluster_dims__(PREP_CLUSTER, 1, 1) __launch_bounds__(PREP_THRE
 }
 
 // ------------------------------------------------------------------------------------------ split
+//
+// Persistent split-K kernel.  The B * Hkv * head_groups (batch, kv-head, head group) units, each
+// seq_len tokens long, are laid end to end and cut into one contiguous range per CTA (one CTA per
+// SM), so every CTA streams the same number of tokens.  A range that crosses a unit boundary is
+// processed as two segments; each segment ends with one (max, sum, o') partial per query head.
+//
+// Per CTA: warp NW (the producer) moves stages of ST = 16 * NW tokens into a ring of shared-memory
+// slots: the key codes, sign bits and value codes of a stage are three contiguous blocks of the
+// cache, fetched with one bulk copy each (cp.async.bulk, completion counted in bytes on the slot's
+// "full" mbarrier), and the three per-token norms go through 4-byte cp.async whose completion the
+// same mbarrier tracks.  Warps 0..NW-1 consume 16 tokens of every stage each and release the slot
+// on its "empty" mbarrier.
 
-template <int KB, int VB, bool QJL>
-struct Layout {
-  static constexpr int W = Cfg<KB, VB>::W;
-  static constexpr int STAGE_TOK = Cfg<KB, VB>::STAGE_TOK;
-  static constexpr int NSTAGE = Cfg<KB, VB>::NSTAGE;
-  static constexpr int K_ROW = 16 * KB;
-  static constexpr int V_ROW = 16 * VB;
-  static constexpr bool kPackedLut = KB == 4 && VB == 4;
-  static constexpr int OFF_KC = 0;
-  static constexpr int OFF_SG = OFF_KC + STAGE_TOK * K_ROW;
-  static constexpr int OFF_VC = OFF_SG + (QJL ? STAGE_TOK * 16 : 0);
-  static constexpr int OFF_NK = OFF_VC + STAGE_TOK * V_ROW;
-  static constexpr int OFF_RN = OFF_NK + STAGE_TOK * 4;
-  static constexpr int OFF_NV = OFF_RN + (QJL ? STAGE_TOK * 4 : 0);
-  static constexpr int STAGE_BYTES = OFF_NV + STAGE_TOK * 4;
-  static constexpr int LUT_BYTES = kPackedLut ? 256 * 256 : ((1 << (2 * KB)) + (1 << (2 * VB))) * 128;
-  // After the main loop the pipeline buffers hold the CTA's own warp merge.
-  static constexpr int WARP_MERGE_BYTES = 4 * (W * HG * 2 + W * HG * D);
-  static constexpr int PIPE_BYTES = NSTAGE * STAGE_BYTES;
-  static constexpr int SMEM = LUT_BYTES + (PIPE_BYTES > WARP_MERGE_BYTES ? PIPE_BYTES : WARP_MERGE_BYTES);
-  static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
+// CTA shape: NW consumer warps + 1 producer.  The register file is split between the SM's four
+// schedulers, so 12 warps (three per scheduler) leave 168 registers a thread: enough for one n-block
+// of four heads (NB = 1).  Two n-blocks (five to eight heads per kv-head) need more registers and
+// run with 8 warps (two per scheduler, up to 255 registers).
+template <int NB>
+struct Shape {
+  static constexpr int NW = NB == 1 ? 11 : 7;
+  static constexpr int THREADS = 32 * (NW + 1);
+  static constexpr int ST = 16 * NW;        // tokens per stage
+};
+constexpr int NS_MAX = 8;                   // ring slots
+constexpr int MIN_TOK_PER_CTA = 256;        // fewer CTAs than SMs below this much work each
+constexpr int CTRL_BYTES = 256;             // mbarriers, slot offsets, flags (end of dynamic smem)
+constexpr long long WAIT_LIMIT = 4000000000LL;  // ~2 s of SM clock per wait
+
+// Flat partition of N = units * seq_len tokens over C CTAs: CTA c takes [start(c), start(c + 1)).
+__host__ __device__ inline int64_t part_start(int64_t N, int C, int c) { return (int64_t)c * N / C; }
+__host__ __device__ inline int part_cta_of(int64_t N, int C, int64_t f) { return (int)(((f + 1) * C - 1) / N); }
+
+struct DArgs {
+  int B, Hq, Hkv, g, hgroups, T_cap, seq_len;
+  int units, ctas, pmax, dyn_smem;
+  int64_t ntot;  // units * seq_len
+  float sK;      // scale*log2e/sqrt(d)                (times n_i)
+  float sQ;      // scale*log2e*2*sqrt(pi/2)/m         (times ||r_i||)
+  const uint8_t* k_codes;
+  const uint8_t* k_signs;
+  const float* k_norm;
+  const float* k_rnorm;
+  const uint8_t* v_codes;
+  const float* v_norm;
+  const float* kc;
+  const float* vc;
+  const float* qrot;
+  const float* sq;
+  float* part;
 };
 
-template <int KB, int VB, bool QJL>
-__device__ __forceinline__ void load_stage(const DArgs& a, unsigned char* stage, int64_t row0,
-                                           int count) {
-  using Lay = Layout<KB, VB, QJL>;
-  constexpr int THREADS = Cfg<KB, VB>::THREADS, STAGE_TOK = Cfg<KB, VB>::STAGE_TOK;
-  const int tid = threadIdx.x;
-  // key codes: KB 16-byte chunks per token
-  {
-    const uint8_t* src = a.k_codes + row0 * Lay::K_ROW;
-    for (int i = tid; i < STAGE_TOK * KB; i += THREADS) {
-      const bool ok = i < count * KB;
-      cp_async16(stage + Lay::OFF_KC + 16 * i, ok ? src + 16 * i : a.k_codes, ok ? 16 : 0);
+__device__ unsigned int g_decode_error;  // bit 0: a wait timed out; bit 1: shared memory too small
+
+template <int KB, int VB, bool QJL, int NB>
+struct Layout {
+  static constexpr int NW = Shape<NB>::NW, ST = Shape<NB>::ST, HGN = 4 * NB;
+  static constexpr int K_ROW = 16 * KB;
+  static constexpr int V_ROW = 16 * VB;
+  static constexpr int OFF_KC = 0;
+  static constexpr int OFF_SG = OFF_KC + ST * K_ROW;
+  static constexpr int OFF_VC = OFF_SG + (QJL ? ST * 16 : 0);
+  static constexpr int OFF_NK = OFF_VC + ST * V_ROW;
+  static constexpr int OFF_RN = OFF_NK + ST * 4;
+  static constexpr int OFF_NV = OFF_RN + (QJL ? ST * 4 : 0);
+  static constexpr int STAGE_BYTES = (OFF_NV + ST * 4 + 127) / 128 * 128;
+  static constexpr int TX_PER_TOKEN = K_ROW + (QJL ? 16 : 0) + V_ROW;  // bulk-copied bytes
+  static constexpr bool kPacked = KB == 4 && VB == 4;
+  static constexpr int K_TBL = kPacked ? 0 : (1 << (2 * KB)) * 128;
+  static constexpr int V_TBL = kPacked ? 0 : (1 << (2 * VB)) * 128;
+  static constexpr int TBL_BYTES = kPacked ? 65536 : K_TBL + V_TBL;
+  // per-warp (max, sum) and o' of the 4 NB heads, for the merge of the warps at a segment's end
+  static constexpr int MERGE_BYTES = 4 * (NW * HGN * 2 + NW * HGN * D);
+  static_assert(STAGE_BYTES % 16 == 0 && K_ROW % 16 == 0 && V_ROW % 16 == 0, "bulk-copy granularity");
+};
+
+// Control block at the end of the dynamic shared memory.
+struct Ctrl {
+  uint64_t full[NS_MAX];
+  uint64_t empty[NS_MAX];
+  uint32_t stage_off[NS_MAX];  // byte offsets of the ring slots from the start of dynamic smem
+  uint32_t tbl_addr;           // shared-window address of the pair tables
+  uint32_t merge_off;
+  int ns;
+  unsigned int err;
+};
+static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
+
+__device__ __forceinline__ void mbar_init_(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx_(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// The thread's earlier cp.async copies arrive on the mbarrier when they land (counted in its init).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+// One bulk copy global -> shared (sizes and addresses multiples of 16), completion in bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(addr), "r"(parity), "r"(100000u)
+      : "memory");
+  return done != 0;
+}
+// Bounded wait of a whole warp on an mbarrier phase (every lane returns the same answer).  Gives up
+// at once when another warp has recorded an error, or after WAIT_LIMIT cycles (then records one).
+__device__ __forceinline__ bool wait_w(Ctrl& c, uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  const long long t0 = clock64();
+  while (true) {
+    if (__any_sync(FULL, mbar_try(addr, parity))) return true;
+    const bool stop = *reinterpret_cast<volatile unsigned int*>(&c.err) != 0 || clock64() - t0 > WAIT_LIMIT;
+    if (__any_sync(FULL, stop)) {
+      if ((threadIdx.x & 31) == 0) atomicOr(&c.err, 1u);
+      return false;
     }
-  }
-  if constexpr (QJL) {
-    const uint8_t* src = a.k_signs + row0 * 16;
-    for (int i = tid; i < STAGE_TOK; i += THREADS) {
-      const bool ok = i < count;
-      cp_async16(stage + Lay::OFF_SG + 16 * i, ok ? src + 16 * i : a.k_signs, ok ? 16 : 0);
-    }
-  }
-  {
-    const uint8_t* src = a.v_codes + row0 * Lay::V_ROW;
-    for (int i = tid; i < STAGE_TOK * VB; i += THREADS) {
-      const bool ok = i < count * VB;
-      cp_async16(stage + Lay::OFF_VC + 16 * i, ok ? src + 16 * i : a.v_codes, ok ? 16 : 0);
-    }
-  }
-  for (int i = tid; i < STAGE_TOK; i += THREADS) {
-    const bool ok = i < count;
-    cp_async4(stage + Lay::OFF_NK + 4 * i, ok ? a.k_norm + row0 + i : a.k_norm, ok ? 4 : 0);
-    if constexpr (QJL)
-      cp_async4(stage + Lay::OFF_RN + 4 * i, ok ? a.k_rnorm + row0 + i : a.k_rnorm, ok ? 4 : 0);
-    cp_async4(stage + Lay::OFF_NV + 4 * i, ok ? a.v_norm + row0 + i : a.v_norm, ok ? 4 : 0);
   }
 }
+// Named barrier of the NW consumer warps (the producer warp never takes part).
+template <int NW>
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(NW * 32) : "memory");
+}
+
+// QJL sign operand: pair P (bits P and P + 16 of the lane's sign word, sketch rows 2t + e of
+// k-half P % 2 of k-step P / 2) as a half2 of 1 + b 2^(q - 10), b the sign bit: the word, shifted
+// so that the pair lands on mantissa bits q and q + 16 (q = 6 + P % 4), masked and ORed into 1.0.
+// The B operand rows of such a pair are pre-scaled by 2^(10 - q), so the MMA yields
+// C + sum_l b_l sq_l with the per-head constant C = sum_l 2^(10 - q_l) sq_l.
+template <int P>
+__device__ __forceinline__ uint32_t sgn(uint32_t w) {
+  constexpr int q = 6 + (P & 3);
+  uint32_t x;
+  if constexpr (P < 4) x = w << 6;
+  else if constexpr (P < 8) x = w << 2;
+  else if constexpr (P < 12) x = w >> 2;
+  else x = w >> 6;
+  return (x & (0x00010001u << q)) | 0x3C003C00u;
+}
+// 2^(10 - q) of pair P: the B-row scale that undoes the mantissa position.
+__host__ __device__ constexpr float sgn_scale(int P) { return (float)(16 >> (P & 3)); }
 
 // Value chunk of one token for this lane group (16 codes of VB bits) as a 64-bit integer.
 template <int VB>
@@ -355,13 +387,470 @@ __device__ __forceinline__ uint64_t load_v_chunk(const unsigned char* row, int g
   }
 }
 
+// Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (m8n8 fragment layout).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Pair tables: a pair of codes -> half2 of centroids, replicated per lane (bank = lane).
+// 4-bit keys and values: 256 entries of 256 bytes (K replicas at +0, V at +128) starting at a
+// 64 KB-aligned address, so one byte permute of the code word and of rk / rv (table address |
+// lane offset) is the entry's address.  Other widths: separate K and V tables of 128-byte entries,
+// address = (index << 7) + rk / rv.
+template <int KB, int VB>
+struct PairLut {
+  static constexpr bool kPacked = KB == 4 && VB == 4;
+  uint32_t rk, rv;
+  __device__ __forceinline__ uint32_t k(uint32_t e) const { return lds32((e << 7) + rk); }
+  __device__ __forceinline__ uint32_t v(uint32_t e) const { return lds32((e << 7) + rv); }
+  template <int Bt>
+  __device__ __forceinline__ uint32_t k_byte(uint32_t w) const { return lds32(__byte_perm(w, rk, 0x7604u | (Bt << 4))); }
+  template <int Bt>
+  __device__ __forceinline__ uint32_t v_byte(uint32_t w) const { return lds32(__byte_perm(w, rv, 0x7604u | (Bt << 4))); }
+};
+
+// Key pair P (0..15) of a thread's code chunk, as a half2 of centroids.
+template <int KB, int VB, int P>
+__device__ __forceinline__ uint32_t k_pair(const PairLut<KB, VB>& L, const uint32_t (&c)[KB]) {
+  if constexpr (PairLut<KB, VB>::kPacked) return L.template k_byte<P & 3>(c[P >> 2]);
+  else return L.k(k_pair_index<KB, P>(c));
+}
+// Value pair NU of a token pair, as a half2 of centroids.
+template <int KB, int VB, int NU>
+__device__ __forceinline__ uint32_t v_pair(const PairLut<KB, VB>& L, const VPairs<VB>& p) {
+  if constexpr (PairLut<KB, VB>::kPacked) return L.template v_byte<((NU & 7) >> 1)>(p.w[2 * (NU >> 3) + (NU & 1)]);
+  else return L.v(p.template index<NU>());
+}
+
+// Shared-memory plan, computed by one thread: the pair tables (at a 64 KB boundary for the packed
+// tables), the warp-merge area and as many ring slots as fit around them.  ns = 0 when the slots
+// do not fit (never with the 227 KB of an sm_100 CTA).
+template <int KB, int VB, bool QJL, int NB>
+__device__ void plan_smem(unsigned char* smem, int dyn, Ctrl& c) {
+  using Lay = Layout<KB, VB, QJL, NB>;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t end = base + (uint32_t)dyn - CTRL_BYTES;
+  const uint32_t tbl = Lay::kPacked ? ((base + 0xFFFFu) & ~0xFFFFu) : base;
+  c.tbl_addr = tbl;
+  // free regions: [base, tbl) and [tbl + TBL_BYTES, end)
+  uint32_t r0 = base, r0e = tbl, r1 = tbl + Lay::TBL_BYTES, r1e = end;
+  if (r1 > end) {
+    c.ns = 0;
+    return;
+  }
+  auto take = [&](uint32_t bytes, uint32_t& off) -> bool {
+    if (r0e - r0 >= bytes) {
+      off = r0 - base;
+      r0 += bytes;
+      return true;
+    }
+    if (r1e - r1 >= bytes) {
+      off = r1 - base;
+      r1 += bytes;
+      return true;
+    }
+    return false;
+  };
+  uint32_t off = 0;
+  if (!take(Lay::MERGE_BYTES, off)) {
+    c.ns = 0;
+    return;
+  }
+  c.merge_off = off;
+  int ns = 0;
+  while (ns < NS_MAX && take(Lay::STAGE_BYTES, off)) c.stage_off[ns++] = off;
+  c.ns = ns >= 2 ? ns : 0;
+}
+
+template <int KB, int VB, bool QJL, int NB>
+__global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __grid_constant__ DArgs a) {
+  using Lay = Layout<KB, VB, QJL, NB>;
+  using Lut = PairLut<KB, VB>;
+  constexpr int NW = Shape<NB>::NW, ST = Shape<NB>::ST, HGN = 4 * NB;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Ctrl& ctl = *reinterpret_cast<Ctrl*>(smem + a.dyn_smem - CTRL_BYTES);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = blockIdx.x;
+  const int64_t f_begin = part_start(a.ntot, a.ctas, c), f_end = part_start(a.ntot, a.ctas, c + 1);
+  const int64_t L = a.seq_len;
+
+  if (tid == 0) {
+    plan_smem<KB, VB, QJL, NB>(smem, a.dyn_smem, ctl);
+    ctl.err = 0;
+    for (int i = 0; i < ctl.ns; ++i) {
+      mbar_init_(&ctl.full[i], 1 + 32);  // producer's expect_tx + the noinc arrivals of its 32 lanes
+      mbar_init_(&ctl.empty[i], NW);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+  const int ns = ctl.ns;
+  if (ns == 0) {
+    if (tid == 0) atomicOr(&g_decode_error, 2u);
+    return;  // uniform: every thread read the same ns
+  }
+
+  if (warp == NW) {
+    // ================================================================ producer
+    int it = 0, issued = 0;
+    for (int64_t f = f_begin; f < f_end;) {
+      const int64_t u = f / L;
+      const int t0 = (int)(f - u * L);
+      const int t1 = (int)(L < t0 + (f_end - f) ? L : t0 + (f_end - f));
+      f += t1 - t0;
+      const int bk = (int)(u / a.hgroups);  // b * Hkv + kv-head
+      const int64_t rowb = (int64_t)bk * a.T_cap;
+      for (int s0 = t0; s0 < t1; s0 += ST, ++it) {
+        const int slot = it % ns;
+        if (it >= ns && !wait_w(ctl, &ctl.empty[slot], ((it / ns) - 1) & 1)) continue;
+        if (*reinterpret_cast<volatile unsigned int*>(&ctl.err)) continue;
+        const int ntok = min(ST, t1 - s0);
+        const int64_t row0 = rowb + s0;
+        unsigned char* st = smem + ctl.stage_off[slot];
+        if (lane == 0) {
+          mbar_expect_tx_(&ctl.full[slot], (uint32_t)(ntok * Lay::TX_PER_TOKEN));
+          bulk_g2s(st + Lay::OFF_KC, a.k_codes + row0 * Lay::K_ROW, ntok * Lay::K_ROW, &ctl.full[slot]);
+          if constexpr (QJL) bulk_g2s(st + Lay::OFF_SG, a.k_signs + row0 * 16, ntok * 16, &ctl.full[slot]);
+          bulk_g2s(st + Lay::OFF_VC, a.v_codes + row0 * Lay::V_ROW, ntok * Lay::V_ROW, &ctl.full[slot]);
+        }
+        for (int i = lane; i < ntok; i += 32) {
+          cp_async4(st + Lay::OFF_NK + 4 * i, a.k_norm + row0 + i, 4);
+          if constexpr (QJL) cp_async4(st + Lay::OFF_RN + 4 * i, a.k_rnorm + row0 + i, 4);
+          cp_async4(st + Lay::OFF_NV + 4 * i, a.v_norm + row0 + i, 4);
+        }
+        cp_async_arrive_noinc(&ctl.full[slot]);
+        issued = it + 1;
+      }
+    }
+    // every copy issued has landed before the CTA may exit (bounded)
+    for (int j = max(0, issued - ns); j < issued; ++j) {
+      const uint32_t addr = smem_u32(&ctl.full[j % ns]);
+      const long long t0 = clock64();
+      while (!__all_sync(FULL, mbar_try(addr, (j / ns) & 1)) && clock64() - t0 < WAIT_LIMIT) {
+      }
+    }
+    if (lane == 0 && *reinterpret_cast<volatile unsigned int*>(&ctl.err)) atomicOr(&g_decode_error, 1u);
+    return;
+  }
+
+  // ================================================================ consumers (warps 0 .. NW-1)
+  // Pair tables: entry e = lo | hi << b -> half2(c[lo], c[hi]), four lane replicas per 16-byte store.
+  Lut lut;
+  {
+    const uint32_t tbl = ctl.tbl_addr;
+    unsigned char* tp = smem + (tbl - smem_u32(smem));
+    if constexpr (Lut::kPacked) {
+      for (int i = tid; i < 256 * 2 * 8; i += NW * 32) {  // (entry, half, group of four lanes)
+        const int e = i >> 4, half = (i >> 3) & 1, q4 = i & 7;
+        const float* cb = half ? a.vc : a.kc;
+        const uint32_t v = pack_half2(__ldg(cb + (e & 15)), __ldg(cb + (e >> 4)));
+        *reinterpret_cast<uint4*>(tp + e * 256 + half * 128 + 16 * q4) = make_uint4(v, v, v, v);
+      }
+      lut.rk = tbl | (4u * lane);
+      lut.rv = tbl | 128u | (4u * lane);
+    } else {
+      for (int i = tid; i < (Lay::K_TBL + Lay::V_TBL) / 16; i += NW * 32) {
+        const bool isv = i >= Lay::K_TBL / 16;
+        const int j = isv ? i - Lay::K_TBL / 16 : i;
+        const int e = j >> 3;
+        const int bits = isv ? VB : KB;
+        const float* cb = isv ? a.vc : a.kc;
+        const uint32_t v = pack_half2(__ldg(cb + (e & ((1 << bits) - 1))), __ldg(cb + (e >> bits)));
+        *reinterpret_cast<uint4*>(tp + 16 * i) = make_uint4(v, v, v, v);
+      }
+      lut.rk = tbl + 4u * lane;
+      lut.rv = tbl + Lay::K_TBL + 4u * lane;
+    }
+  }
+  consumers_sync<NW>();
+  // The rotated queries come from the prep kernel; everything above reads only the cache.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // the merge kernel may launch now; its CTAs wait for this grid to finish before reading
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  const int gq = lane >> 2, t = lane & 3;
+  float* mrg = reinterpret_cast<float*>(smem + ctl.merge_off);
+  float* mw = mrg;                 // [NW][HGN]
+  float* lw = mw + NW * HGN;       // [NW][HGN]
+  float* ow = lw + NW * HGN;       // [NW][HGN][D]
+  int it = 0;
+  for (int64_t f = f_begin; f < f_end;) {
+    const int64_t u = f / L;
+    const int t0 = (int)(f - u * L);
+    const int t1 = (int)(L < t0 + (f_end - f) ? L : t0 + (f_end - f));
+    f += t1 - t0;
+    const int bk = (int)(u / a.hgroups), hg = (int)(u % a.hgroups);
+    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    const int h0 = kvh * a.g + hg * HG;
+    const int nh = min(HG, a.g - hg * HG);
+
+    // ---- B operands of this unit's heads.  Column gq of n-block nb = head 4 nb + gq / 2, part
+    // gq % 2 (0: fp16 hi, 1: fp16 lo); k-step kk holds k = 16kk + 2t, +1 (reg 0), +8, +9 (reg 1).
+    // Each head is scaled by a power of two 2^-e so that q' and 16 S q' stay far inside fp16 range.
+    uint32_t bq[NB][8][2], bsq[NB][8][2];
+    float fK[NB], fQ[NB], Kh[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int hh = 4 * nb + (gq >> 1);
+      const bool live = hh < nh;
+      const bool lo = gq & 1;
+      const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
+      const float* sp = a.sq + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
+      float qv[8][2][2], sv[8][2][2];
+      float mx = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int k = 16 * kk + 8 * r + 2 * t + e;
+            qv[kk][r][e] = live ? qp[k] : 0.0f;
+            sv[kk][r][e] = (live && QJL) ? sp[k] : 0.0f;
+            mx = fmaxf(mx, fmaxf(fabsf(qv[kk][r][e]), 16.0f * fabsf(sv[kk][r][e])));
+          }
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));  // both parts of the head
+      // 2^-e with mx 2^-e < 2^14 (e >= 0); inf / nan stay inf / nan
+      const int ex = (mx < 16384.0f || !(mx < INFINITY)) ? 0 : ((__float_as_int(mx) >> 23) & 255) - 127 - 13;
+      const float dn = __int_as_float((127 - ex) << 23);  // 2^-ex
+      float csum = 0.0f, ssum = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          float hx, lx, hy, ly;
+          split_half(qv[kk][r][0] * dn, hx, lx);
+          split_half(qv[kk][r][1] * dn, hy, ly);
+          bq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
+          if constexpr (QJL) {
+            const float scl = sgn_scale(2 * kk + r);
+            split_half(sv[kk][r][0] * dn * scl, hx, lx);
+            split_half(sv[kk][r][1] * dn * scl, hy, ly);
+            bsq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
+            const float p0 = lo ? lx : hx, p1 = lo ? ly : hy;  // this lane's column values
+            csum += p0 + p1;
+            ssum += (p0 + p1) * (1.0f / scl);
+          } else {
+            bsq[nb][kk][r] = 0u;
+          }
+        }
+      // column sums over the four lanes of the column, then per head (hi + lo columns) for the
+      // score layout, where lane (gq, t) holds head 4 nb + t
+      csum += __shfl_xor_sync(FULL, csum, 1);
+      csum += __shfl_xor_sync(FULL, csum, 2);
+      ssum += __shfl_xor_sync(FULL, ssum, 1);
+      ssum += __shfl_xor_sync(FULL, ssum, 2);
+      const float ch = __shfl_sync(FULL, csum, 8 * t) + __shfl_sync(FULL, csum, 8 * t + 4);
+      const float sh = __shfl_sync(FULL, ssum, 8 * t) + __shfl_sync(FULL, ssum, 8 * t + 4);
+      const int ext = __shfl_sync(FULL, ex, 8 * t);
+      const float up = __int_as_float((127 + ext) << 23);  // 2^e of head 4 nb + t
+      fK[nb] = a.sK * up;
+      fQ[nb] = a.sQ * up;
+      Kh[nb] = -ch - 0.5f * sh;  // sum_l sq_l (2 b_l - 1) = 2 (D_hi + D_lo + Kh)
+    }
+
+    // Output accumulators: n-block nb, dim block db: (dim 16db + gq, head 4nb + t) hi/lo in [0]/[1],
+    // (dim 16db + 8 + gq) in [2]/[3].
+    float oacc[NB][8][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) oacc[nb][i][0] = oacc[nb][i][1] = oacc[nb][i][2] = oacc[nb][i][3] = 0.0f;
+    float m_run[NB], l_run[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      m_run[nb] = -1e30f;  // finite: ex2(s - m) and ex2(m_old - m_new) never see inf - inf
+      l_run[nb] = 0.0f;
+    }
+
+    for (int s0 = t0; s0 < t1; s0 += ST, ++it) {
+      const int slot = it % ns;
+      const bool ok = wait_w(ctl, &ctl.full[slot], (it / ns) & 1);
+      const int nvalid = min(16, t1 - s0 - 16 * warp);
+      if (ok && nvalid > 0) {
+        const unsigned char* stage = smem + ctl.stage_off[slot];
+        const int r0 = 16 * warp + gq, r1 = r0 + 8;  // this lane's token rows in the stage
+
+        // ---- scores for tokens r0, r1 and heads 4nb + t ----
+        float kacc[NB][4], qacc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = 0.0f;
+        {
+          uint32_t c0[KB], c1[KB];
+          const uint32_t* k0 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r0 * Lay::K_ROW + 4 * KB * t);
+          const uint32_t* k1 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r1 * Lay::K_ROW + 4 * KB * t);
+#pragma unroll
+          for (int i = 0; i < KB; ++i) {
+            c0[i] = k0[i];
+            c1[i] = k1[i];
+          }
+#define TQ_KSTEP(KK)                                                                         \
+          {                                                                                  \
+            const uint32_t A[4] = {k_pair<KB, VB, 2 * (KK)>(lut, c0), k_pair<KB, VB, 2 * (KK)>(lut, c1), \
+                                   k_pair<KB, VB, 2 * (KK) + 1>(lut, c0),                    \
+                                   k_pair<KB, VB, 2 * (KK) + 1>(lut, c1)};                   \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                \
+                mma16816(kacc[nb], A, bq[nb][KK][0], bq[nb][KK][1]);                          \
+          }
+          TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
+#undef TQ_KSTEP
+        }
+        if constexpr (QJL) {
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r0 * 16 + 4 * t);
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r1 * 16 + 4 * t);
+#define TQ_SSTEP(KK)                                                                         \
+          {                                                                                  \
+            const uint32_t A[4] = {sgn<2 * (KK)>(w0), sgn<2 * (KK)>(w1), sgn<2 * (KK) + 1>(w0), \
+                                   sgn<2 * (KK) + 1>(w1)};                                   \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                \
+                mma16816(qacc[nb], A, bsq[nb][KK][0], bsq[nb][KK][1]);                         \
+          }
+          TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
+#undef TQ_SSTEP
+        }
+
+        // ---- online softmax (log2 units) per head 4nb + t over this warp's 16 tokens ----
+        const bool v0ok = gq < nvalid, v1ok = gq + 8 < nvalid;
+        const float nk0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r0);
+        const float nk1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r1);
+        float rn0 = 0.0f, rn1 = 0.0f;
+        if constexpr (QJL) {
+          rn0 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r0);
+          rn1 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r1);
+        }
+        // rows past the segment's end hold stale or uninitialised words: their weight is 0 and
+        // their value scale too, so nothing of them reaches the sums
+        const float nv0 = v0ok ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r0) * 0.08838834764831845f : 0.0f;
+        const float nv1 = v1ok ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r1) * 0.08838834764831845f : 0.0f;
+        uint32_t bp[NB][2];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          float s0v = (kacc[nb][0] + kacc[nb][1]) * (nk0 * fK[nb]);
+          float s1v = (kacc[nb][2] + kacc[nb][3]) * (nk1 * fK[nb]);
+          if constexpr (QJL) {
+            s0v = fmaf(qacc[nb][0] + qacc[nb][1] + Kh[nb], rn0 * fQ[nb], s0v);
+            s1v = fmaf(qacc[nb][2] + qacc[nb][3] + Kh[nb], rn1 * fQ[nb], s1v);
+          }
+          s0v = v0ok ? s0v : -INFINITY;
+          s1v = v1ok ? s1v : -INFINITY;
+          float mx = fmaxf(s0v, s1v);
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+          if (mx > m_run[nb]) {  // uniform over the 8 lanes of head 4nb + t
+            const float alpha = ex2(m_run[nb] - mx);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              oacc[nb][i][0] *= alpha;
+              oacc[nb][i][1] *= alpha;
+              oacc[nb][i][2] *= alpha;
+              oacc[nb][i][3] *= alpha;
+            }
+            l_run[nb] *= alpha;
+            m_run[nb] = mx;
+          }
+          const float p0 = ex2(s0v - m_run[nb]);  // ex2(-inf) = 0 for rows past the end
+          const float p1 = ex2(s1v - m_run[nb]);
+          l_run[nb] += p0 + p1;
+          // P~ = p nV / sqrt(d) as fp16 hi + lo: row token, columns (head t, hi) and (head t, lo)
+          float hx, lx, hy, ly;
+          split_half(p0 * nv0, hx, lx);
+          split_half(p1 * nv1, hy, ly);
+          bp[nb][0] = movmatrix_trans(pack_half2(hx, lx));  // tokens 2t, 2t+1 of column gq
+          bp[nb][1] = movmatrix_trans(pack_half2(hy, ly));  // tokens 2t+8, 2t+9
+        }
+
+        // ---- O'^T += Vhat^T P~: dim blocks of 16; A holds token pairs (2t,2t+1), (2t+8,2t+9) ----
+        {
+          const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
+          const uint64_t cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
+          const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
+          const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
+          const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
+          VPairs<VB> p01, p89;
+          p01.build(cv0, cv1);
+          p89.build(cv2, cv3);
+#define TQ_VSTEP(DB)                                                                          \
+          {                                                                                   \
+            const uint32_t A[4] = {v_pair<KB, VB, 2 * (DB)>(lut, p01), v_pair<KB, VB, 2 * (DB) + 1>(lut, p01), \
+                                   v_pair<KB, VB, 2 * (DB)>(lut, p89), v_pair<KB, VB, 2 * (DB) + 1>(lut, p89)}; \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                 \
+                mma16816(oacc[nb][DB], A, bp[nb][0], bp[nb][1]);                               \
+          }
+          TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3) TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
+#undef TQ_VSTEP
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_(&ctl.empty[slot]);
+    }
+
+    // ---- merge the NW warps: one (max, sum, o') partial per head of this segment ----
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int hh = 4 * nb + t;
+      float lq = l_run[nb];
+      lq += __shfl_xor_sync(FULL, lq, 4);
+      lq += __shfl_xor_sync(FULL, lq, 8);
+      lq += __shfl_xor_sync(FULL, lq, 16);
+      if (gq == 0) {
+        mw[warp * HGN + hh] = m_run[nb];
+        lw[warp * HGN + hh] = lq;
+      }
+      float* o = ow + (warp * HGN + hh) * D;
+#pragma unroll
+      for (int db = 0; db < 8; ++db) {
+        o[16 * db + gq] = oacc[nb][db][0] + oacc[nb][db][1];
+        o[16 * db + 8 + gq] = oacc[nb][db][2] + oacc[nb][db][3];
+      }
+    }
+    consumers_sync<NW>();
+    {
+      const int j = c - part_cta_of(a.ntot, a.ctas, u * L);  // partial slot of this CTA in unit u
+      for (int idx = tid; idx < nh * D; idx += NW * 32) {
+        const int r = idx / D, dd = idx % D;
+        float M = -1e30f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w * HGN + r]);
+        float Ls = 0.0f, O = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const float fw = ex2(mw[w * HGN + r] - M);
+          Ls = fmaf(fw, lw[w * HGN + r], Ls);
+          O = fmaf(fw, ow[(w * HGN + r) * D + dd], O);
+        }
+        float* dst = a.part + (((int64_t)b * a.Hq + h0 + r) * a.pmax + j) * PART;
+        dst[4 + dd] = O;
+        if (dd == 0) {
+          dst[0] = M;
+          dst[1] = Ls;
+        }
+      }
+    }
+    consumers_sync<NW>();  // the merge area is reused by the next segment
+  }
+  if (tid == 0 && *reinterpret_cast<volatile unsigned int*>(&ctl.err)) atomicOr(&g_decode_error, 1u);
+}
+
 // ------------------------------------------------------------------------------------------ merge
 
 // One 512-thread CTA per (batch, query head), a programmatic dependent of the split kernel: it
-// waits for the split grid, merges the head's split partials by log-sum-exp and writes
-// o = Pi^T o'.  Thread (d, q), d = tid % 128 and q = tid / 128, sums the splits s = q (mod 4) of
-// dimension d; the un-rotation gives thread (i, q) the rows 32q .. 32q + 31 of Pi.  Each phase
-// issues its loads at once (one L2 round trip each).
+// waits for the split grid, merges the head's partials (one per CTA that streamed part of the
+// head's unit) by log-sum-exp and writes o = Pi^T o'.  Thread (d, q), d = tid % 128 and
+// q = tid / 128, sums the partials s = q (mod 4) of dimension d; the un-rotation gives thread
+// (i, q) the rows 32q .. 32q + 31 of Pi.  Each phase issues its loads at once (one L2 round trip).
 constexpr int MERGE_THREADS = 4 * D;
 
 __device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
@@ -386,22 +875,31 @@ __device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) 
 
 // (The partials are written by the still-running split grid: they are read with ld.global.cg,
 // through L2 only, never through the non-coherent read-only path.)
-__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
-                                                              const float* __restrict__ Pi,
-                                                              float* __restrict__ out, int S) {
+__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part, const float* __restrict__ Pi,
+                                                              float* __restrict__ out, int Hq, int g, int Hkv,
+                                                              int hgroups, int64_t seq_len, int64_t ntot, int ctas,
+                                                              int pmax) {
   extern __shared__ __align__(16) float msm[];  // [S] weights, [S] sums, [4][D] partial o', [D] o', [4][D]
   __shared__ float red[32];
   const int tid = threadIdx.x, d = tid % D, q = tid / D;
+  const int64_t bh = blockIdx.x;
+  if (seq_len == 0) {  // empty context: the output is zero (no split grid ran)
+    if (tid < D) out[bh * D + d] = 0.0f;
+    return;
+  }
   // Pi is an input, not an output of split: its rows load while the split grid finishes
   float pj[32];
 #pragma unroll
   for (int jj = 0; jj < 32; ++jj) pj[jj] = __ldg(Pi + (32 * q + jj) * D + d);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  const int64_t bh = blockIdx.x;
-  const float* p = part + bh * S * PART;
+  const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+  const int64_t u = ((int64_t)b * Hkv + h / g) * hgroups + (h % g) / HG;
+  const int first = part_cta_of(ntot, ctas, u * seq_len);
+  const int S = part_cta_of(ntot, ctas, u * seq_len + seq_len - 1) - first + 1;
+  const float* p = part + bh * pmax * PART;
   float* wts = msm;
-  float* ls = wts + S;
-  float* osum = ls + ((S + 3) & ~3);
+  float* ls = wts + pmax;
+  float* osum = ls + ((pmax + 3) & ~3);
   float* ob = osum + 4 * D;
   float* rsum = ob + D;
   // phase 1: (max, sum) of every partial
@@ -416,13 +914,12 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
   // phase 2: weights 2^(m_s - M) and L = sum_s w_s l_s
   float l = 0.0f;
   for (int s2 = tid; s2 < S; s2 += MERGE_THREADS) {
-    const float ms = wts[s2];
-    const float f = (ms == -INFINITY) ? 0.0f : ex2(ms - M);
+    const float f = ex2(wts[s2] - M);
     wts[s2] = f;
     l = fmaf(f, ls[s2], l);
   }
-  const float L = block_reduce(l, red, false);  // also makes the weights visible
-  // phase 3: thread (d, q) sums splits q, q + 4, ...
+  const float Lsum = block_reduce(l, red, false);  // also makes the weights visible
+  // phase 3: thread (d, q) sums partials q, q + 4, ...
   float acc = 0.0f;
 #pragma unroll 16
   for (int s2 = q; s2 < S; s2 += 4) acc = fmaf(wts[s2], __ldcg(p + (int64_t)s2 * PART + 4 + d), acc);
@@ -430,7 +927,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
   __syncthreads();
   if (tid < D) {
     const float o = osum[d] + osum[D + d] + osum[2 * D + d] + osum[3 * D + d];
-    ob[d] = L > 0.0f ? o / L : 0.0f;
+    ob[d] = Lsum > 0.0f ? o / Lsum : 0.0f;
   }
   __syncthreads();
   // phase 4: o_i = sum_j Pi[j][i] o'_j, thread (i = d, q) over rows 32q .. 32q + 31
@@ -442,415 +939,72 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
   if (tid < D) out[bh * D + d] = rsum[d] + rsum[D + d] + rsum[2 * D + d] + rsum[3 * D + d];
 }
 
-inline size_t merge_smem_bytes(int S) { return sizeof(float) * ((size_t)S + ((S + 3) & ~3) + 9 * D); }
-
-// Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (m8n8 fragment layout).
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-  return y;
-}
-
-// Pair-table lookups.  With 4-bit keys and values the K and V pair tables share 256-byte entry
-// slots (K replicas at +0, V replicas at +128): one byte permute turns a code byte e and the lane
-// offset into the byte address (e << 8) | 4 lane, so a pair costs one PRMT and one LDS.  Other bit
-// widths use separate tables with 128-byte entries (lane-replicated, bank = lane).
-template <int KB, int VB>
-struct PairLut {
-  static constexpr bool kPacked = KB == 4 && VB == 4;
-  static constexpr int K_BYTES = kPacked ? 0 : (1 << (2 * KB)) * 128;
-  static constexpr int V_BYTES = kPacked ? 0 : (1 << (2 * VB)) * 128;
-  static constexpr int BYTES = kPacked ? 256 * 256 : K_BYTES + V_BYTES;
-  uint32_t base;   // shared-window address of the tables
-  uint32_t lane4;  // 4 * lane
-  __device__ __forceinline__ static uint32_t lds(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
-    return v;
-  }
-  __device__ __forceinline__ uint32_t k(uint32_t e) const { return lds(base + ((e << 7) | lane4)); }
-  __device__ __forceinline__ uint32_t v(uint32_t e) const { return lds(base + K_BYTES + ((e << 7) | lane4)); }
-  // byte `Bt` of word w as the pair index (packed layout only)
-  template <int Bt>
-  __device__ __forceinline__ uint32_t k_byte(uint32_t w) const {
-    return lds(base + __byte_perm(w, lane4, 0x5504u | (Bt << 4)));
-  }
-  template <int Bt>
-  __device__ __forceinline__ uint32_t v_byte(uint32_t w) const {
-    return lds(base + 128 + __byte_perm(w, lane4, 0x5504u | (Bt << 4)));
-  }
-};
-
-// Key pair P (0..15) of a thread's code chunk, as a half2 of centroids.
-template <int KB, int VB, int P>
-__device__ __forceinline__ uint32_t k_pair(const PairLut<KB, VB>& L, const uint32_t (&c)[KB]) {
-  if constexpr (PairLut<KB, VB>::kPacked) {
-    return L.template k_byte<P & 3>(c[P >> 2]);
-  } else {
-    return L.k(k_pair_index<KB, P>(c));
-  }
-}
-// Value pair NU of a token pair, as a half2 of centroids.
-template <int KB, int VB, int NU>
-__device__ __forceinline__ uint32_t v_pair(const PairLut<KB, VB>& L, const VPairs<VB>& p) {
-  if constexpr (PairLut<KB, VB>::kPacked) {
-    return L.template v_byte<((NU & 7) >> 1)>(p.w[2 * (NU >> 3) + (NU & 1)]);
-  } else {
-    return L.v(p.template index<NU>());
-  }
-}
-
-// Split-K decode over one token range.  Transposed MMAs: tokens are the M dimension and the
-// columns are (head, part) pairs, part 0 = fp16 hi and part 1 = fp16 lo of the query-side operand,
-// so one m16n8k16 covers 16 tokens of four heads:
-//   scores   D[tok x (h,p)] += Khat[tok x dim] . Q'[dim x (h,p)]        (A from the pair tables)
-//   QJL      D[tok x (h,p)] += sign[tok x row] . SQ'[row x (h,p)]        (A = +-0.5 from the bits)
-//   values   O'[dim x (h,p)] += Vhat^T[dim x tok] . P~[tok x (h,p)]      (B = P~ transposed in
-//                                                                          registers by movmatrix)
-// NB = 1 (up to 4 heads per kv-head) or 2 (up to 8): n-blocks of four heads share the A operands.
-template <int KB, int VB, bool QJL, int NB>
-__global__ void __launch_bounds__(Cfg<KB, VB>::THREADS, Cfg<KB, VB>::MIN_BLOCKS) split_kernel(DArgs a) {
-  using Lay = Layout<KB, VB, QJL>;
-  using Lut = PairLut<KB, VB>;
-  constexpr int THREADS = Cfg<KB, VB>::THREADS, STAGE_TOK = Cfg<KB, VB>::STAGE_TOK;
-  constexpr int NSTAGE = Cfg<KB, VB>::NSTAGE, WARPS = Cfg<KB, VB>::W;
-  static_assert(Lay::LUT_BYTES == Lut::BYTES && Lut::K_BYTES + Lut::V_BYTES <= Lut::BYTES, "pair tables");
-  extern __shared__ __align__(16) unsigned char smem[];
-  unsigned char* pipe = smem + Lay::LUT_BYTES;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, t = lane & 3;
-  const int split = blockIdx.x;
-  const int kvh = blockIdx.y / a.hgroups, hg = blockIdx.y % a.hgroups;
-  const int b = blockIdx.z;
-  const int h0 = kvh * a.g + hg * HG;
-  const int nh = min(HG, a.g - hg * HG);
-  const int tok_begin = split * a.tps;
-  const int tok_end = min(a.seq_len, tok_begin + a.tps);
-  const int ntok = max(0, tok_end - tok_begin);
-  const int nstages = (ntok + STAGE_TOK - 1) / STAGE_TOK;
-  const int64_t row_base = ((int64_t)b * a.Hkv + kvh) * a.T_cap;
-
-  // Start the pipeline before building the tables.
-#pragma unroll
-  for (int s = 0; s < NSTAGE - 1; ++s) {
-    if (s < nstages)
-      load_stage<KB, VB, QJL>(a, pipe + s * Lay::STAGE_BYTES, row_base + tok_begin + s * STAGE_TOK,
-                              min(STAGE_TOK, ntok - s * STAGE_TOK));
-    cp_commit();
-  }
-
-  // Pair tables: entry e = lo | hi << B  ->  half2(c[lo], c[hi]), replicated per lane (bank = lane).
-  if constexpr (Lut::kPacked) {
-    for (int i = tid; i < 256 * 64; i += THREADS) {
-      const int e = i >> 6, half = (i >> 5) & 1, ln = i & 31;
-      const float* c = half ? a.vc : a.kc;
-      *reinterpret_cast<uint32_t*>(smem + e * 256 + half * 128 + 4 * ln) = pack_half2(c[e & 15], c[e >> 4]);
-    }
-  } else {
-    for (int i = tid; i < Lut::K_BYTES / 4; i += THREADS) {
-      const int e = i >> 5;
-      reinterpret_cast<uint32_t*>(smem)[i] = pack_half2(a.kc[e & ((1 << KB) - 1)], a.kc[e >> KB]);
-    }
-    for (int i = tid; i < Lut::V_BYTES / 4; i += THREADS) {
-      const int e = i >> 5;
-      reinterpret_cast<uint32_t*>(smem + Lut::K_BYTES)[i] = pack_half2(a.vc[e & ((1 << VB) - 1)], a.vc[e >> VB]);
-    }
-  }
-  Lut L;
-  L.base = smem_u32(smem);
-  L.lane4 = 4u * (uint32_t)lane;
-
-  // Everything above reads only the cache; the rotated queries come from the prep kernel.
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  // the merge kernel may launch now; its CTAs wait for this grid to finish before reading
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-
-  // B operands: column gq of n-block nb = head 4 nb + gq/2, part gq%2 (0: fp16 hi, 1: fp16 lo);
-  // k-step kk: dims 16kk + 2t, +1 (reg 0) and 16kk + 8 + 2t, +1 (reg 1).
-  uint32_t bq[NB][8][2], bsq[NB][8][2];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    const int hh = 4 * nb + (gq >> 1);
-    const bool live = hh < nh;
-    const bool lo = gq & 1;
-    const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
-    const float* sp = a.sq + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int c0 = 16 * kk + 8 * r + 2 * t;
-        float hx, lx, hy, ly;
-        split_half(live ? qp[c0] : 0.0f, hx, lx);
-        split_half(live ? qp[c0 + 1] : 0.0f, hy, ly);
-        bq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
-        if constexpr (QJL) {
-          split_half(live ? sp[c0] : 0.0f, hx, lx);
-          split_half(live ? sp[c0 + 1] : 0.0f, hy, ly);
-          bsq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
-        } else {
-          bsq[nb][kk][r] = 0u;
-        }
-      }
-    }
-  }
-
-  // Output accumulators: n-block nb, dim block db: (dim 16db + gq, head 4nb + t) hi/lo in [0]/[1],
-  // (dim 16db + 8 + gq) in [2]/[3].
-  float oacc[NB][8][4];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) oacc[nb][i][0] = oacc[nb][i][1] = oacc[nb][i][2] = oacc[nb][i][3] = 0.0f;
-  float m_run[NB], l_run[NB];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    m_run[nb] = -INFINITY;
-    l_run[nb] = 0.0f;
-  }
-
-  for (int st = 0; st < nstages; ++st) {
-    cp_wait<NSTAGE - 2>();
-    __syncthreads();
-    {
-      const int s = st + NSTAGE - 1;
-      if (s < nstages)
-        load_stage<KB, VB, QJL>(a, pipe + (s % NSTAGE) * Lay::STAGE_BYTES,
-                                row_base + tok_begin + s * STAGE_TOK,
-                                min(STAGE_TOK, ntok - s * STAGE_TOK));
-      cp_commit();
-    }
-    const int wtok0 = st * STAGE_TOK + 16 * warp;  // first token of this warp, relative to range
-    if (wtok0 >= ntok) continue;                    // warp-uniform
-    const unsigned char* stage = pipe + (st % NSTAGE) * Lay::STAGE_BYTES;
-    const int r0 = 16 * warp + gq, r1 = r0 + 8;    // this lane's token rows in the stage
-
-    // ---- scores for tokens r0, r1 and heads 4nb + t ----
-    float kacc[NB][4], qacc[NB][4];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = 0.0f;
-    {
-      uint32_t c0[KB], c1[KB];
-      const uint32_t* k0 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r0 * Lay::K_ROW + 4 * KB * t);
-      const uint32_t* k1 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r1 * Lay::K_ROW + 4 * KB * t);
-#pragma unroll
-      for (int i = 0; i < KB; ++i) {
-        c0[i] = k0[i];
-        c1[i] = k1[i];
-      }
-#define TQ_KSTEP(KK)                                                                         \
-      {                                                                                      \
-        const uint32_t A[4] = {k_pair<KB, VB, 2 * (KK)>(L, c0), k_pair<KB, VB, 2 * (KK)>(L, c1), \
-                               k_pair<KB, VB, 2 * (KK) + 1>(L, c0),                          \
-                               k_pair<KB, VB, 2 * (KK) + 1>(L, c1)};                         \
-        _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                    \
-            mma16816(kacc[nb], A, bq[nb][KK][0], bq[nb][KK][1]);                              \
-      }
-      TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
-#undef TQ_KSTEP
-    }
-    if constexpr (QJL) {
-      const uint32_t s0 = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r0 * 16 + 4 * t);
-      const uint32_t s1 = *reinterpret_cast<const uint32_t*>(stage + Lay::OFF_SG + r1 * 16 + 4 * t);
-#define TQ_SSTEP(KK)                                                                         \
-      {                                                                                      \
-        const uint32_t A[4] = {sign_pair<2 * (KK)>(s0), sign_pair<2 * (KK)>(s1),             \
-                               sign_pair<2 * (KK) + 1>(s0), sign_pair<2 * (KK) + 1>(s1)};    \
-        _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                    \
-            mma16816(qacc[nb], A, bsq[nb][KK][0], bsq[nb][KK][1]);                            \
-      }
-      TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
-#undef TQ_SSTEP
-    }
-
-    // ---- online softmax (log2 units) per head 4nb + t over this warp's 16 tokens ----
-    const float nk0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r0);
-    const float nk1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r1);
-    float rn0 = 0.0f, rn1 = 0.0f;
-    if constexpr (QJL) {
-      rn0 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r0);
-      rn1 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r1);
-    }
-    const float nv0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r0) * 0.08838834764831845f;
-    const float nv1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r1) * 0.08838834764831845f;
-    const bool v0ok = wtok0 + gq < ntok, v1ok = wtok0 + 8 + gq < ntok;
-    uint32_t bp[NB][2];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      float s0 = (kacc[nb][0] + kacc[nb][1]) * (nk0 * a.sK);
-      float s1 = (kacc[nb][2] + kacc[nb][3]) * (nk1 * a.sK);
-      if constexpr (QJL) {
-        s0 = fmaf(qacc[nb][0] + qacc[nb][1], rn0 * a.sQ, s0);
-        s1 = fmaf(qacc[nb][2] + qacc[nb][3], rn1 * a.sQ, s1);
-      }
-      s0 = v0ok ? s0 : -INFINITY;
-      s1 = v1ok ? s1 : -INFINITY;
-      float mx = fmaxf(s0, s1);
-      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
-      const float m_new = fmaxf(m_run[nb], mx);
-      if (m_new > m_run[nb]) {  // uniform over the 8 lanes of head 4nb + t
-        const float alpha = ex2(m_run[nb] - m_new);  // ex2(-inf) = 0
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          oacc[nb][i][0] *= alpha;
-          oacc[nb][i][1] *= alpha;
-          oacc[nb][i][2] *= alpha;
-          oacc[nb][i][3] *= alpha;
-        }
-        l_run[nb] *= alpha;
-        m_run[nb] = m_new;
-      }
-      const float p0 = m_run[nb] == -INFINITY ? 0.0f : ex2(s0 - m_run[nb]);
-      const float p1 = m_run[nb] == -INFINITY ? 0.0f : ex2(s1 - m_run[nb]);
-      l_run[nb] += p0 + p1;
-      // P~ = p nV / sqrt(d) as fp16 hi + lo: row token, columns (head t, hi) and (head t, lo)
-      float hx, lx, hy, ly;
-      split_half(p0 * nv0, hx, lx);
-      split_half(p1 * nv1, hy, ly);
-      bp[nb][0] = movmatrix_trans(pack_half2(hx, lx));  // tokens 2t, 2t+1 of column gq
-      bp[nb][1] = movmatrix_trans(pack_half2(hy, ly));  // tokens 2t+8, 2t+9
-    }
-
-    // ---- O'^T += Vhat^T P~: dim blocks of 16; A holds token pairs (2t,2t+1), (2t+8,2t+9) ----
-    {
-      const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
-      const uint64_t cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
-      const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
-      const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
-      const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
-      VPairs<VB> p01, p89;
-      p01.build(cv0, cv1);
-      p89.build(cv2, cv3);
-#define TQ_VSTEP(DB)                                                                          \
-      {                                                                                       \
-        const uint32_t A[4] = {v_pair<KB, VB, 2 * (DB)>(L, p01), v_pair<KB, VB, 2 * (DB) + 1>(L, p01), \
-                               v_pair<KB, VB, 2 * (DB)>(L, p89), v_pair<KB, VB, 2 * (DB) + 1>(L, p89)}; \
-        _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                     \
-            mma16816(oacc[nb][DB], A, bp[nb][0], bp[nb][1]);                                   \
-      }
-      TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3) TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
-#undef TQ_VSTEP
-    }
-  }
-  cp_wait<0>();
-  __syncthreads();  // pipeline buffers are reused for the merge below
-
-  // ---- merge the 4 warps of this CTA ----
-  float* mw = reinterpret_cast<float*>(pipe);  // [WARPS][HG]
-  float* lw = mw + WARPS * HG;                 // [WARPS][HG]
-  float* ow = lw + WARPS * HG;                 // [WARPS][HG][D]
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    const int hh = 4 * nb + t;
-    float lq = l_run[nb];
-    lq += __shfl_xor_sync(FULL, lq, 4);
-    lq += __shfl_xor_sync(FULL, lq, 8);
-    lq += __shfl_xor_sync(FULL, lq, 16);
-    if (gq == 0) {
-      mw[warp * HG + hh] = m_run[nb];
-      lw[warp * HG + hh] = lq;
-    }
-    float* o = ow + (warp * HG + hh) * D;
-#pragma unroll
-    for (int db = 0; db < 8; ++db) {
-      o[16 * db + gq] = oacc[nb][db][0] + oacc[nb][db][1];
-      o[16 * db + 8 + gq] = oacc[nb][db][2] + oacc[nb][db][3];
-    }
-  }
-  __syncthreads();
-  for (int r = 0; r < nh && tid < D; ++r) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, mw[w * HG + r]);
-    float Ls = 0.0f, O = 0.0f;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) {
-      const float mwr = mw[w * HG + r];
-      const float f = (mwr == -INFINITY) ? 0.0f : ex2(mwr - M);
-      Ls += f * lw[w * HG + r];
-      O += f * ow[(w * HG + r) * D + tid];
-    }
-    float* dst = a.part + (((int64_t)b * a.Hq + h0 + r) * a.splits + split) * PART;
-    dst[4 + tid] = O;
-    if (tid == 0) {
-      dst[0] = M;
-      dst[1] = Ls;
-    }
-  }
-
-}
+inline size_t merge_smem_bytes(int pmax) { return sizeof(float) * ((size_t)pmax + ((pmax + 3) & ~3) + 9 * D); }
 
 // ------------------------------------------------------------------------------------------ host
 
 struct Plan {
-  int hgroups, splits, tps;
+  int hgroups, units, ctas, pmax;
+  int64_t ntot;
 };
 
-int device_sms() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+int device_attr(cudaDeviceAttr attr, int fallback) {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, attr, dev) != cudaSuccess || v <= 0) {
     cudaGetLastError();
-    return 148;
+    return fallback;
   }
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
-    cudaGetLastError();
-    return 148;
-  }
-  return sms;
+  return v;
 }
+int device_sms() { return device_attr(cudaDevAttrMultiProcessorCount, 148); }
+// Dynamic shared memory of a split CTA: all an SM gives one block, in whole 256-byte units.
+int split_dyn_smem() { return device_attr(cudaDevAttrMaxSharedMemoryPerBlockOptin, 232448) / 256 * 256; }
 
-// Resident split CTAs per SM: the 4-bit pair tables (64 KB) allow two, the smaller ones three
-// (register-bound, see split_kernel's launch bounds).
-int resident_ctas(int kb, int vb) { return (kb == 4 && vb == 4) ? 2 : 3; }
-// (two six-warp CTAs with the 4-bit tables, three four-warp CTAs otherwise)
-
-Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms, int resident, int stage_tok) {
-  const int STAGE_TOK = stage_tok;
+Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
   Plan p;
   const int g = Hq / Hkv;
   p.hgroups = (g + HG - 1) / HG;
-  const int64_t units = (int64_t)B * Hkv * p.hgroups;
+  p.units = B * Hkv * p.hgroups;
+  p.ntot = (int64_t)p.units * seq_len;
   if (seq_len <= 0) {
-    p.splits = 1;
-    p.tps = STAGE_TOK;
+    p.ctas = 0;
+    p.pmax = 0;
     return p;
   }
-  // One wave of resident CTAs: the largest split count whose grid still fits it.
-  const int64_t slots = (int64_t)resident * sms;
-  int64_t splits = slots / units;
-  const int64_t max_splits = (seq_len + 4 * STAGE_TOK - 1) / (4 * STAGE_TOK);  // >= 4 stages each
-  if (splits > max_splits) splits = max_splits;
-  if (splits > SPLITS_MAX) splits = SPLITS_MAX;
-  if (splits < 1) splits = 1;
-  int64_t tps = (seq_len + splits - 1) / splits;
-  tps = (tps + STAGE_TOK - 1) / STAGE_TOK * STAGE_TOK;
-  p.tps = (int)tps;
-  p.splits = (int)((seq_len + tps - 1) / tps);
+  int64_t c = p.ntot / MIN_TOK_PER_CTA;
+  if (c > sms) c = sms;
+  if (c < 1) c = 1;
+  p.ctas = (int)c;
+  // partial slots per head: the most CTA ranges one unit meets (exact for up to 2^16 units)
+  if (p.units <= (1 << 16)) {
+    int pm = 1;
+    for (int64_t u = 0; u < p.units; ++u) {
+      const int n = part_cta_of(p.ntot, p.ctas, u * seq_len + seq_len - 1) - part_cta_of(p.ntot, p.ctas, u * seq_len) + 1;
+      pm = n > pm ? n : pm;
+    }
+    p.pmax = pm;
+  } else {  // ranges are at least floor(N / C) >= MIN_TOK_PER_CTA long
+    const int64_t minlen = p.ntot / p.ctas;
+    p.pmax = (int)std::min<int64_t>(p.ctas, (seq_len + minlen - 1) / minlen + 1);
+  }
   return p;
 }
 
-// Workspace: q' and S q' [B*Hq][128] fp32, then the split partials [B*Hq][splits][132] fp32.
-size_t workspace_bytes(int B, int Hq, int Hkv, const Plan& p) {
-  (void)Hkv;
-  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.splits * PART);
+// Workspace: q' and S q' [B*Hq][128] fp32, then the partials [B*Hq][pmax][132] fp32.
+size_t workspace_bytes(int B, int Hq, const Plan& p) {
+  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.pmax * PART);
 }
 
 template <int KB, int VB, bool QJL, int NB>
-tq_status launch_split_nb(const DArgs& a, dim3 grid, cudaStream_t stream) {
-  using Lay = Layout<KB, VB, QJL>;
-  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+tq_status launch_split_nb(const DArgs& a, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       a.dyn_smem);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
   // programmatic dependent launch: the prologue (tables, first cache stages) overlaps prep
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(Cfg<KB, VB>::THREADS);
-  cfg.dynamicSmemBytes = Lay::SMEM;
+  cfg.gridDim = dim3(a.ctas);
+  cfg.blockDim = dim3(Shape<NB>::THREADS);
+  cfg.dynamicSmemBytes = a.dyn_smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -864,25 +1018,25 @@ tq_status launch_split_nb(const DArgs& a, dim3 grid, cudaStream_t stream) {
 
 // One n-block of four heads when a group has at most four query heads, else two.
 template <int KB, int VB, bool QJL>
-tq_status launch_split(const DArgs& a, dim3 grid, cudaStream_t stream) {
-  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1>(a, grid, stream) : launch_split_nb<KB, VB, QJL, 2>(a, grid, stream);
+tq_status launch_split(const DArgs& a, cudaStream_t stream) {
+  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1>(a, stream) : launch_split_nb<KB, VB, QJL, 2>(a, stream);
 }
 
 template <int KB, bool QJL>
-tq_status dispatch_v(int vb, const DArgs& a, dim3 grid, cudaStream_t s) {
+tq_status dispatch_v(int vb, const DArgs& a, cudaStream_t s) {
   switch (vb) {
-    case 2: return launch_split<KB, 2, QJL>(a, grid, s);
-    case 3: return launch_split<KB, 3, QJL>(a, grid, s);
-    default: return launch_split<KB, 4, QJL>(a, grid, s);
+    case 2: return launch_split<KB, 2, QJL>(a, s);
+    case 3: return launch_split<KB, 3, QJL>(a, s);
+    default: return launch_split<KB, 4, QJL>(a, s);
   }
 }
 
 template <bool QJL>
-tq_status dispatch(int kb, int vb, const DArgs& a, dim3 grid, cudaStream_t s) {
+tq_status dispatch(int kb, int vb, const DArgs& a, cudaStream_t s) {
   switch (kb) {
-    case 2: return dispatch_v<2, QJL>(vb, a, grid, s);
-    case 3: return dispatch_v<3, QJL>(vb, a, grid, s);
-    default: return dispatch_v<4, QJL>(vb, a, grid, s);
+    case 2: return dispatch_v<2, QJL>(vb, a, s);
+    case 3: return dispatch_v<3, QJL>(vb, a, s);
+    default: return dispatch_v<4, QJL>(vb, a, s);
   }
 }
 
@@ -892,9 +1046,14 @@ tq_status dispatch(int kb, int vb, const DArgs& a, dim3 grid, cudaStream_t s) {
 extern "C" size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_len) {
   using namespace tq;
   if (!cache || B < 1 || Hq < 1 || cache->Hkv < 1 || Hq % cache->Hkv || seq_len < 0) return 0;
-  const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms(),
-                           resident_ctas(cache->k_bits, cache->v_bits), stage_tokens(cache->k_bits, cache->v_bits));
-  return workspace_bytes(B, Hq, cache->Hkv, p);
+  const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
+  return workspace_bytes(B, Hq, p);
+}
+
+extern "C" int tq_decode_device_errors(void) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tq::g_decode_error, sizeof(v)) != cudaSuccess) return -1;
+  return (int)v;
 }
 
 extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, int Hq,
@@ -914,70 +1073,76 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
     return fail(TQ_ERR_INVALID_ARG, "q / out / workspace must be 16-byte aligned");
   const int B = cache->B;
-  const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms(),
-                              resident_ctas(cache->k_bits, cache->v_bits), stage_tokens(cache->k_bits, cache->v_bits));
-  const size_t need = workspace_bytes(B, Hq, cache->Hkv, plan);
+  const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
+  const size_t need = workspace_bytes(B, Hq, plan);
   if (ws_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
 
   const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)D);
   float* ws = reinterpret_cast<float*>(workspace);
-  DArgs a;
-  a.B = B;
-  a.Hq = Hq;
-  a.Hkv = cache->Hkv;
-  a.g = Hq / cache->Hkv;
-  a.hgroups = plan.hgroups;
-  a.T_cap = cache->T_cap;
-  a.seq_len = seq_len;
-  a.splits = plan.splits;
-  a.tps = plan.tps;
-  a.sK = (float)((double)sc * 1.4426950408889634 / sqrt((double)D));
-  a.sQ = cache->qjl_m ? (float)((double)sc * 1.4426950408889634 * 2.0 * sqrt(M_PI / 2.0) / cache->qjl_m)
-                      : 0.0f;
-  a.k_codes = cache->k_codes;
-  a.k_signs = cache->k_signs;
-  a.k_norm = cache->k_norm;
-  a.k_rnorm = cache->k_rnorm;
-  a.v_codes = cache->v_codes;
-  a.v_norm = cache->v_norm;
-  a.kc = params->k_centroids;
-  a.vc = params->v_centroids;
-  a.qrot = ws;
-  a.sq = ws + (size_t)B * Hq * D;
-  a.part = ws + (size_t)2 * B * Hq * D;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
   const int BH = B * Hq;
-  // heads per cluster: about 16 clusters at least (one CTA on each of 128 SMs), at most PREP_HB
-  const int hb = std::max(1, std::min(PREP_HB, BH / 16));
-  const int prep_ctas = (BH + hb - 1) / hb * PREP_CLUSTER;
-  if (q_dtype == TQ_F32)
-    prep_kernel<float><<<prep_ctas, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), BH, hb, params->Pi,
-                                                           params->S, cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D);
-  else
-    prep_kernel<__nv_bfloat16><<<prep_ctas, PREP_THREADS, 0, s>>>(
-        reinterpret_cast<const __nv_bfloat16*>(q), BH, hb, params->Pi, params->S, cache->qjl_m ? 1 : 0, ws,
-        ws + (size_t)BH * D);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
+  const int g = Hq / cache->Hkv;
+  cudaError_t e;
+  if (seq_len > 0) {
+    DArgs a;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = cache->Hkv;
+    a.g = g;
+    a.hgroups = plan.hgroups;
+    a.T_cap = cache->T_cap;
+    a.seq_len = seq_len;
+    a.units = plan.units;
+    a.ctas = plan.ctas;
+    a.pmax = plan.pmax;
+    a.ntot = plan.ntot;
+    a.dyn_smem = split_dyn_smem();
+    a.sK = (float)((double)sc * 1.4426950408889634 / sqrt((double)D));
+    a.sQ = cache->qjl_m ? (float)((double)sc * 1.4426950408889634 * 2.0 * sqrt(M_PI / 2.0) / cache->qjl_m)
+                        : 0.0f;
+    a.k_codes = cache->k_codes;
+    a.k_signs = cache->k_signs;
+    a.k_norm = cache->k_norm;
+    a.k_rnorm = cache->k_rnorm;
+    a.v_codes = cache->v_codes;
+    a.v_norm = cache->v_norm;
+    a.kc = params->k_centroids;
+    a.vc = params->v_centroids;
+    a.qrot = ws;
+    a.sq = ws + (size_t)BH * D;
+    a.part = ws + (size_t)2 * BH * D;
 
-  const dim3 grid(plan.splits, cache->Hkv * plan.hgroups, B);
-  st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, a, grid, s)
-                    : dispatch<false>(cache->k_bits, cache->v_bits, a, grid, s);
-  if (st != TQ_OK) return st;
-  // merge: programmatic dependent of split (its CTAs wait for the split grid before reading)
+    // heads per cluster: about 16 clusters at least (one CTA on each of 128 SMs), at most PREP_HB
+    const int hb = std::max(1, std::min(PREP_HB, BH / 16));
+    const int prep_ctas = (BH + hb - 1) / hb * PREP_CLUSTER;
+    if (q_dtype == TQ_F32)
+      prep_kernel<float><<<prep_ctas, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), BH, hb, params->Pi,
+                                                             params->S, cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D);
+    else
+      prep_kernel<__nv_bfloat16><<<prep_ctas, PREP_THREADS, 0, s>>>(
+          reinterpret_cast<const __nv_bfloat16*>(q), BH, hb, params->Pi, params->S, cache->qjl_m ? 1 : 0, ws,
+          ws + (size_t)BH * D);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
+    st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, a, s)
+                      : dispatch<false>(cache->k_bits, cache->v_bits, a, s);
+    if (st != TQ_OK) return st;
+  }
+  // merge: programmatic dependent of split (its CTAs wait for the split grid before reading); with
+  // an empty context it only writes zeros
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH);
   cfg.blockDim = dim3(MERGE_THREADS);
-  cfg.dynamicSmemBytes = merge_smem_bytes(plan.splits);
+  cfg.dynamicSmemBytes = merge_smem_bytes(plan.pmax);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, merge_kernel, (const float*)a.part, params->Pi, out, plan.splits);
+  cfg.numAttrs = seq_len > 0 ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, merge_kernel, (const float*)(ws + (size_t)2 * BH * D), params->Pi, out, Hq, g,
+                         cache->Hkv, plan.hgroups, (int64_t)seq_len, plan.ntot, plan.ctas, plan.pmax);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }

@@ -225,6 +225,16 @@ tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, in
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Diagnostics of tq_decode_attn (host; synchronizes with the device).  The split kernel's waits on
+ * its shared-memory pipeline are bounded (about two seconds each); one that gives up records it
+ * here and the call's output is not valid.
+ *   bit 0: a pipeline wait timed out;  bit 1: the device's shared memory per block was too small
+ *   for the pipeline.  0 = no error since the library was loaded; -1 if the device could not be
+ *   queried.
+ */
+int tq_decode_device_errors(void);
+
+/*
  * One autoregressive decode step: compress the new token's K and V into cache row t of every
  * (batch, kv-head), then attend q over rows [0, t].  Enqueues tq_quantize (T_new = 1) and
  * tq_decode_attn (seq_len = t + 1) back to back on `stream`, so one CUDA graph can hold a whole
