@@ -126,7 +126,10 @@ __device__ __forceinline__ uint64_t desc_at(const uint8_t* tile, int kstep) {
 
 // Load a row-major fp32 [128 x 128] matrix, times `scale` (a power of two), into an fp16 hi
 // (+ optional lo) operand tile, one 16-byte chunk (8 consecutive elements of a row) per step.
-__device__ void load_matrix(const float* __restrict__ M, float scale, uint8_t* hi, uint8_t* lo) {
+// Returns (per thread) whether any lo element it wrote is nonzero: a matrix exact in fp16 (the
+// structured rotation) then needs no lo MMA pass.
+__device__ bool load_matrix(const float* __restrict__ M, float scale, uint8_t* hi, uint8_t* lo) {
+  bool lo_nz = false;
   for (int i = threadIdx.x; i < D * D / 8; i += THREADS) {
     const int r = i / 16, c = i % 16;
     const float4 p0 = reinterpret_cast<const float4*>(M + r * D + 8 * c)[0];
@@ -144,7 +147,9 @@ __device__ void load_matrix(const float* __restrict__ M, float scale, uint8_t* h
     }
     *reinterpret_cast<uint4*>(hi + sw_chunk(r, c)) = make_uint4(h[0], h[1], h[2], h[3]);
     if (lo) *reinterpret_cast<uint4*>(lo + sw_chunk(r, c)) = make_uint4(l[0], l[1], l[2], l[3]);
+    lo_nz = lo_nz || ((l[0] | l[1] | l[2] | l[3]) & 0x7fff7fffu) != 0;
   }
+  return lo_nz;
 }
 
 // Positive-half search: k = #{T_j <= a} over the 2^(B-1)-1 positive thresholds T[1..], and the
@@ -325,7 +330,8 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   if (tid < TM) s.vflag[tid] = 0;
   // Pi enters as 2^8 Pi so that its fp16 lo part stays clear of the subnormal range (the hi + lo
   // pair then carries ~22 significant bits of every entry); the 2^-8 is folded into u's scale.
-  load_matrix(a.Pi, PI_SCALE, s.pih, s.pil);
+  // (a Pi exact in fp16, like the structured rotation, has no lo part: its MMA pass is skipped)
+  const bool pi_lo = __syncthreads_or(load_matrix(a.Pi, PI_SCALE, s.pih, s.pil) ? 1 : 0) != 0;
   if (a.qjl) load_matrix(a.S, 1.0f, s.sm, nullptr);
 
   const int tiles_per_bh = (a.T_new + TM - 1) / TM;
@@ -440,10 +446,10 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         umma_f16(tmem + COL_K, desc_at(s.xk, ks), desc_at(s.pih, ks), IDESC, ks > 0);
-        umma_f16(tmem + COL_K, desc_at(s.xk, ks), desc_at(s.pil, ks), IDESC, 1);
+        if (pi_lo) umma_f16(tmem + COL_K, desc_at(s.xk, ks), desc_at(s.pil, ks), IDESC, 1);
         if constexpr (sizeof(InT) == 4) umma_f16(tmem + COL_K, desc_at(s.xl, ks), desc_at(s.pih, ks), IDESC, 1);
         umma_f16(tmem + COL_V, desc_at(s.xv, ks), desc_at(s.pih, ks), IDESC, ks > 0);
-        umma_f16(tmem + COL_V, desc_at(s.xv, ks), desc_at(s.pil, ks), IDESC, 1);
+        if (pi_lo) umma_f16(tmem + COL_V, desc_at(s.xv, ks), desc_at(s.pil, ks), IDESC, 1);
       }
       umma_commit(&s.bar_kv);
     }

@@ -158,6 +158,7 @@ struct __align__(1024) PSmem {
   unsigned int main_done;
   unsigned int fix_done[N_FIX];
   uint32_t epoch;            // this launch's ring epoch
+  unsigned int pi_lo;        // Pi has a nonzero fp16 lo part (else its lo MMA pass is skipped)
 };
 
 static_assert(sizeof(PSmem) <= 232448, "shared memory per CTA");
@@ -227,7 +228,10 @@ __device__ __forceinline__ bool pwait_w(PSmem& s, uint64_t* bar, uint32_t parity
 }
 
 // Row-major fp32 [128 x 128] matrix times `scale` (a power of two) into fp16 hi (+ lo) tiles.
-__device__ void load_matrix(const float* __restrict__ M, float scale, uint8_t* hi, uint8_t* lo) {
+// Returns (per thread) whether any lo element it wrote is nonzero: a matrix exact in fp16 (the
+// structured rotation) then needs no lo MMA pass.
+__device__ bool load_matrix(const float* __restrict__ M, float scale, uint8_t* hi, uint8_t* lo) {
+  bool lo_nz = false;
   for (int i = threadIdx.x; i < D * D / 8; i += THREADS) {
     const int r = i / 16, c = i % 16;
     const float4 p0 = reinterpret_cast<const float4*>(M + r * D + 8 * c)[0];
@@ -244,7 +248,9 @@ __device__ void load_matrix(const float* __restrict__ M, float scale, uint8_t* h
     }
     *reinterpret_cast<uint4*>(hi + sw_chunk(r, c)) = make_uint4(h[0], h[1], h[2], h[3]);
     if (lo) *reinterpret_cast<uint4*>(lo + sw_chunk(r, c)) = make_uint4(l[0], l[1], l[2], l[3]);
+    lo_nz = lo_nz || ((l[0] | l[1] | l[2] | l[3]) & 0x7fff7fffu) != 0;
   }
+  return lo_nz;
 }
 
 // Uniform-cell code table for one codebook (one warp).  Cell k covers the u with
@@ -799,6 +805,7 @@ __device__ __noinline__ void role_mma(const PArgs& a, uint32_t tmem, int n_tiles
   const int lane = threadIdx.x & 31;
   // Y_K = X_K (Pi_hi + Pi_lo)^T and Y_V likewise, into tensor-memory buffer (tile & 1).  The sketch
   // MMA of a tile is issued by the epilogue warp that finishes its residuals last.
+  const bool pi_lo = s.pi_lo != 0;  // a structured (fp16-exact) Pi needs one pass, not two
   if (lane == 0) {
     int it = 0;
     for (; it < n_tiles; ++it) {
@@ -812,13 +819,13 @@ __device__ __noinline__ void role_mma(const PArgs& a, uint32_t tmem, int n_tiles
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         umma_f16(dk, desc_at(s.slot[sK], ks), desc_at(s.pih, ks), IDESC, ks > 0);
-        umma_f16(dk, desc_at(s.slot[sK], ks), desc_at(s.pil, ks), IDESC, 1);
+        if (pi_lo) umma_f16(dk, desc_at(s.slot[sK], ks), desc_at(s.pil, ks), IDESC, 1);
       }
       umma_commit(&s.empty[sK]);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         umma_f16(dv, desc_at(s.slot[sV], ks), desc_at(s.pih, ks), IDESC, ks > 0);
-        umma_f16(dv, desc_at(s.slot[sV], ks), desc_at(s.pil, ks), IDESC, 1);
+        if (pi_lo) umma_f16(dv, desc_at(s.slot[sV], ks), desc_at(s.pil, ks), IDESC, 1);
       }
       umma_commit(&s.empty[sV]);
       umma_commit(&s.yfull[bb]);
@@ -1238,6 +1245,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     s.stored_seq = 0;
     s.main_done = 0;
     s.epoch = *reinterpret_cast<volatile unsigned int*>(&g_pipe_epoch);
+    s.pi_lo = 0;
     for (int i = 0; i < N_FIX; ++i) s.fix_done[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -1250,7 +1258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == W_FIX + 1) build_lut(a.vt, LV, s.vlut, &s.alpha_v, &s.err);
   // Pi enters as 2^8 Pi so that its fp16 lo part stays clear of the subnormal range; the 2^-8 is
   // folded into the scale of u.
-  load_matrix(a.Pi, PI_SCALE, s.pih, s.pil);
+  if (load_matrix(a.Pi, PI_SCALE, s.pih, s.pil)) s.pi_lo = 1;
   if (a.qjl) load_matrix(a.S, 1.0f, s.sm, nullptr);
   fence_proxy_async_smem();
   tc_fence_before();
