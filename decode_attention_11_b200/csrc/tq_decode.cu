@@ -399,6 +399,23 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
   return v;
 }
+// Vector shared loads at addresses the caller guarantees aligned (stage rows are 16-byte aligned).
+__device__ __forceinline__ uint4 lds128(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(const void* p) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+  return v;
+}
+// x as fp16 hi + lo (about 22 significant bits) packed into one half2 (hi in the low half).
+__device__ __forceinline__ uint32_t hilo_half2(float x) {
+  const float hi = __half2float(__float2half_rn(x));
+  const __half2 h = __floats2half2_rn(hi, x - hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 // Pair tables: a pair of codes -> half2 of centroids, replicated per lane (bank = lane).
 // 4-bit keys and values: 256 entries of 256 bytes (K replicas at +0, V at +128) starting at a
@@ -500,7 +517,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
 
   if (warp == NW) {
     // ================================================================ producer
-    int it = 0, issued = 0;
+    int it = 0, issued = 0, slot = 0, round = 0;  // stage count, ring slot, times round the ring
     for (int64_t f = f_begin; f < f_end;) {
       const int64_t u = f / L;
       const int t0 = (int)(f - u * L);
@@ -509,24 +526,29 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       const int bk = (int)(u / a.hgroups);  // b * Hkv + kv-head
       const int64_t rowb = (int64_t)bk * a.T_cap;
       for (int s0 = t0; s0 < t1; s0 += ST, ++it) {
-        const int slot = it % ns;
-        if (it >= ns && !wait_w(ctl, &ctl.empty[slot], ((it / ns) - 1) & 1)) continue;
+        const int cur = slot, cur_round = round;  // this stage's slot, and its earlier uses
+        if (++slot == ns) {
+          slot = 0;
+          ++round;
+        }
+        // the slot's previous contents (use cur_round - 1) have been consumed
+        if (cur_round > 0 && !wait_w(ctl, &ctl.empty[cur], (cur_round - 1) & 1)) continue;
         if (*reinterpret_cast<volatile unsigned int*>(&ctl.err)) continue;
         const int ntok = min(ST, t1 - s0);
         const int64_t row0 = rowb + s0;
-        unsigned char* st = smem + ctl.stage_off[slot];
+        unsigned char* st = smem + ctl.stage_off[cur];
         if (lane == 0) {
-          mbar_expect_tx_(&ctl.full[slot], (uint32_t)(ntok * Lay::TX_PER_TOKEN));
-          bulk_g2s(st + Lay::OFF_KC, a.k_codes + row0 * Lay::K_ROW, ntok * Lay::K_ROW, &ctl.full[slot]);
-          if constexpr (QJL) bulk_g2s(st + Lay::OFF_SG, a.k_signs + row0 * 16, ntok * 16, &ctl.full[slot]);
-          bulk_g2s(st + Lay::OFF_VC, a.v_codes + row0 * Lay::V_ROW, ntok * Lay::V_ROW, &ctl.full[slot]);
+          mbar_expect_tx_(&ctl.full[cur], (uint32_t)(ntok * Lay::TX_PER_TOKEN));
+          bulk_g2s(st + Lay::OFF_KC, a.k_codes + row0 * Lay::K_ROW, ntok * Lay::K_ROW, &ctl.full[cur]);
+          if constexpr (QJL) bulk_g2s(st + Lay::OFF_SG, a.k_signs + row0 * 16, ntok * 16, &ctl.full[cur]);
+          bulk_g2s(st + Lay::OFF_VC, a.v_codes + row0 * Lay::V_ROW, ntok * Lay::V_ROW, &ctl.full[cur]);
         }
         for (int i = lane; i < ntok; i += 32) {
           cp_async4(st + Lay::OFF_NK + 4 * i, a.k_norm + row0 + i, 4);
           if constexpr (QJL) cp_async4(st + Lay::OFF_RN + 4 * i, a.k_rnorm + row0 + i, 4);
           cp_async4(st + Lay::OFF_NV + 4 * i, a.v_norm + row0 + i, 4);
         }
-        cp_async_arrive_noinc(&ctl.full[slot]);
+        cp_async_arrive_noinc(&ctl.full[cur]);
         issued = it + 1;
       }
     }
@@ -581,7 +603,8 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
   float* mw = mrg;                 // [NW][HGN]
   float* lw = mw + NW * HGN;       // [NW][HGN]
   float* ow = lw + NW * HGN;       // [NW][HGN][D]
-  int it = 0;
+  int slot = 0;
+  uint32_t phase = 0;  // parity of the ring round being consumed
   for (int64_t f = f_begin; f < f_end;) {
     const int64_t u = f / L;
     const int t0 = (int)(f - u * L);
@@ -673,28 +696,38 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       l_run[nb] = 0.0f;
     }
 
-    for (int s0 = t0; s0 < t1; s0 += ST, ++it) {
-      const int slot = it % ns;
-      const bool ok = wait_w(ctl, &ctl.full[slot], (it / ns) & 1);
+    for (int s0 = t0; s0 < t1; s0 += ST) {
+      const bool ok = wait_w(ctl, &ctl.full[slot], phase);
       const int nvalid = min(16, t1 - s0 - 16 * warp);
       if (ok && nvalid > 0) {
         const unsigned char* stage = smem + ctl.stage_off[slot];
         const int r0 = 16 * warp + gq, r1 = r0 + 8;  // this lane's token rows in the stage
 
         // ---- scores for tokens r0, r1 and heads 4nb + t ----
-        float kacc[NB][4], qacc[NB][4];
+        // two accumulators per product (even / odd k-steps) halve the dependent MMA chains
+        float kacc[NB][4], qacc[NB][4], kacc2[NB][4], qacc2[NB][4];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = 0.0f;
+          for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = kacc2[nb][e] = qacc2[nb][e] = 0.0f;
         {
           uint32_t c0[KB], c1[KB];
-          const uint32_t* k0 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r0 * Lay::K_ROW + 4 * KB * t);
-          const uint32_t* k1 = reinterpret_cast<const uint32_t*>(stage + Lay::OFF_KC + r1 * Lay::K_ROW + 4 * KB * t);
+          const unsigned char* k0 = stage + Lay::OFF_KC + r0 * Lay::K_ROW + 4 * KB * t;
+          const unsigned char* k1 = stage + Lay::OFF_KC + r1 * Lay::K_ROW + 4 * KB * t;
+          if constexpr (KB == 4) {
+            const uint4 x0 = lds128(k0), x1 = lds128(k1);
+            c0[0] = x0.x; c0[1] = x0.y; c0[2] = x0.z; c0[3] = x0.w;
+            c1[0] = x1.x; c1[1] = x1.y; c1[2] = x1.z; c1[3] = x1.w;
+          } else if constexpr (KB == 2) {
+            const uint2 x0 = lds64(k0), x1 = lds64(k1);
+            c0[0] = x0.x; c0[1] = x0.y;
+            c1[0] = x1.x; c1[1] = x1.y;
+          } else {
 #pragma unroll
-          for (int i = 0; i < KB; ++i) {
-            c0[i] = k0[i];
-            c1[i] = k1[i];
+            for (int i = 0; i < KB; ++i) {
+              c0[i] = reinterpret_cast<const uint32_t*>(k0)[i];
+              c1[i] = reinterpret_cast<const uint32_t*>(k1)[i];
+            }
           }
 #define TQ_KSTEP(KK)                                                                         \
           {                                                                                  \
@@ -702,7 +735,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
                                    k_pair<KB, VB, 2 * (KK) + 1>(lut, c0),                    \
                                    k_pair<KB, VB, 2 * (KK) + 1>(lut, c1)};                   \
             _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                \
-                mma16816(kacc[nb], A, bq[nb][KK][0], bq[nb][KK][1]);                          \
+                mma16816((KK) & 1 ? kacc2[nb] : kacc[nb], A, bq[nb][KK][0], bq[nb][KK][1]);    \
           }
           TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
 #undef TQ_KSTEP
@@ -715,7 +748,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
             const uint32_t A[4] = {sgn<2 * (KK)>(w0), sgn<2 * (KK)>(w1), sgn<2 * (KK) + 1>(w0), \
                                    sgn<2 * (KK) + 1>(w1)};                                   \
             _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                \
-                mma16816(qacc[nb], A, bsq[nb][KK][0], bsq[nb][KK][1]);                         \
+                mma16816((KK) & 1 ? qacc2[nb] : qacc[nb], A, bsq[nb][KK][0], bsq[nb][KK][1]);  \
           }
           TQ_SSTEP(0) TQ_SSTEP(1) TQ_SSTEP(2) TQ_SSTEP(3) TQ_SSTEP(4) TQ_SSTEP(5) TQ_SSTEP(6) TQ_SSTEP(7)
 #undef TQ_SSTEP
@@ -737,11 +770,11 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         uint32_t bp[NB][2];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          float s0v = (kacc[nb][0] + kacc[nb][1]) * (nk0 * fK[nb]);
-          float s1v = (kacc[nb][2] + kacc[nb][3]) * (nk1 * fK[nb]);
+          float s0v = ((kacc[nb][0] + kacc2[nb][0]) + (kacc[nb][1] + kacc2[nb][1])) * (nk0 * fK[nb]);
+          float s1v = ((kacc[nb][2] + kacc2[nb][2]) + (kacc[nb][3] + kacc2[nb][3])) * (nk1 * fK[nb]);
           if constexpr (QJL) {
-            s0v = fmaf(qacc[nb][0] + qacc[nb][1] + Kh[nb], rn0 * fQ[nb], s0v);
-            s1v = fmaf(qacc[nb][2] + qacc[nb][3] + Kh[nb], rn1 * fQ[nb], s1v);
+            s0v = fmaf(((qacc[nb][0] + qacc2[nb][0]) + (qacc[nb][1] + qacc2[nb][1])) + Kh[nb], rn0 * fQ[nb], s0v);
+            s1v = fmaf(((qacc[nb][2] + qacc2[nb][2]) + (qacc[nb][3] + qacc2[nb][3])) + Kh[nb], rn1 * fQ[nb], s1v);
           }
           s0v = v0ok ? s0v : -INFINITY;
           s1v = v1ok ? s1v : -INFINITY;
@@ -765,20 +798,34 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
           const float p1 = ex2(s1v - m_run[nb]);
           l_run[nb] += p0 + p1;
           // P~ = p nV / sqrt(d) as fp16 hi + lo: row token, columns (head t, hi) and (head t, lo)
-          float hx, lx, hy, ly;
-          split_half(p0 * nv0, hx, lx);
-          split_half(p1 * nv1, hy, ly);
-          bp[nb][0] = movmatrix_trans(pack_half2(hx, lx));  // tokens 2t, 2t+1 of column gq
-          bp[nb][1] = movmatrix_trans(pack_half2(hy, ly));  // tokens 2t+8, 2t+9
+          bp[nb][0] = movmatrix_trans(hilo_half2(p0 * nv0));  // tokens 2t, 2t+1 of column gq
+          bp[nb][1] = movmatrix_trans(hilo_half2(p1 * nv1));  // tokens 2t+8, 2t+9
         }
 
         // ---- O'^T += Vhat^T P~: dim blocks of 16; A holds token pairs (2t,2t+1), (2t+8,2t+9) ----
         {
           const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
-          const uint64_t cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
-          const uint64_t cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
-          const uint64_t cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
-          const uint64_t cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
+          uint64_t cv0, cv1, cv2, cv3;
+          if constexpr (VB == 4) {
+            // lanes with odd t read their odd row first, so that in each load the four t-lanes
+            // of a column group hit two bank groups instead of one (64-byte rows)
+            const int sw = t & 1;
+            const uint2 a0 = lds64(vbase + (2 * t + sw) * Lay::V_ROW + 8 * gq);
+            const uint2 a1 = lds64(vbase + (2 * t + 1 - sw) * Lay::V_ROW + 8 * gq);
+            const uint2 a2 = lds64(vbase + (2 * t + 8 + sw) * Lay::V_ROW + 8 * gq);
+            const uint2 a3 = lds64(vbase + (2 * t + 9 - sw) * Lay::V_ROW + 8 * gq);
+            const uint64_t x0 = (uint64_t)a0.x | ((uint64_t)a0.y << 32), x1 = (uint64_t)a1.x | ((uint64_t)a1.y << 32);
+            const uint64_t x2 = (uint64_t)a2.x | ((uint64_t)a2.y << 32), x3 = (uint64_t)a3.x | ((uint64_t)a3.y << 32);
+            cv0 = sw ? x1 : x0;
+            cv1 = sw ? x0 : x1;
+            cv2 = sw ? x3 : x2;
+            cv3 = sw ? x2 : x3;
+          } else {
+            cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
+            cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
+            cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
+            cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
+          }
           VPairs<VB> p01, p89;
           p01.build(cv0, cv1);
           p89.build(cv2, cv3);
@@ -795,6 +842,10 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_(&ctl.empty[slot]);
+      if (++slot == ns) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
 
     // ---- merge the NW warps: one (max, sum, o') partial per head of this segment ----
