@@ -367,6 +367,181 @@ def exact_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: Optional
 
 
 # ---------------------------------------------------------------------------
+# Outlier-aware mixed precision (tproger.ru, section on TheTom's llama.cpp fork: "turbo3" is
+# 3.5-bit KV quantization, 4.6x smaller than FP16; ai-manual.ru M5 Max KV-cache benchmark,
+# "when TurboQuant is needed": per-layer outlier-aware 3/4-bit quantization)
+#
+# Reading (the pages give no construction): the head's channels split into two fixed halves,
+# an "outlier" half O (a per-layer parameter, 64 channels) coded with bits_O and the other half
+# R with bits_R (4 and 3 bits average 3.5).  Each half is an instance of the method's first two
+# steps on its own: its own random rotation (the block rotation Pi_blk puts Pi_O x_O in rows
+# 0..63 and Pi_R x_R in rows 64..127), its own norm n_g = ||x_g||, coordinates
+# u_g = sqrt(64) (Pi_blk x)_g / n_g and its own Lloyd-Max codebook.  The QJL step is unchanged
+# but acts on the whole residual in the block-rotated basis,
+#     r = Pi_blk x - khat,   khat_g = (n_g / sqrt(64)) c_g[idx_g],
+# so the estimator <q,k> ~= <q',khat> + ||r|| sqrt(pi/2)/m <S q', sign(S r)> (q' = Pi_blk q) keeps
+# its form.  The sketch value compared with 0 is taken in the units of the plain method,
+# sigma = sqrt(128)/||x|| S r (which equals S rho when both halves share one norm).
+# ---------------------------------------------------------------------------
+
+HALF = D // 2
+
+
+def quantize_vectors_mixed(X: np.ndarray, Pi_blk: np.ndarray, outlier_channels, bits_O: int,
+                           bits_R: int, S: Optional[np.ndarray] = None) -> dict:
+    """Compress N vectors (rows of X, taken exactly in float64) in the mixed layout.
+
+    n_g = ||x restricted to the channels of half g||;  y = Pi_blk x;
+    u_g = sqrt(64) y_g / n_g (0 when n_g = 0);  idx_g = #{i : u_g >= t_i of codebook(bits_g)};
+    with S: r = y - khat, ||r||, sigma = sqrt(128)/||x|| S r, sign_l = [sigma_l >= 0]."""
+    X = np.asarray(X, dtype=np.float64)
+    P = np.asarray(Pi_blk, dtype=np.float64)
+    O = np.sort(np.asarray(outlier_channels, dtype=np.int64))
+    R = np.setdiff1d(np.arange(D), O)
+    n = {0: np.sqrt(np.sum(X[:, O] ** 2, axis=-1)), 1: np.sqrt(np.sum(X[:, R] ** 2, axis=-1))}
+    Y = X @ P.T
+    u = np.zeros_like(Y)
+    idx = np.zeros(Y.shape, dtype=np.int64)
+    khat = np.zeros_like(Y)
+    for g, bits in ((0, bits_O), (1, bits_R)):
+        cols = slice(HALF * g, HALF * (g + 1))
+        ng = n[g]
+        safe = np.where(ng > 0, ng, 1.0)
+        u[:, cols] = np.where((ng > 0)[:, None], math.sqrt(HALF) * Y[:, cols] / safe[:, None], 0.0)
+        cb = codebook(bits)
+        idx[:, cols] = quantize_index(u[:, cols], cb.thresholds)
+        khat[:, cols] = (ng[:, None] / math.sqrt(HALF)) * cb.centroids[idx[:, cols]]
+    out = {"n_O": n[0], "n_R": n[1], "u": u, "idx": idx, "y": Y, "khat": khat}
+    if S is not None:
+        S = np.asarray(S, dtype=np.float64)
+        r = Y - khat
+        out["rnorm"] = np.sqrt(np.sum(r * r, axis=-1))
+        nx = np.sqrt(n[0] ** 2 + n[1] ** 2)
+        sproj = np.where((nx > 0)[:, None], math.sqrt(D) * (r @ S.T) / np.where(nx > 0, nx, 1.0)[:, None], 0.0)
+        out["sproj"] = sproj
+        out["signs"] = (sproj >= 0).astype(np.int64)
+    return out
+
+
+def k_slot_of_coord_mixed(j: int) -> int:
+    """Mixed key row: half g = j // 64 is its own bit stream (half O first); within it,
+    j - 64 g = 16 a + 8 h + 2 tau + eps sits at slot 16 tau + 4 a + 2 h + eps."""
+    jj = j % HALF
+    a, rem = divmod(jj, 16)
+    h, rem = divmod(rem, 8)
+    tau, eps = divmod(rem, 2)
+    return 16 * tau + 4 * a + 2 * h + eps
+
+
+def v_slot_of_coord_mixed(j: int) -> int:
+    """Mixed value row: within half g, coordinate j - 64 g = 8 nu + gam sits at slot 8 gam + nu."""
+    nu, gam = divmod(j % HALF, 8)
+    return 8 * gam + nu
+
+
+def pack_codes_mixed(idx: np.ndarray, bits_O: int, bits_R: int, slot_of_coord) -> np.ndarray:
+    """Rows of 128 codes -> bytes[N, 8 (bits_O + bits_R)]: the half-O stream (64 codes of bits_O
+    bits, slot s at bits [bits_O s, bits_O s + bits_O)), then the half-R stream."""
+    N = idx.shape[0]
+    parts = []
+    for g, bits in ((0, bits_O), (1, bits_R)):
+        part = np.zeros((N, HALF * bits // 8), dtype=np.uint8)
+        for j in range(HALF * g, HALF * (g + 1)):
+            s = slot_of_coord(j)
+            for i in range(bits):
+                k = bits * s + i
+                part[:, k // 8] |= (((idx[:, j] >> i) & 1).astype(np.uint8)) << (k % 8)
+        parts.append(part)
+    return np.concatenate(parts, axis=1)
+
+
+def unpack_codes_mixed(rows: np.ndarray, bits_O: int, bits_R: int, slot_of_coord) -> np.ndarray:
+    rows = np.asarray(rows, dtype=np.uint8)
+    N = rows.shape[0]
+    idx = np.zeros((N, D), dtype=np.int64)
+    off = 0
+    for g, bits in ((0, bits_O), (1, bits_R)):
+        for j in range(HALF * g, HALF * (g + 1)):
+            s = slot_of_coord(j)
+            for i in range(bits):
+                k = bits * s + i
+                idx[:, j] |= ((rows[:, off + k // 8] >> (k % 8)) & 1).astype(np.int64) << i
+        off += HALF * bits // 8
+    return idx
+
+
+def quantize_cache_mixed(K: np.ndarray, V: np.ndarray, Pi_blk: np.ndarray, outlier_channels,
+                         k_bits: tuple, v_bits: tuple, S: Optional[np.ndarray]) -> dict:
+    """K, V: [B, Hkv, T, d]; k_bits, v_bits = (bits_O, bits_R).  Packed arrays in the mixed
+    layout (norms [B, Hkv, T, 2] = (n_O, n_R)) plus the float64 intermediates."""
+    B, H, T, d = K.shape
+    kq = quantize_vectors_mixed(K.reshape(-1, d), Pi_blk, outlier_channels, *k_bits, S)
+    vq = quantize_vectors_mixed(V.reshape(-1, d), Pi_blk, outlier_channels, *v_bits, None)
+    cache = {
+        "k_codes": pack_codes_mixed(kq["idx"], *k_bits, k_slot_of_coord_mixed).reshape(B, H, T, -1),
+        "k_norm": np.stack([kq["n_O"], kq["n_R"]], -1).astype(np.float32).reshape(B, H, T, 2),
+        "v_codes": pack_codes_mixed(vq["idx"], *v_bits, v_slot_of_coord_mixed).reshape(B, H, T, -1),
+        "v_norm": np.stack([vq["n_O"], vq["n_R"]], -1).astype(np.float32).reshape(B, H, T, 2),
+        "k_u": kq["u"].reshape(B, H, T, d), "k_idx": kq["idx"].reshape(B, H, T, d),
+        "v_u": vq["u"].reshape(B, H, T, d), "v_idx": vq["idx"].reshape(B, H, T, d),
+    }
+    if S is not None:
+        cache["k_signs"] = pack_signs(kq["signs"]).reshape(B, H, T, -1)
+        cache["k_rnorm"] = kq["rnorm"].astype(np.float32).reshape(B, H, T)
+        cache["k_sproj"] = kq["sproj"].reshape(B, H, T, -1)
+    return cache
+
+
+def dequantize_mixed(codes: np.ndarray, norms: np.ndarray, bits: tuple, slot_of_coord) -> np.ndarray:
+    """khat (or vhat) in the block-rotated basis: half g = (n_g / sqrt(64)) c_g[idx_g]."""
+    idx = unpack_codes_mixed(codes, bits[0], bits[1], slot_of_coord)
+    norms = np.asarray(norms, np.float64)
+    out = np.zeros(idx.shape, dtype=np.float64)
+    for g in range(2):
+        cols = slice(HALF * g, HALF * (g + 1))
+        out[:, cols] = (norms[:, g:g + 1] / math.sqrt(HALF)) * codebook(bits[g]).centroids[idx[:, cols]]
+    return out
+
+
+def decode_attention_mixed(q: np.ndarray, Pi_blk: np.ndarray, S: Optional[np.ndarray], cache: dict,
+                           k_bits: tuple, v_bits: tuple, seq_len: int,
+                           scale: Optional[float] = None) -> np.ndarray:
+    """Decode attention over a mixed-layout cache: est_i = <q', khat_i> + ||r_i|| sqrt(pi/2)/m
+    <S q', 2 sign_i - 1>, q' = Pi_blk q; o = Pi_blk^T sum_i softmax(scale est)_i vhat_i."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    Hkv = cache["k_codes"].shape[1]
+    g = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    P = np.asarray(Pi_blk, dtype=np.float64)
+    out = np.zeros((B, Hq, d))
+    for b in range(B):
+        for kv in range(Hkv):
+            sl = (b, kv, slice(0, seq_len))
+            khat = dequantize_mixed(cache["k_codes"][sl], cache["k_norm"][sl], k_bits, k_slot_of_coord_mixed)
+            vhat = dequantize_mixed(cache["v_codes"][sl], cache["v_norm"][sl], v_bits, v_slot_of_coord_mixed)
+            for h in range(kv * g, (kv + 1) * g):
+                qp = P @ q[b, h]
+                est = khat @ qp
+                if S is not None:
+                    S64 = np.asarray(S, np.float64)
+                    pm = 2.0 * unpack_signs(cache["k_signs"][sl]) - 1.0
+                    est = est + np.asarray(cache["k_rnorm"][sl], np.float64) * (SQRT_PI_OVER_2 / S64.shape[0]) * (pm @ (S64 @ qp))
+                out[b, h] = P.T @ softmax_weighted_sum(scale * est, vhat)
+    return out
+
+
+def code_exempt_mixed(u: np.ndarray, bits_O: int, bits_R: int, band: float = 1e-6) -> np.ndarray:
+    """Per coordinate: within `band` of a threshold of its half's codebook."""
+    ex = np.zeros(u.shape, dtype=bool)
+    for g, bits in ((0, bits_O), (1, bits_R)):
+        cols = slice(HALF * g, HALF * (g + 1))
+        ex[..., cols] = code_exempt(u[..., cols], bits, band)
+    return ex
+
+
+# ---------------------------------------------------------------------------
 # Comparison rules for code/sign bytes (exemptions near decision boundaries)
 # ---------------------------------------------------------------------------
 
@@ -390,4 +565,7 @@ __all__ = [
     "k_slot_of_coord", "v_slot_of_coord", "sign_bit_of_row", "pack_codes", "unpack_codes",
     "pack_signs", "unpack_signs", "quantize_cache", "score_estimates", "softmax_weighted_sum",
     "decode_attention", "exact_attention", "code_exempt", "sign_exempt", "CODE_BAND", "SIGN_BAND",
+    "HALF", "quantize_vectors_mixed", "k_slot_of_coord_mixed", "v_slot_of_coord_mixed",
+    "pack_codes_mixed", "unpack_codes_mixed", "quantize_cache_mixed", "dequantize_mixed",
+    "decode_attention_mixed", "code_exempt_mixed",
 ]

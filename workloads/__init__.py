@@ -179,6 +179,30 @@ def make_hadamard_rotation(seed: int, d: int = HEAD_DIM) -> np.ndarray:
     return P.astype(np.float32)
 
 
+def make_block_rotation(seed: int, outlier_channels, d: int = HEAD_DIM) -> np.ndarray:
+    """Rotation of the outlier-aware mixed-precision layout: two independent Haar-random
+    (d/2) x (d/2) matrices (seeds `seed` and `seed` + 1, drawn like make_rotation), the first
+    acting on the outlier channels (ascending) into rows 0 .. d/2 - 1, the second on the other
+    channels into rows d/2 .. d - 1.  fp32."""
+    half = d // 2
+    O = np.sort(np.asarray(outlier_channels, dtype=np.int64))
+    assert O.size == half and np.unique(O).size == half and O.min() >= 0 and O.max() < d
+    R = np.setdiff1d(np.arange(d), O)
+    P = np.zeros((d, d), dtype=np.float32)
+    P[:half][:, O] = make_rotation(seed, half)
+    P[half:][:, R] = make_rotation(seed + 1, half)
+    return P
+
+
+def outlier_channels_for(w: Workload, count: int = HEAD_DIM // 2) -> np.ndarray:
+    """The `count` channels with the largest key scale summed over the kv-heads, from the
+    workload's own per-channel scale draw (a per-layer choice, as the outlier-aware variant keeps
+    one channel split per layer); ascending channel indices."""
+    sc = _channel_scales(w, 0, "cpu").sum(dim=0)
+    order = torch.argsort(sc, descending=True, stable=True)[:count]
+    return np.sort(order.numpy().astype(np.int64))
+
+
 def rotation_for(w: Workload) -> np.ndarray:
     if w.rotation == "hadamard":
         return make_hadamard_rotation(1000 + w.seed, w.head_dim)
@@ -266,6 +290,7 @@ def nbytes_human(n: int) -> str:
 
 __all__ = [
     "HEAD_DIM", "Workload", "CONFIGS", "CONFIG_ORDER", "make_rotation", "make_hadamard_rotation",
+    "make_block_rotation", "outlier_channels_for",
     "splitmix64", "make_qjl_matrix",
     "rotation_for", "qjl_for", "make_kv", "make_queries", "gqa_kv_head", "shard_units",
     "nbytes_human",
