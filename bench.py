@@ -201,6 +201,14 @@ def oracle_sample(w: W.Workload, tokens: int):
     V = W.make_kv(sw, "v").double().numpy()
     q = W.make_queries(sw).double().numpy()
     Pi, S = W.rotation_for(w), W.qjl_for(w)
+    if w.layout == "mixed":
+        oc, kb, vb = W.outlier_channels_for(w), (w.k_bits, w.k_bits - 1), (w.v_bits, w.v_bits - 1)
+        t0 = time.perf_counter()
+        cache = O.quantize_cache_mixed(K, V, Pi, oc, kb, vb, S)
+        t1 = time.perf_counter()
+        O.decode_attention_mixed(q, Pi, S, cache, kb, vb, tokens)
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1, sw
     t0 = time.perf_counter()
     cache = O.quantize_cache(K, V, Pi, w.k_bits, w.v_bits, S)
     t1 = time.perf_counter()
@@ -258,6 +266,7 @@ def workload_config(w: W.Workload, **extra):
     c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.head_dim,
          "context": w.T, "k_bits": w.k_bits, "v_bits": w.v_bits, "qjl_m": w.qjl_m,
          "input_dtype": w.in_dtype, "quantize_chunk": w.chunk, "rotation": w.rotation,
+         "layout": w.layout,
          "l2": f"flushed before every kernel call ({L2_FLUSH_BYTES >> 20} MiB write)"}
     c.update(extra)
     return c
@@ -278,11 +287,14 @@ def run_gpu(args, w):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
 
-    params = tq.Params.create(W.rotation_for(w), W.qjl_for(w), w.k_bits, w.v_bits, device=dev)
+    mixed = w.layout == "mixed"
+    params = tq.Params.create(W.rotation_for(w), W.qjl_for(w), w.k_bits, w.v_bits, device=dev,
+                              outlier_channels=W.outlier_channels_for(w) if mixed else None)
     K = W.make_kv(w, "k", device=dev)
     V = W.make_kv(w, "v", device=dev)
     q = W.make_queries(w, device=dev)
-    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m, device=dev)
+    cache = tq.Cache.allocate(w.B, w.Hkv, w.T, w.k_bits, w.v_bits, w.qjl_m, device=dev,
+                              layout=tq.TQ_LAYOUT_MIXED if mixed else tq.TQ_LAYOUT_PLAIN)
     out = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=dev)
     ws = torch.empty(tq.decode_workspace_size(w.B, w.Hq, cache, w.T), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -461,6 +473,9 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch every op directly in the timed steps")
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
                     help="Pi: dense Haar-random (default) or the structured D1 H D2 H D3 / 128")
+    ap.add_argument("--layout", default="plain", choices=["plain", "mixed"],
+                    help="cache layout: plain, or outlier-aware mixed precision (3.5 bits: the outlier "
+                         "half of the channels at 4 bits, the rest at 3; needs 4-bit keys and values)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--context", type=int, default=None, help="override the workload's context")
     args = ap.parse_args()
@@ -471,6 +486,10 @@ def main():
         w = w.scaled(B=args.batch, T=args.context, name=w.name + "(resized)")
     if args.rotation != w.rotation:
         w = dataclasses.replace(w, rotation=args.rotation)
+    if args.layout != w.layout:
+        if w.k_bits != 4 or w.v_bits != 4:
+            ap.error("--layout mixed needs a workload with 4-bit keys and values")
+        w = dataclasses.replace(w, layout=args.layout)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -31,6 +31,8 @@ TQ_ERR_WORKSPACE = 4
 TQ_ERR_CUDA = 5
 TQ_F32 = 0
 TQ_BF16 = 1
+TQ_LAYOUT_PLAIN = 0
+TQ_LAYOUT_MIXED = 1
 
 # Functions declared in include/tq.h (checked by the test-suite against the header).
 EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codebook",
@@ -38,7 +40,8 @@ EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codeboo
             "tq_quantize_code_fixups", "tq_quantize_exempt_codes", "tq_quantize_exempt_signs",
             "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
             "tq_decode_static_workspace_limit", "tq_sketch_rotation", "tq_build_hadamard_rotation",
-            "tq_decode_step", "tq_decode_device_errors")
+            "tq_decode_step", "tq_decode_device_errors", "tq_reset_device_errors",
+            "tq_debug_quantize_stall")
 
 
 class TqError(RuntimeError):
@@ -53,14 +56,18 @@ class _Cache(ctypes.Structure):
                 ("qjl_m", ctypes.c_int),
                 ("k_codes", ctypes.c_void_p), ("k_signs", ctypes.c_void_p),
                 ("k_norm", ctypes.c_void_p), ("k_rnorm", ctypes.c_void_p),
-                ("v_codes", ctypes.c_void_p), ("v_norm", ctypes.c_void_p)]
+                ("v_codes", ctypes.c_void_p), ("v_norm", ctypes.c_void_p),
+                ("layout", ctypes.c_int)]
 
 
 class _Params(ctypes.Structure):
     _fields_ = [("Pi", ctypes.c_void_p), ("S", ctypes.c_void_p),
                 ("k_centroids", ctypes.c_void_p), ("k_thresholds", ctypes.c_void_p),
                 ("v_centroids", ctypes.c_void_p), ("v_thresholds", ctypes.c_void_p),
-                ("S_Pi", ctypes.c_void_p)]
+                ("S_Pi", ctypes.c_void_p),
+                ("k_centroids_lo", ctypes.c_void_p), ("k_thresholds_lo", ctypes.c_void_p),
+                ("v_centroids_lo", ctypes.c_void_p), ("v_thresholds_lo", ctypes.c_void_p),
+                ("outlier_mask", ctypes.c_uint32 * 4)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -97,6 +104,10 @@ def lib() -> ctypes.CDLL:
     L.tq_quantize_exempt_codes.argtypes = []
     L.tq_quantize_exempt_signs.restype = ctypes.c_longlong
     L.tq_quantize_exempt_signs.argtypes = []
+    L.tq_reset_device_errors.restype = ctypes.c_int
+    L.tq_reset_device_errors.argtypes = []
+    L.tq_debug_quantize_stall.restype = ctypes.c_int
+    L.tq_debug_quantize_stall.argtypes = [ctypes.c_int, ctypes.c_longlong]
     L.tq_decode_device_errors.restype = ctypes.c_int
     L.tq_decode_device_errors.argtypes = []
     L.tq_decode_workspace_size.restype = ctypes.c_size_t
@@ -202,15 +213,32 @@ class Params:
     v_centroids: torch.Tensor
     v_thresholds: torch.Tensor
     S_Pi: Optional[torch.Tensor] = None
+    # mixed layout: codebooks of the non-outlier half (one bit fewer) and the outlier channels
+    k_centroids_lo: Optional[torch.Tensor] = None
+    k_thresholds_lo: Optional[torch.Tensor] = None
+    v_centroids_lo: Optional[torch.Tensor] = None
+    v_thresholds_lo: Optional[torch.Tensor] = None
+    outlier_mask: tuple = (0, 0, 0, 0)
 
     @classmethod
-    def create(cls, Pi, S, k_bits: int, v_bits: int, device="cuda", sketch_rotation=True) -> "Params":
+    def create(cls, Pi, S, k_bits: int, v_bits: int, device="cuda", sketch_rotation=True,
+               outlier_channels=None) -> "Params":
         """Upload the constants; with a sketch, also S Pi in fp64 (tq_sketch_rotation) unless
-        `sketch_rotation` is False."""
+        `sketch_rotation` is False.  With `outlier_channels` (64 channel indices) the constants
+        are those of the mixed layout: Pi must then be the block rotation of those channels."""
         kc, kt, _ = build_codebook(k_bits)
         vc, vt, _ = build_codebook(v_bits)
         f = lambda x: torch.as_tensor(np.ascontiguousarray(x, dtype=np.float32)).to(device)
         p = cls(f(Pi), None if S is None else f(S), f(kc), f(kt), f(vc), f(vt))
+        if outlier_channels is not None:
+            kc2, kt2, _ = build_codebook(k_bits - 1)
+            vc2, vt2, _ = build_codebook(v_bits - 1)
+            p.k_centroids_lo, p.k_thresholds_lo = f(kc2), f(kt2)
+            p.v_centroids_lo, p.v_thresholds_lo = f(vc2), f(vt2)
+            mask = [0, 0, 0, 0]
+            for c in np.asarray(outlier_channels, dtype=np.int64).tolist():
+                mask[c // 32] |= 1 << (c % 32)
+            p.outlier_mask = tuple(mask)
         if p.S is not None and sketch_rotation and p.Pi.is_cuda:
             p.S_Pi = sketch_rotation_product(p.Pi, p.S)
         return p
@@ -218,7 +246,9 @@ class Params:
     def as_c(self) -> _Params:
         return _Params(_ptr(self.Pi), _ptr(self.S), _ptr(self.k_centroids),
                        _ptr(self.k_thresholds), _ptr(self.v_centroids), _ptr(self.v_thresholds),
-                       _ptr(self.S_Pi))
+                       _ptr(self.S_Pi), _ptr(self.k_centroids_lo), _ptr(self.k_thresholds_lo),
+                       _ptr(self.v_centroids_lo), _ptr(self.v_thresholds_lo),
+                       (ctypes.c_uint32 * 4)(*self.outlier_mask))
 
 
 @dataclasses.dataclass
@@ -237,36 +267,47 @@ class Cache:
     k_rnorm: Optional[torch.Tensor]
     v_codes: torch.Tensor
     v_norm: torch.Tensor
+    layout: int = TQ_LAYOUT_PLAIN
+
+    @staticmethod
+    def code_bytes(bits: int, layout: int) -> int:
+        """Bytes of a packed row of 128 codes (mixed layout: halves of bits and bits - 1)."""
+        return 8 * (2 * bits - 1) if layout == TQ_LAYOUT_MIXED else 16 * bits
 
     @classmethod
-    def allocate(cls, B, Hkv, T_cap, k_bits, v_bits, qjl_m=128, device="cuda") -> "Cache":
+    def allocate(cls, B, Hkv, T_cap, k_bits, v_bits, qjl_m=128, device="cuda",
+                 layout=TQ_LAYOUT_PLAIN) -> "Cache":
         u8 = dict(dtype=torch.uint8, device=device)
         f32 = dict(dtype=torch.float32, device=device)
+        nrm = (2,) if layout == TQ_LAYOUT_MIXED else ()
         return cls(B, Hkv, T_cap, k_bits, v_bits, qjl_m,
-                   torch.zeros(B, Hkv, T_cap, 16 * k_bits, **u8),
+                   torch.zeros(B, Hkv, T_cap, cls.code_bytes(k_bits, layout), **u8),
                    torch.zeros(B, Hkv, T_cap, 16, **u8) if qjl_m else None,
-                   torch.zeros(B, Hkv, T_cap, **f32),
+                   torch.zeros(B, Hkv, T_cap, *nrm, **f32),
                    torch.zeros(B, Hkv, T_cap, **f32) if qjl_m else None,
-                   torch.zeros(B, Hkv, T_cap, 16 * v_bits, **u8),
-                   torch.zeros(B, Hkv, T_cap, **f32))
+                   torch.zeros(B, Hkv, T_cap, cls.code_bytes(v_bits, layout), **u8),
+                   torch.zeros(B, Hkv, T_cap, *nrm, **f32), layout)
 
     @classmethod
-    def from_arrays(cls, arrays: dict, k_bits, v_bits, qjl_m, device="cuda") -> "Cache":
+    def from_arrays(cls, arrays: dict, k_bits, v_bits, qjl_m, device="cuda",
+                    layout=TQ_LAYOUT_PLAIN) -> "Cache":
         """Wrap host arrays (k_codes, k_signs, k_norm, k_rnorm, v_codes, v_norm) as a device cache."""
         g = lambda n: None if arrays.get(n) is None else torch.as_tensor(
             np.ascontiguousarray(arrays[n])).to(device)
         kc = g("k_codes")
         B, Hkv, T_cap = kc.shape[:3]
         return cls(B, Hkv, T_cap, k_bits, v_bits, qjl_m, kc, g("k_signs") if qjl_m else None,
-                   g("k_norm"), g("k_rnorm") if qjl_m else None, g("v_codes"), g("v_norm"))
+                   g("k_norm"), g("k_rnorm") if qjl_m else None, g("v_codes"), g("v_norm"), layout)
 
     def as_c(self) -> _Cache:
         return _Cache(self.B, self.Hkv, self.T_cap, 128, self.k_bits, self.v_bits, self.qjl_m,
                       _ptr(self.k_codes), _ptr(self.k_signs), _ptr(self.k_norm),
-                      _ptr(self.k_rnorm), _ptr(self.v_codes), _ptr(self.v_norm))
+                      _ptr(self.k_rnorm), _ptr(self.v_codes), _ptr(self.v_norm), self.layout)
 
     def row_bytes(self) -> int:
-        return 16 * self.k_bits + (20 if self.qjl_m else 0) + 4 + 16 * self.v_bits + 4
+        nb = 8 if self.layout == TQ_LAYOUT_MIXED else 4
+        return (self.code_bytes(self.k_bits, self.layout) + (20 if self.qjl_m else 0) + nb
+                + self.code_bytes(self.v_bits, self.layout) + nb)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -316,6 +357,17 @@ def quantize_exempt_codes() -> int:
 def quantize_exempt_signs() -> int:
     """QJL sketch values so far that were flagged near 0 and lay within 1e-5 of 0 exactly."""
     return int(lib().tq_quantize_exempt_signs())
+
+
+def reset_device_errors() -> None:
+    """Clear the recorded device error bits of both operations; synchronizes."""
+    if lib().tq_reset_device_errors() != 0:
+        raise TqError(TQ_ERR_CUDA, "could not reach the device")
+
+
+def debug_quantize_stall(enable: bool, wait_cycles: int = 0) -> None:
+    """Test hook: make the bf16 quantize kernel's bounded waits run out (see tq.h)."""
+    _check(lib().tq_debug_quantize_stall(1 if enable else 0, int(wait_cycles)))
 
 
 def decode_device_errors() -> int:
@@ -406,7 +458,8 @@ __all__ = [
     "build_codebook", "Params", "Cache", "quantize", "quantize_device_errors",
     "decode_attn_static", "decode_static_workspace_limit",
     "quantize_vector_fixups", "quantize_code_fixups", "quantize_exempt_codes", "quantize_exempt_signs",
-    "decode_workspace_size", "decode_attn", "decode_device_errors",
+    "decode_workspace_size", "decode_attn", "decode_device_errors", "reset_device_errors",
+    "debug_quantize_stall",
     "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
-    "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16",
+    "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16", "TQ_LAYOUT_PLAIN", "TQ_LAYOUT_MIXED",
 ]

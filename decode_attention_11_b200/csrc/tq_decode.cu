@@ -6,19 +6,19 @@
 // second ideas plus the third, QJL, component; tproger.ru "Step 1: PolarQuant", "Step 2: QJL").
 // Softmax and the value sum also run in the rotated basis; one final o = Pi^T o' per head.
 //
-// Kernels (all on the caller's stream; split and merge are programmatic dependent launches):
-//   prep    q' = Pi q and sq = S q' per (batch, query head), fp32, into the workspace: clusters of
-//           eight CTAs, each CTA holding 16 rows of Pi and S for a batch of up to 16 heads.
-//   split   one persistent CTA per SM over an even share of all (unit, token) pairs.  A producer
-//           warp streams 128-token stages of the packed cache into a ring of shared-memory slots
-//           with bulk copies (mbarrier completion); 11 (7 for groups of 5-8 heads) consumer warps take 16 tokens each per
-//           stage: codes become fp16 pairs through a lane-replicated shared-memory table (one
-//           permute + one load per two coordinates), and m16n8k16 tensor-core MMAs compute q'.khat,
-//           the QJL sign dot (sign bits placed in fp16 mantissas by a shift and one logic op, B rows
-//           pre-scaled to match) and P.vhat (P split into fp16 hi + lo).  Online softmax runs in
-//           log2 units; each segment ends with one (max, sum, o'[128]) partial per head.
-//   merge   one CTA per (batch, query head), a programmatic dependent of split: log-sum-exp
-//           merge of the head's partials, then o = Pi^T o'.
+// Kernels (on the caller's stream; merge is a programmatic dependent of split):
+//   split   one persistent CTA per SM over an even share of all (unit, token) pairs.  At the start of
+//           each segment the CTA computes q' = Pi q and sq = S q' of the unit's heads in fp32 (shared
+//           memory).  A producer warp streams stages of the packed cache into a ring of
+//           shared-memory slots with bulk copies (mbarrier completion); 11 (7 for groups of 5-8
+//           heads) consumer warps take 16 tokens each per stage: codes become fp16 pairs through a
+//           lane-replicated shared-memory table (one permute + one load per two coordinates), and
+//           m16n8k16 tensor-core MMAs compute q'.khat, the QJL sign dot (sign bits placed in fp16
+//           mantissas by a shift and one logic op, B rows pre-scaled to match) and P.vhat (P split
+//           into fp16 hi + lo).  Online softmax runs in log2 units; each segment ends with one
+//           (max, sum, o'[128]) partial per head.
+//   merge   one CTA per (batch, query head): log-sum-exp merge of the head's partials, then
+//           o = Pi^T o'.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -62,6 +62,9 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ void cp_async4(void* dst, const void* src, int src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
                "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(dst)), "l"(src));
 }
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __halves2half2(__float2half_rn(lo), __float2half_rn(hi));
@@ -128,90 +131,6 @@ struct VPairs {
   }
 };
 
-// ------------------------------------------------------------------------------------------ prep
-
-// Clusters of eight 128-thread CTAs; cluster k handles query heads hb*k .. hb*k + hb - 1 (flattened
-// over the batch; hb <= 16 is chosen on the host so that there are enough clusters to spread the
-// work) and CTA c of it rows 16c .. 16c+15 of q' = Pi q and of sq = S q', eight threads per row
-// with 16 columns each.  Each CTA loads its rows of Pi and S once (one memory round trip,
-// together with the query vectors) and reuses them for all its heads; the full q' of every head
-// reaches the other CTAs of the cluster through distributed shared memory.  The split kernel is
-// launched as a programmatic dependent of this one and starts its prologue early.
-constexpr int PREP_CLUSTER = 8, PREP_THREADS = 128, PREP_ROWS = D / PREP_CLUSTER, PREP_HB = 16;
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-// Shared-memory float at the same offset as `p` in CTA `rank` of this cluster.
-__device__ __forceinline__ float ld_cluster_f32(const float* p, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
-template <typename QT>
-__global__ void __cluster_dims__(PREP_CLUSTER, 1, 1) __launch_bounds__(PREP_THREADS)
-    prep_kernel(const QT* __restrict__ q, int BH, int hb, const float* __restrict__ Pi, const float* __restrict__ S,
-                int qjl, float* __restrict__ qrot, float* __restrict__ sq) {
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  __shared__ __align__(16) float qs[PREP_HB][D];           // query vectors, then q' of the cluster
-  __shared__ __align__(16) float qpart[PREP_HB][PREP_ROWS];  // this CTA's rows of q'
-  const int tid = threadIdx.x;
-  const uint32_t c = blockIdx.x % PREP_CLUSTER;  // rank in the cluster (clusters are consecutive CTAs)
-  const int h0 = (int)(blockIdx.x / PREP_CLUSTER) * hb;
-  const int nhb = min(hb, BH - h0);
-  const int rl = tid >> 3, part = tid & 7;
-  const int row = PREP_ROWS * (int)c + rl;
-  float4 p[4], s4[4];
-  const float4* pr = reinterpret_cast<const float4*>(Pi + row * D + 16 * part);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = pr[i];
-  if (qjl) {
-    const float4* sr = reinterpret_cast<const float4*>(S + row * D + 16 * part);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s4[i] = sr[i];
-  }
-  for (int h = 0; h < nhb; ++h) {
-    if constexpr (sizeof(QT) == 4) qs[h][tid] = (float)q[(int64_t)(h0 + h) * D + tid];
-    else qs[h][tid] = __bfloat162float(q[(int64_t)(h0 + h) * D + tid]);
-  }
-  __syncthreads();
-  auto dot16 = [&](const float4 (&m)[4], const float* vec) {
-    const float4* v4 = reinterpret_cast<const float4*>(vec + 16 * part);
-    float acc = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 x = v4[i];
-      acc = fmaf(m[i].x, x.x, acc);
-      acc = fmaf(m[i].y, x.y, acc);
-      acc = fmaf(m[i].z, x.z, acc);
-      acc = fmaf(m[i].w, x.w, acc);
-    }
-    acc += __shfl_xor_sync(FULL, acc, 1);
-    acc += __shfl_xor_sync(FULL, acc, 2);
-    acc += __shfl_xor_sync(FULL, acc, 4);
-    return acc;
-  };
-  for (int h = 0; h < nhb; ++h) {
-    const float v = dot16(p, qs[h]);
-    if (part == 0) {
-      qpart[h][rl] = v;
-      qrot[(int64_t)(h0 + h) * D + row] = v;
-    }
-  }
-  if (!qjl) return;  // uniform over the cluster: no CTA waits at the barriers below
-  cluster_sync_all();
-  for (int h = 0; h < nhb; ++h)
-    qs[h][tid] = ld_cluster_f32(&qpart[h][tid % PREP_ROWS], (uint32_t)(tid / PREP_ROWS));
-  cluster_sync_all();  // every remote read is done before any CTA of the cluster exits
-  for (int h = 0; h < nhb; ++h) {
-    const float w = dot16(s4, qs[h]);
-    if (part == 0) sq[(int64_t)(h0 + h) * D + row] = w;
-  }
-}
-
 // ------------------------------------------------------------------------------------------ split
 //
 // Persistent split-K kernel.  The B * Hkv * head_groups (batch, kv-head, head group) units, each
@@ -259,33 +178,48 @@ struct DArgs {
   const float* v_norm;
   const float* kc;
   const float* vc;
-  const float* qrot;
-  const float* sq;
+  const float* kc2;  // mixed layout: codebooks of the non-outlier half (3 bits)
+  const float* vc2;
+  const void* q;    // [B, Hq, 128] fp32 or bf16 (q_bf16)
+  int q_bf16;
+  const float* Pi;  // [128 x 128]
+  const float* S;   // [128 x 128] (QJL)
   float* part;
 };
 
 __device__ unsigned int g_decode_error;  // bit 0: a wait timed out; bit 1: shared memory too small
 
-template <int KB, int VB, bool QJL, int NB>
+// MX: the outlier-aware mixed layout (TQ_LAYOUT_MIXED, KB = VB = 4): rows of 56 bytes (a 4-bit
+// outlier half, then a 3-bit half) and two norms per token; the 4-bit halves use the packed pair
+// table, the 3-bit halves two more 64-entry tables.
+template <int KB, int VB, bool QJL, int NB, bool MX = false>
 struct Layout {
   static constexpr int NW = Shape<NB>::NW, ST = Shape<NB>::ST, HGN = 4 * NB;
-  static constexpr int K_ROW = 16 * KB;
-  static constexpr int V_ROW = 16 * VB;
+  static constexpr int K_ROW = MX ? 8 * (2 * KB - 1) : 16 * KB;
+  static constexpr int V_ROW = MX ? 8 * (2 * VB - 1) : 16 * VB;
+  static constexpr int NORM = MX ? 8 : 4;  // norm bytes per token
   static constexpr int OFF_KC = 0;
   static constexpr int OFF_SG = OFF_KC + ST * K_ROW;
   static constexpr int OFF_VC = OFF_SG + (QJL ? ST * 16 : 0);
   static constexpr int OFF_NK = OFF_VC + ST * V_ROW;
-  static constexpr int OFF_RN = OFF_NK + ST * 4;
+  static constexpr int OFF_RN = OFF_NK + ST * NORM;
   static constexpr int OFF_NV = OFF_RN + (QJL ? ST * 4 : 0);
-  static constexpr int STAGE_BYTES = (OFF_NV + ST * 4 + 127) / 128 * 128;
-  static constexpr int TX_PER_TOKEN = K_ROW + (QJL ? 16 : 0) + V_ROW;  // bulk-copied bytes
+  static constexpr int STAGE_BYTES = (OFF_NV + ST * NORM + 127) / 128 * 128;
+  // bulk-copied bytes (mixed rows of 56 bytes go through 8-byte cp.async instead)
+  static constexpr int TX_PER_TOKEN = (QJL ? 16 : 0) + (MX ? 0 : K_ROW + V_ROW);
   static constexpr bool kPacked = KB == 4 && VB == 4;
   static constexpr int K_TBL = kPacked ? 0 : (1 << (2 * KB)) * 128;
   static constexpr int V_TBL = kPacked ? 0 : (1 << (2 * VB)) * 128;
   static constexpr int TBL_BYTES = kPacked ? 65536 : K_TBL + V_TBL;
+  static constexpr int TBL2_BYTES = MX ? 2 * 64 * 128 : 0;  // 3-bit K and V pair tables
   // per-warp (max, sum) and o' of the 4 NB heads, for the merge of the warps at a segment's end
-  static constexpr int MERGE_BYTES = 4 * (NW * HGN * 2 + NW * HGN * D);
-  static_assert(STAGE_BYTES % 16 == 0 && K_ROW % 16 == 0 && V_ROW % 16 == 0, "bulk-copy granularity");
+  static constexpr int MERGE_BYTES_W = 4 * (NW * HGN * 2 + NW * HGN * D);
+  static constexpr int PREP_BYTES = 4 * 3 * HGN * D;  // query prep at a segment's start
+  static constexpr int MERGE_BYTES = MERGE_BYTES_W > PREP_BYTES ? MERGE_BYTES_W : PREP_BYTES;
+  static_assert(STAGE_BYTES % 16 == 0 && OFF_SG % 16 == 0 && OFF_VC % 16 == 0 && OFF_NK % 16 == 0,
+                "bulk-copy granularity");
+  static_assert(MX || (K_ROW % 16 == 0 && V_ROW % 16 == 0), "bulk-copy granularity");
+  static_assert(!MX || kPacked, "mixed layout: 4-bit outlier halves");
 };
 
 // Control block at the end of the dynamic shared memory.
@@ -294,6 +228,7 @@ struct Ctrl {
   uint64_t empty[NS_MAX];
   uint32_t stage_off[NS_MAX];  // byte offsets of the ring slots from the start of dynamic smem
   uint32_t tbl_addr;           // shared-window address of the pair tables
+  uint32_t tbl2_addr;          // mixed layout: the 3-bit pair tables
   uint32_t merge_off;
   int ns;
   unsigned int err;
@@ -426,6 +361,9 @@ template <int KB, int VB>
 struct PairLut {
   static constexpr bool kPacked = KB == 4 && VB == 4;
   uint32_t rk, rv;
+  uint32_t rk2, rv2;  // mixed layout: the 3-bit tables of the non-outlier half
+  __device__ __forceinline__ uint32_t k2(uint32_t e) const { return lds32((e << 7) + rk2); }
+  __device__ __forceinline__ uint32_t v2(uint32_t e) const { return lds32((e << 7) + rv2); }
   __device__ __forceinline__ uint32_t k(uint32_t e) const { return lds32((e << 7) + rk); }
   __device__ __forceinline__ uint32_t v(uint32_t e) const { return lds32((e << 7) + rv); }
   template <int Bt>
@@ -450,9 +388,9 @@ __device__ __forceinline__ uint32_t v_pair(const PairLut<KB, VB>& L, const VPair
 // Shared-memory plan, computed by one thread: the pair tables (at a 64 KB boundary for the packed
 // tables), the warp-merge area and as many ring slots as fit around them.  ns = 0 when the slots
 // do not fit (never with the 227 KB of an sm_100 CTA).
-template <int KB, int VB, bool QJL, int NB>
+template <int KB, int VB, bool QJL, int NB, bool MX>
 __device__ void plan_smem(unsigned char* smem, int dyn, Ctrl& c) {
-  using Lay = Layout<KB, VB, QJL, NB>;
+  using Lay = Layout<KB, VB, QJL, NB, MX>;
   const uint32_t base = smem_u32(smem);
   const uint32_t end = base + (uint32_t)dyn - CTRL_BYTES;
   const uint32_t tbl = Lay::kPacked ? ((base + 0xFFFFu) & ~0xFFFFu) : base;
@@ -482,14 +420,21 @@ __device__ void plan_smem(unsigned char* smem, int dyn, Ctrl& c) {
     return;
   }
   c.merge_off = off;
+  if (Lay::TBL2_BYTES) {
+    if (!take(Lay::TBL2_BYTES, off)) {
+      c.ns = 0;
+      return;
+    }
+    c.tbl2_addr = base + off;
+  }
   int ns = 0;
   while (ns < NS_MAX && take(Lay::STAGE_BYTES, off)) c.stage_off[ns++] = off;
   c.ns = ns >= 2 ? ns : 0;
 }
 
-template <int KB, int VB, bool QJL, int NB>
+template <int KB, int VB, bool QJL, int NB, bool MX>
 __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __grid_constant__ DArgs a) {
-  using Lay = Layout<KB, VB, QJL, NB>;
+  using Lay = Layout<KB, VB, QJL, NB, MX>;
   using Lut = PairLut<KB, VB>;
   constexpr int NW = Shape<NB>::NW, ST = Shape<NB>::ST, HGN = 4 * NB;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -500,7 +445,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
   const int64_t L = a.seq_len;
 
   if (tid == 0) {
-    plan_smem<KB, VB, QJL, NB>(smem, a.dyn_smem, ctl);
+    plan_smem<KB, VB, QJL, NB, MX>(smem, a.dyn_smem, ctl);
     ctl.err = 0;
     for (int i = 0; i < ctl.ns; ++i) {
       mbar_init_(&ctl.full[i], 1 + 32);  // producer's expect_tx + the noinc arrivals of its 32 lanes
@@ -539,14 +484,30 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         unsigned char* st = smem + ctl.stage_off[cur];
         if (lane == 0) {
           mbar_expect_tx_(&ctl.full[cur], (uint32_t)(ntok * Lay::TX_PER_TOKEN));
-          bulk_g2s(st + Lay::OFF_KC, a.k_codes + row0 * Lay::K_ROW, ntok * Lay::K_ROW, &ctl.full[cur]);
+          if constexpr (!MX)
+            bulk_g2s(st + Lay::OFF_KC, a.k_codes + row0 * Lay::K_ROW, ntok * Lay::K_ROW, &ctl.full[cur]);
           if constexpr (QJL) bulk_g2s(st + Lay::OFF_SG, a.k_signs + row0 * 16, ntok * 16, &ctl.full[cur]);
-          bulk_g2s(st + Lay::OFF_VC, a.v_codes + row0 * Lay::V_ROW, ntok * Lay::V_ROW, &ctl.full[cur]);
+          if constexpr (!MX)
+            bulk_g2s(st + Lay::OFF_VC, a.v_codes + row0 * Lay::V_ROW, ntok * Lay::V_ROW, &ctl.full[cur]);
         }
-        for (int i = lane; i < ntok; i += 32) {
-          cp_async4(st + Lay::OFF_NK + 4 * i, a.k_norm + row0 + i, 4);
-          if constexpr (QJL) cp_async4(st + Lay::OFF_RN + 4 * i, a.k_rnorm + row0 + i, 4);
-          cp_async4(st + Lay::OFF_NV + 4 * i, a.v_norm + row0 + i, 4);
+        if constexpr (MX) {  // 56-byte rows: seven 8-byte copies per row (every row is 8-byte aligned)
+          const uint8_t* kg = a.k_codes + row0 * Lay::K_ROW;
+          const uint8_t* vg = a.v_codes + row0 * Lay::V_ROW;
+          for (int i = lane; i < ntok * (Lay::K_ROW / 8); i += 32) {
+            cp_async8(st + Lay::OFF_KC + 8 * i, kg + 8 * i);
+            cp_async8(st + Lay::OFF_VC + 8 * i, vg + 8 * i);
+          }
+          for (int i = lane; i < ntok; i += 32) {
+            cp_async8(st + Lay::OFF_NK + 8 * i, a.k_norm + 2 * (row0 + i));
+            if constexpr (QJL) cp_async4(st + Lay::OFF_RN + 4 * i, a.k_rnorm + row0 + i, 4);
+            cp_async8(st + Lay::OFF_NV + 8 * i, a.v_norm + 2 * (row0 + i));
+          }
+        } else {
+          for (int i = lane; i < ntok; i += 32) {
+            cp_async4(st + Lay::OFF_NK + 4 * i, a.k_norm + row0 + i, 4);
+            if constexpr (QJL) cp_async4(st + Lay::OFF_RN + 4 * i, a.k_rnorm + row0 + i, 4);
+            cp_async4(st + Lay::OFF_NV + 4 * i, a.v_norm + row0 + i, 4);
+          }
         }
         cp_async_arrive_noinc(&ctl.full[cur]);
         issued = it + 1;
@@ -578,6 +539,17 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       }
       lut.rk = tbl | (4u * lane);
       lut.rv = tbl | 128u | (4u * lane);
+      if constexpr (MX) {  // 3-bit pair tables of the other half: K at +0, V at +8 KB
+        unsigned char* tp2 = smem + (ctl.tbl2_addr - smem_u32(smem));
+        for (int i = tid; i < 2 * 64 * 8; i += NW * 32) {  // (table, entry, group of four lanes)
+          const int isv = i >> 9, e = (i >> 3) & 63, q4 = i & 7;
+          const float* cb = isv ? a.vc2 : a.kc2;
+          const uint32_t v = pack_half2(__ldg(cb + (e & 7)), __ldg(cb + (e >> 3)));
+          *reinterpret_cast<uint4*>(tp2 + isv * 8192 + e * 128 + 16 * q4) = make_uint4(v, v, v, v);
+        }
+        lut.rk2 = ctl.tbl2_addr + 4u * lane;
+        lut.rv2 = ctl.tbl2_addr + 8192u + 4u * lane;
+      }
     } else {
       for (int i = tid; i < (Lay::K_TBL + Lay::V_TBL) / 16; i += NW * 32) {
         const bool isv = i >= Lay::K_TBL / 16;
@@ -593,8 +565,6 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
     }
   }
   consumers_sync<NW>();
-  // The rotated queries come from the prep kernel; everything above reads only the cache.
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   // the merge kernel may launch now; its CTAs wait for this grid to finish before reading
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
@@ -615,6 +585,46 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
     const int h0 = kvh * a.g + hg * HG;
     const int nh = min(HG, a.g - hg * HG);
 
+    // ---- query prep for this unit's heads (the merge area is free at a segment's start):
+    // q' = Pi q, then sq = S q', fp32, into shared memory.  Thread (i, half) sums 64 of the 128
+    // products of output row i for every head, reading its half-row of Pi (S) once.
+    float* qsm = mrg;             // [HGN][D] query vectors
+    float* qpm = qsm + HGN * D;   // [HGN][D] q'
+    float* sqm = qpm + HGN * D;   // [HGN][D] S q'
+    for (int i = tid; i < nh * D; i += NW * 32) {
+      const int64_t qi = ((int64_t)b * a.Hq + h0 + i / D) * D + i % D;
+      qsm[i] = a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[qi])
+                        : reinterpret_cast<const float*>(a.q)[qi];
+    }
+    consumers_sync<NW>();
+    for (int pass = 0; pass < (QJL ? 2 : 1); ++pass) {
+      const float* Mtx = pass ? a.S : a.Pi;
+      const float* vin = pass ? qpm : qsm;
+      float* vout = pass ? sqm : qpm;
+      for (int task = tid; task < 2 * D; task += NW * 32) {  // 32 NW is a multiple of 32: pairs stay in a warp
+        const int row = task >> 1, half = task & 1;
+        const float4* mr = reinterpret_cast<const float4*>(Mtx + row * D + 64 * half);
+        float4 m4[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) m4[k] = __ldg(mr + k);
+        for (int hh = 0; hh < nh; ++hh) {
+          const float4* v4 = reinterpret_cast<const float4*>(vin + hh * D + 64 * half);
+          float acc = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float4 x = v4[k];
+            acc = fmaf(m4[k].x, x.x, acc);
+            acc = fmaf(m4[k].y, x.y, acc);
+            acc = fmaf(m4[k].z, x.z, acc);
+            acc = fmaf(m4[k].w, x.w, acc);
+          }
+          acc += __shfl_xor_sync(FULL, acc, 1);
+          if (half == 0) vout[hh * D + row] = acc;
+        }
+      }
+      consumers_sync<NW>();
+    }
+
     // ---- B operands of this unit's heads.  Column gq of n-block nb = head 4 nb + gq / 2, part
     // gq % 2 (0: fp16 hi, 1: fp16 lo); k-step kk holds k = 16kk + 2t, +1 (reg 0), +8, +9 (reg 1).
     // Each head is scaled by a power of two 2^-e so that q' and 16 S q' stay far inside fp16 range.
@@ -625,8 +635,8 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       const int hh = 4 * nb + (gq >> 1);
       const bool live = hh < nh;
       const bool lo = gq & 1;
-      const float* qp = a.qrot + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
-      const float* sp = a.sq + ((int64_t)b * a.Hq + h0 + (live ? hh : 0)) * D;
+      const float* qp = qpm + (live ? hh : 0) * D;
+      const float* sp = sqm + (live ? hh : 0) * D;
       float qv[8][2][2], sv[8][2][2];
       float mx = 0.0f;
 #pragma unroll
@@ -682,6 +692,8 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       Kh[nb] = -ch - 0.5f * sh;  // sum_l sq_l (2 b_l - 1) = 2 (D_hi + D_lo + Kh)
     }
 
+    consumers_sync<NW>();  // q' / S q' are read; the merge at this segment's end reuses the area
+
     // Output accumulators: n-block nb, dim block db: (dim 16db + gq, head 4nb + t) hi/lo in [0]/[1],
     // (dim 16db + 8 + gq) in [2]/[3].
     float oacc[NB][8][4];
@@ -710,7 +722,38 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
           for (int e = 0; e < 4; ++e) kacc[nb][e] = qacc[nb][e] = kacc2[nb][e] = qacc2[nb][e] = 0.0f;
-        {
+        if constexpr (MX) {
+          // outlier half: 16 4-bit codes at byte 8t (k-steps 0..3, the packed table, accumulated in
+          // kacc); other half: 16 3-bit codes at byte 32 + 6t (k-steps 4..7, kacc2)
+          const unsigned char* k0 = stage + Lay::OFF_KC + r0 * Lay::K_ROW;
+          const unsigned char* k1 = stage + Lay::OFF_KC + r1 * Lay::K_ROW;
+          const uint2 o0 = lds64(k0 + 8 * t), o1 = lds64(k1 + 8 * t);
+          const uint32_t c0[2] = {o0.x, o0.y}, c1[2] = {o1.x, o1.y};
+          const int rb = 32 + 6 * t, ra = rb & ~3, rsh = 8 * (rb & 3);  // (rb & 3) is 0 or 2
+          const uint64_t g0 = ((uint64_t)lds32(smem_u32(k0 + ra + 4)) << 32 | lds32(smem_u32(k0 + ra))) >> rsh;
+          const uint64_t g1 = ((uint64_t)lds32(smem_u32(k1 + ra + 4)) << 32 | lds32(smem_u32(k1 + ra))) >> rsh;
+#define TQ_KSTEP_O(KK)                                                                       \
+          {                                                                                  \
+            const uint32_t A[4] = {lut.template k_byte<(2 * (KK)) & 3>(c0[(2 * (KK)) >> 2]),   \
+                                   lut.template k_byte<(2 * (KK)) & 3>(c1[(2 * (KK)) >> 2]),   \
+                                   lut.template k_byte<(2 * (KK) + 1) & 3>(c0[(2 * (KK) + 1) >> 2]), \
+                                   lut.template k_byte<(2 * (KK) + 1) & 3>(c1[(2 * (KK) + 1) >> 2])}; \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                \
+                mma16816(kacc[nb], A, bq[nb][KK][0], bq[nb][KK][1]);                           \
+          }
+#define TQ_KSTEP_R(KK)                                                                       \
+          {                                                                                  \
+            const uint32_t A[4] = {lut.k2((uint32_t)(g0 >> (12 * ((KK) - 4))) & 63u),          \
+                                   lut.k2((uint32_t)(g1 >> (12 * ((KK) - 4))) & 63u),          \
+                                   lut.k2((uint32_t)(g0 >> (12 * ((KK) - 4) + 6)) & 63u),      \
+                                   lut.k2((uint32_t)(g1 >> (12 * ((KK) - 4) + 6)) & 63u)};     \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                \
+                mma16816(kacc2[nb], A, bq[nb][KK][0], bq[nb][KK][1]);                          \
+          }
+          TQ_KSTEP_O(0) TQ_KSTEP_O(1) TQ_KSTEP_O(2) TQ_KSTEP_O(3) TQ_KSTEP_R(4) TQ_KSTEP_R(5) TQ_KSTEP_R(6) TQ_KSTEP_R(7)
+#undef TQ_KSTEP_O
+#undef TQ_KSTEP_R
+        } else {
           uint32_t c0[KB], c1[KB];
           const unsigned char* k0 = stage + Lay::OFF_KC + r0 * Lay::K_ROW + 4 * KB * t;
           const unsigned char* k1 = stage + Lay::OFF_KC + r1 * Lay::K_ROW + 4 * KB * t;
@@ -756,8 +799,11 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
 
         // ---- online softmax (log2 units) per head 4nb + t over this warp's 16 tokens ----
         const bool v0ok = gq < nvalid, v1ok = gq + 8 < nvalid;
-        const float nk0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r0);
-        const float nk1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + 4 * r1);
+        // (mixed layout: two norms per token, the outlier half's first)
+        const float nk0 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + Lay::NORM * r0);
+        const float nk1 = *reinterpret_cast<const float*>(stage + Lay::OFF_NK + Lay::NORM * r1);
+        const float nk0b = MX ? *reinterpret_cast<const float*>(stage + Lay::OFF_NK + Lay::NORM * r0 + 4) : 0.0f;
+        const float nk1b = MX ? *reinterpret_cast<const float*>(stage + Lay::OFF_NK + Lay::NORM * r1 + 4) : 0.0f;
         float rn0 = 0.0f, rn1 = 0.0f;
         if constexpr (QJL) {
           rn0 = *reinterpret_cast<const float*>(stage + Lay::OFF_RN + 4 * r0);
@@ -765,13 +811,23 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         }
         // rows past the segment's end hold stale or uninitialised words: their weight is 0 and
         // their value scale too, so nothing of them reaches the sums
-        const float nv0 = v0ok ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r0) * 0.08838834764831845f : 0.0f;
-        const float nv1 = v1ok ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + 4 * r1) * 0.08838834764831845f : 0.0f;
-        uint32_t bp[NB][2];
+        // value scale ||v|| / sqrt(128) (mixed layout: ||v_g|| / 8 of each half)
+        constexpr float VSC = MX ? 0.125f : 0.08838834764831845f;
+        const float nv0 = v0ok ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + Lay::NORM * r0) * VSC : 0.0f;
+        const float nv1 = v1ok ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + Lay::NORM * r1) * VSC : 0.0f;
+        const float nv0b = (MX && v0ok) ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + Lay::NORM * r0 + 4) * VSC : 0.0f;
+        const float nv1b = (MX && v1ok) ? *reinterpret_cast<const float*>(stage + Lay::OFF_NV + Lay::NORM * r1 + 4) * VSC : 0.0f;
+        uint32_t bp[NB][2], bp2[NB][2];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          float s0v = ((kacc[nb][0] + kacc2[nb][0]) + (kacc[nb][1] + kacc2[nb][1])) * (nk0 * fK[nb]);
-          float s1v = ((kacc[nb][2] + kacc2[nb][2]) + (kacc[nb][3] + kacc2[nb][3])) * (nk1 * fK[nb]);
+          float s0v, s1v;
+          if constexpr (MX) {  // the halves carry their own norms
+            s0v = fmaf(kacc2[nb][0] + kacc2[nb][1], nk0b * fK[nb], (kacc[nb][0] + kacc[nb][1]) * (nk0 * fK[nb]));
+            s1v = fmaf(kacc2[nb][2] + kacc2[nb][3], nk1b * fK[nb], (kacc[nb][2] + kacc[nb][3]) * (nk1 * fK[nb]));
+          } else {
+            s0v = ((kacc[nb][0] + kacc2[nb][0]) + (kacc[nb][1] + kacc2[nb][1])) * (nk0 * fK[nb]);
+            s1v = ((kacc[nb][2] + kacc2[nb][2]) + (kacc[nb][3] + kacc2[nb][3])) * (nk1 * fK[nb]);
+          }
           if constexpr (QJL) {
             s0v = fmaf(((qacc[nb][0] + qacc2[nb][0]) + (qacc[nb][1] + qacc2[nb][1])) + Kh[nb], rn0 * fQ[nb], s0v);
             s1v = fmaf(((qacc[nb][2] + qacc2[nb][2]) + (qacc[nb][3] + qacc2[nb][3])) + Kh[nb], rn1 * fQ[nb], s1v);
@@ -800,10 +856,52 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
           // P~ = p nV / sqrt(d) as fp16 hi + lo: row token, columns (head t, hi) and (head t, lo)
           bp[nb][0] = movmatrix_trans(hilo_half2(p0 * nv0));  // tokens 2t, 2t+1 of column gq
           bp[nb][1] = movmatrix_trans(hilo_half2(p1 * nv1));  // tokens 2t+8, 2t+9
+          if constexpr (MX) {  // the other half's values: their own scale
+            bp2[nb][0] = movmatrix_trans(hilo_half2(p0 * nv0b));
+            bp2[nb][1] = movmatrix_trans(hilo_half2(p1 * nv1b));
+          }
         }
 
         // ---- O'^T += Vhat^T P~: dim blocks of 16; A holds token pairs (2t,2t+1), (2t+8,2t+9) ----
-        {
+        if constexpr (MX) {
+          // lane group gq: outlier half, 8 4-bit codes at byte 4gq (dim blocks 0..3); other half,
+          // 8 3-bit codes at byte 32 + 3gq (dim blocks 4..7)
+          const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
+          const int rb = 32 + 3 * gq, ra = rb & ~3, rsh = 8 * (rb & 3);
+          uint32_t vo[4], vr[4];
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const unsigned char* row = vbase + (2 * t + (k4 & 1) + 8 * (k4 >> 1)) * Lay::V_ROW;
+            vo[k4] = lds32(smem_u32(row + 4 * gq));
+            vr[k4] = (uint32_t)((((uint64_t)lds32(smem_u32(row + ra + 4)) << 32) | lds32(smem_u32(row + ra))) >> rsh);
+          }
+          // token pairs (2t, 2t+1) and (2t+8, 2t+9): codes of both tokens interleaved per byte
+          const uint32_t w01e = (vo[0] & 0x0F0F0F0Fu) | ((vo[1] << 4) & 0xF0F0F0F0u);
+          const uint32_t w01o = ((vo[0] >> 4) & 0x0F0F0F0Fu) | (vo[1] & 0xF0F0F0F0u);
+          const uint32_t w89e = (vo[2] & 0x0F0F0F0Fu) | ((vo[3] << 4) & 0xF0F0F0F0u);
+          const uint32_t w89o = ((vo[2] >> 4) & 0x0F0F0F0Fu) | (vo[3] & 0xF0F0F0F0u);
+#define TQ_VSTEP_O(DB)                                                                        \
+          {                                                                                   \
+            const uint32_t A[4] = {lut.template v_byte<DB>(w01e), lut.template v_byte<DB>(w01o), \
+                                   lut.template v_byte<DB>(w89e), lut.template v_byte<DB>(w89o)}; \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                 \
+                mma16816(oacc[nb][DB], A, bp[nb][0], bp[nb][1]);                               \
+          }
+#define TQ_VPAIR_R(X, Y, NU) (((X >> (3 * (NU))) & 7u) | (((Y >> (3 * (NU))) & 7u) << 3))
+#define TQ_VSTEP_R(DB)                                                                        \
+          {                                                                                   \
+            const uint32_t A[4] = {lut.v2(TQ_VPAIR_R(vr[0], vr[1], 2 * ((DB) - 4))),           \
+                                   lut.v2(TQ_VPAIR_R(vr[0], vr[1], 2 * ((DB) - 4) + 1)),       \
+                                   lut.v2(TQ_VPAIR_R(vr[2], vr[3], 2 * ((DB) - 4))),           \
+                                   lut.v2(TQ_VPAIR_R(vr[2], vr[3], 2 * ((DB) - 4) + 1))};      \
+            _Pragma("unroll") for (int nb = 0; nb < NB; ++nb)                                 \
+                mma16816(oacc[nb][DB], A, bp2[nb][0], bp2[nb][1]);                             \
+          }
+          TQ_VSTEP_O(0) TQ_VSTEP_O(1) TQ_VSTEP_O(2) TQ_VSTEP_O(3) TQ_VSTEP_R(4) TQ_VSTEP_R(5) TQ_VSTEP_R(6) TQ_VSTEP_R(7)
+#undef TQ_VSTEP_O
+#undef TQ_VSTEP_R
+#undef TQ_VPAIR_R
+        } else {
           const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
           uint64_t cv0, cv1, cv2, cv3;
           if constexpr (VB == 4) {
@@ -900,29 +998,10 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
 // One 512-thread CTA per (batch, query head), a programmatic dependent of the split kernel: it
 // waits for the split grid, merges the head's partials (one per CTA that streamed part of the
 // head's unit) by log-sum-exp and writes o = Pi^T o'.  Thread (d, q), d = tid % 128 and
-// q = tid / 128, sums the partials s = q (mod 4) of dimension d; the un-rotation gives thread
-// (i, q) the rows 32q .. 32q + 31 of Pi.  Each phase issues its loads at once (one L2 round trip).
+// q = tid / 128, takes the partials s = q (mod 4) of dimension d with a running maximum, so all of
+// its loads issue at once (one L2 round trip); the four quarters are then combined per dimension.
+// The un-rotation gives thread (i, q) the rows 32q .. 32q + 31 of Pi, loaded before the wait.
 constexpr int MERGE_THREADS = 4 * D;
-
-__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float x = __shfl_xor_sync(FULL, v, o);
-    v = is_max ? fmaxf(v, x) : v + x;
-  }
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  v = red[lane < MERGE_THREADS / 32 ? lane : 0];
-  if (lane >= MERGE_THREADS / 32) v = is_max ? -INFINITY : 0.0f;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {  // every lane ends with the full result
-    const float x = __shfl_xor_sync(FULL, v, o);
-    v = is_max ? fmaxf(v, x) : v + x;
-  }
-  __syncthreads();  // red is reused by the next reduction
-  return v;
-}
 
 // (The partials are written by the still-running split grid: they are read with ld.global.cg,
 // through L2 only, never through the non-coherent read-only path.)
@@ -930,8 +1009,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
                                                               float* __restrict__ out, int Hq, int g, int Hkv,
                                                               int hgroups, int64_t seq_len, int64_t ntot, int ctas,
                                                               int pmax) {
-  extern __shared__ __align__(16) float msm[];  // [S] weights, [S] sums, [4][D] partial o', [D] o', [4][D]
-  __shared__ float red[32];
+  __shared__ float mq[4][D], lq[4][D], oq[4][D], ob[D];
   const int tid = threadIdx.x, d = tid % D, q = tid / D;
   const int64_t bh = blockIdx.x;
   if (seq_len == 0) {  // empty context: the output is zero (no split grid ran)
@@ -948,49 +1026,41 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
   const int first = part_cta_of(ntot, ctas, u * seq_len);
   const int S = part_cta_of(ntot, ctas, u * seq_len + seq_len - 1) - first + 1;
   const float* p = part + bh * pmax * PART;
-  float* wts = msm;
-  float* ls = wts + pmax;
-  float* osum = ls + ((pmax + 3) & ~3);
-  float* ob = osum + 4 * D;
-  float* rsum = ob + D;
-  // phase 1: (max, sum) of every partial
-  float m = -INFINITY;
-  for (int s2 = tid; s2 < S; s2 += MERGE_THREADS) {
+  float M = -1e30f, Ls = 0.0f, O = 0.0f;
+#pragma unroll 4
+  for (int s2 = q; s2 < S; s2 += 4) {
     const float2 ml = __ldcg(reinterpret_cast<const float2*>(p + (int64_t)s2 * PART));
-    wts[s2] = ml.x;
-    ls[s2] = ml.y;
-    m = fmaxf(m, ml.x);
+    const float o = __ldcg(p + (int64_t)s2 * PART + 4 + d);
+    const float Mn = fmaxf(M, ml.x);
+    const float a0 = ex2(M - Mn), a1 = ex2(ml.x - Mn);
+    Ls = fmaf(a1, ml.y, Ls * a0);
+    O = fmaf(a1, o, O * a0);
+    M = Mn;
   }
-  const float M = block_reduce(m, red, true);
-  // phase 2: weights 2^(m_s - M) and L = sum_s w_s l_s
-  float l = 0.0f;
-  for (int s2 = tid; s2 < S; s2 += MERGE_THREADS) {
-    const float f = ex2(wts[s2] - M);
-    wts[s2] = f;
-    l = fmaf(f, ls[s2], l);
-  }
-  const float Lsum = block_reduce(l, red, false);  // also makes the weights visible
-  // phase 3: thread (d, q) sums partials q, q + 4, ...
-  float acc = 0.0f;
-#pragma unroll 16
-  for (int s2 = q; s2 < S; s2 += 4) acc = fmaf(wts[s2], __ldcg(p + (int64_t)s2 * PART + 4 + d), acc);
-  osum[q * D + d] = acc;
+  mq[q][d] = M;
+  lq[q][d] = Ls;
+  oq[q][d] = O;
   __syncthreads();
   if (tid < D) {
-    const float o = osum[d] + osum[D + d] + osum[2 * D + d] + osum[3 * D + d];
-    ob[d] = Lsum > 0.0f ? o / Lsum : 0.0f;
+    const float Mx = fmaxf(fmaxf(mq[0][d], mq[1][d]), fmaxf(mq[2][d], mq[3][d]));
+    float Lt = 0.0f, Ot = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float w = ex2(mq[k][d] - Mx);
+      Lt = fmaf(w, lq[k][d], Lt);
+      Ot = fmaf(w, oq[k][d], Ot);
+    }
+    ob[d] = Lt > 0.0f ? Ot / Lt : 0.0f;
   }
   __syncthreads();
-  // phase 4: o_i = sum_j Pi[j][i] o'_j, thread (i = d, q) over rows 32q .. 32q + 31
+  // o_i = sum_j Pi[j][i] o'_j, thread (i = d, q) over rows 32q .. 32q + 31
   float r = 0.0f;
 #pragma unroll
   for (int jj = 0; jj < 32; ++jj) r = fmaf(pj[jj], ob[32 * q + jj], r);
-  rsum[q * D + d] = r;
+  mq[q][d] = r;  // (the combine above has read mq: a barrier separates them)
   __syncthreads();
-  if (tid < D) out[bh * D + d] = rsum[d] + rsum[D + d] + rsum[2 * D + d] + rsum[3 * D + d];
+  if (tid < D) out[bh * D + d] = mq[0][d] + mq[1][d] + mq[2][d] + mq[3][d];
 }
-
-inline size_t merge_smem_bytes(int pmax) { return sizeof(float) * ((size_t)pmax + ((pmax + 3) & ~3) + 9 * D); }
 
 // ------------------------------------------------------------------------------------------ host
 
@@ -1041,36 +1111,29 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
   return p;
 }
 
-// Workspace: q' and S q' [B*Hq][128] fp32, then the partials [B*Hq][pmax][132] fp32.
-size_t workspace_bytes(int B, int Hq, const Plan& p) {
-  return sizeof(float) * ((size_t)2 * B * Hq * D + (size_t)B * Hq * p.pmax * PART);
-}
+// Workspace: the partials [B*Hq][pmax][132] fp32.
+size_t workspace_bytes(int B, int Hq, const Plan& p) { return sizeof(float) * (size_t)B * Hq * p.pmax * PART; }
 
-template <int KB, int VB, bool QJL, int NB>
+template <int KB, int VB, bool QJL, int NB, bool MX>
 tq_status launch_split_nb(const DArgs& a, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        a.dyn_smem);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
-  // programmatic dependent launch: the prologue (tables, first cache stages) overlaps prep
+  // an ordinary launch: the cache it reads may come from the kernel just before (tq_quantize)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.ctas);
   cfg.blockDim = dim3(Shape<NB>::THREADS);
   cfg.dynamicSmemBytes = a.dyn_smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL, NB>, a);
+  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL, NB, MX>, a);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "split launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
 
 // One n-block of four heads when a group has at most four query heads, else two.
-template <int KB, int VB, bool QJL>
+template <int KB, int VB, bool QJL, bool MX = false>
 tq_status launch_split(const DArgs& a, cudaStream_t stream) {
-  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1>(a, stream) : launch_split_nb<KB, VB, QJL, 2>(a, stream);
+  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1, MX>(a, stream) : launch_split_nb<KB, VB, QJL, 2, MX>(a, stream);
 }
 
 template <int KB, bool QJL>
@@ -1083,7 +1146,8 @@ tq_status dispatch_v(int vb, const DArgs& a, cudaStream_t s) {
 }
 
 template <bool QJL>
-tq_status dispatch(int kb, int vb, const DArgs& a, cudaStream_t s) {
+tq_status dispatch(int kb, int vb, bool mixed, const DArgs& a, cudaStream_t s) {
+  if (mixed) return launch_split<4, 4, QJL, true>(a, s);  // (the mixed layout is checked to be 4 / 4)
   switch (kb) {
     case 2: return dispatch_v<2, QJL>(vb, a, s);
     case 3: return dispatch_v<3, QJL>(vb, a, s);
@@ -1100,6 +1164,13 @@ extern "C" size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache,
   const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
   return workspace_bytes(B, Hq, p);
 }
+
+namespace tq {
+int decode_reset_errors() {
+  const unsigned int z = 0;
+  return cudaMemcpyToSymbol(g_decode_error, &z, sizeof(z)) == cudaSuccess ? 0 : -1;
+}
+}  // namespace tq
 
 extern "C" int tq_decode_device_errors(void) {
   unsigned int v = 0;
@@ -1134,7 +1205,7 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * Hq;
   const int g = Hq / cache->Hkv;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   if (seq_len > 0) {
     DArgs a;
     a.B = B;
@@ -1149,7 +1220,8 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
     a.pmax = plan.pmax;
     a.ntot = plan.ntot;
     a.dyn_smem = split_dyn_smem();
-    a.sK = (float)((double)sc * 1.4426950408889634 / sqrt((double)D));
+    // k-hat = ||k|| / sqrt(128) c (mixed layout: ||k_g|| / sqrt(64) c_g of each half)
+    a.sK = (float)((double)sc * 1.4426950408889634 / sqrt(cache->layout == TQ_LAYOUT_MIXED ? 64.0 : (double)D));
     a.sQ = cache->qjl_m ? (float)((double)sc * 1.4426950408889634 * 2.0 * sqrt(M_PI / 2.0) / cache->qjl_m)
                         : 0.0f;
     a.k_codes = cache->k_codes;
@@ -1160,24 +1232,16 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
     a.v_norm = cache->v_norm;
     a.kc = params->k_centroids;
     a.vc = params->v_centroids;
-    a.qrot = ws;
-    a.sq = ws + (size_t)BH * D;
-    a.part = ws + (size_t)2 * BH * D;
-
-    // heads per cluster: about 16 clusters at least (one CTA on each of 128 SMs), at most PREP_HB
-    const int hb = std::max(1, std::min(PREP_HB, BH / 16));
-    const int prep_ctas = (BH + hb - 1) / hb * PREP_CLUSTER;
-    if (q_dtype == TQ_F32)
-      prep_kernel<float><<<prep_ctas, PREP_THREADS, 0, s>>>(reinterpret_cast<const float*>(q), BH, hb, params->Pi,
-                                                             params->S, cache->qjl_m ? 1 : 0, ws, ws + (size_t)BH * D);
-    else
-      prep_kernel<__nv_bfloat16><<<prep_ctas, PREP_THREADS, 0, s>>>(
-          reinterpret_cast<const __nv_bfloat16*>(q), BH, hb, params->Pi, params->S, cache->qjl_m ? 1 : 0, ws,
-          ws + (size_t)BH * D);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
-    st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, a, s)
-                      : dispatch<false>(cache->k_bits, cache->v_bits, a, s);
+    a.kc2 = params->k_centroids_lo;
+    a.vc2 = params->v_centroids_lo;
+    a.q = q;
+    a.q_bf16 = q_dtype == TQ_BF16 ? 1 : 0;
+    a.Pi = params->Pi;
+    a.S = params->S;
+    a.part = ws;
+    const bool mixed = cache->layout == TQ_LAYOUT_MIXED;
+    st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, mixed, a, s)
+                      : dispatch<false>(cache->k_bits, cache->v_bits, mixed, a, s);
     if (st != TQ_OK) return st;
   }
   // merge: programmatic dependent of split (its CTAs wait for the split grid before reading); with
@@ -1185,14 +1249,14 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH);
   cfg.blockDim = dim3(MERGE_THREADS);
-  cfg.dynamicSmemBytes = merge_smem_bytes(plan.pmax);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = seq_len > 0 ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, merge_kernel, (const float*)(ws + (size_t)2 * BH * D), params->Pi, out, Hq, g,
+  e = cudaLaunchKernelEx(&cfg, merge_kernel, (const float*)ws, params->Pi, out, Hq, g,
                          cache->Hkv, plan.hgroups, (int64_t)seq_len, plan.ntot, plan.ctas, plan.pmax);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
   return TQ_OK;

@@ -32,6 +32,11 @@ tq_status check_cache(const tq_cache* c) {
     return fail(TQ_ERR_UNSUPPORTED, "k_bits %d / v_bits %d (2..4)", c->k_bits, c->v_bits);
   if (c->qjl_m != 0 && c->qjl_m != kQjlRows)
     return fail(TQ_ERR_UNSUPPORTED, "qjl_m %d (0 or 128)", c->qjl_m);
+  if (c->layout != TQ_LAYOUT_PLAIN && c->layout != TQ_LAYOUT_MIXED)
+    return fail(TQ_ERR_UNSUPPORTED, "layout %d", c->layout);
+  if (c->layout == TQ_LAYOUT_MIXED && (c->k_bits != 4 || c->v_bits != 4))
+    return fail(TQ_ERR_UNSUPPORTED, "mixed layout with k_bits %d / v_bits %d (only 4 / 4: halves of 4 and 3 bits)",
+                c->k_bits, c->v_bits);
   if (c->B < 1 || c->Hkv < 1 || c->T_cap < 1)
     return fail(TQ_ERR_INVALID_ARG, "cache shape B=%d Hkv=%d T_cap=%d", c->B, c->Hkv, c->T_cap);
   if ((int64_t)c->B * c->Hkv * c->T_cap > (int64_t)1 << 40)
@@ -53,6 +58,14 @@ tq_status check_params(const tq_params* p, const tq_cache* c) {
   if (c->qjl_m && !p->S) return fail(TQ_ERR_INVALID_ARG, "S is NULL with qjl_m=%d", c->qjl_m);
   if (!aligned16(p->Pi) || (c->qjl_m && !aligned16(p->S)) || !aligned16(p->S_Pi))
     return fail(TQ_ERR_INVALID_ARG, "Pi / S / S_Pi must be 16-byte aligned");
+  if (c->layout == TQ_LAYOUT_MIXED) {
+    if (!p->k_centroids_lo || !p->k_thresholds_lo || !p->v_centroids_lo || !p->v_thresholds_lo)
+      return fail(TQ_ERR_INVALID_ARG, "mixed layout: a codebook of the non-outlier half is NULL");
+    int bits = 0;
+    for (int w = 0; w < 4; ++w) bits += __builtin_popcount(p->outlier_mask[w]);
+    if (bits != kHeadDim / 2)
+      return fail(TQ_ERR_INVALID_ARG, "mixed layout: outlier_mask has %d channels (needs %d)", bits, kHeadDim / 2);
+  }
   return TQ_OK;
 }
 

@@ -40,6 +40,22 @@ __host__ __device__ inline int v_slot_of_coord(int j) {
   const int n = j >> 3, g = j & 7;
   return 16 * g + n;
 }
+// Mixed layout (TQ_LAYOUT_MIXED): each half g = j / 64 is its own bit stream; within it the key
+// coordinate 16a + 8h + 2t + e (a < 4) sits at slot 16t + 4a + 2h + e, the value coordinate
+// 8n + g' at slot 8g' + n.  Bit position of coordinate j in the row (half O of `bits_o` bits first):
+__host__ __device__ inline int k_slot_of_coord_mixed(int j) {
+  const int jj = j & 63;
+  const int a = jj >> 4, h = (jj >> 3) & 1, t = (jj >> 1) & 3, e = jj & 1;
+  return 16 * t + 4 * a + 2 * h + e;
+}
+__host__ __device__ inline int v_slot_of_coord_mixed(int j) {
+  const int jj = j & 63;
+  return 8 * (jj & 7) + (jj >> 3);
+}
+__host__ __device__ inline int mixed_bit_pos(int j, int slot, int bits_o) {
+  return j < 64 ? bits_o * slot : 64 * bits_o + (bits_o - 1) * slot;
+}
+
 __host__ __device__ inline int sign_bit_of_row(int l) {
   const int a = l >> 4, h = (l >> 3) & 1, t = (l >> 1) & 3, e = l & 1;
   return 32 * t + (2 * a + h) + 16 * e;
@@ -54,6 +70,9 @@ unsigned int pipe_device_errors();
 long long pipe_vector_fixups();
 long long pipe_code_fixups();
 long long pipe_exempt_codes();
+void pipe_set_test_stall(int enable, long long wait_cycles);
+int decode_reset_errors();
+int pipe_reset_errors();
 long long pipe_exempt_signs();
 
 // Validation shared by tq_quantize / tq_decode_attn.

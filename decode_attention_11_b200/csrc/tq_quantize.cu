@@ -79,6 +79,12 @@ struct QArgs {
   const float* vc;
   const float* vt;
   Guards guard;
+  // mixed layout: codebooks of the non-outlier half (one bit fewer) and the outlier channels
+  const float* kc2;
+  const float* kt2;
+  const float* vc2;
+  const float* vt2;
+  uint32_t omask[4];
 };
 
 constexpr int FL_CAP = 1024;  // deferred single-coordinate fixups per tile
@@ -104,6 +110,10 @@ struct __align__(1024) Smem {
   double fx64[D];           // exact residual of one vector (vector path)
   double red64[THREADS / 32];
   float kcent[16], kthr[16], vcent[16], vthr[16];
+  // mixed layout: half R (non-outlier channels) scales, norms and codebooks
+  float sclk2[TM], sclv2[TM], kn2[TM], vn2[TM];
+  double nrmk2[TM], nrmv2[TM];
+  float kcent2[16], kthr2[16], vcent2[16], vthr2[16];
   uint8_t fcode[D];
   uint8_t fsign[D];
   int nfl, nvfl;
@@ -235,16 +245,15 @@ __device__ __forceinline__ bool code_exempt_exact(double u, const float* thr, in
   return near;
 }
 
-// Read / replace the b-bit code at slot `slot` of a staged row (32-bit shared words).
-__device__ __forceinline__ uint32_t get_code(const uint8_t* row, int bits, int slot) {
-  const int P = bits * slot;
+// Read / replace the b-bit code at bit position P of a staged row (32-bit shared words; in the
+// plain layout P = b * slot, in the mixed layout the position within the row's two streams).
+__device__ __forceinline__ uint32_t get_code_at(const uint8_t* row, int bits, int P) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(row);
   uint64_t v = w[P >> 5];
   if ((P & 31) + bits > 32) v |= (uint64_t)w[(P >> 5) + 1] << 32;
   return (uint32_t)(v >> (P & 31)) & ((1u << bits) - 1u);
 }
-__device__ __forceinline__ void set_code(uint8_t* row, int bits, int slot, uint32_t code) {
-  const int P = bits * slot;
+__device__ __forceinline__ void set_code_at(uint8_t* row, int bits, int P, uint32_t code) {
   uint32_t* w = reinterpret_cast<uint32_t*>(row);
   const int wi = P >> 5, sh = P & 31;
   const uint64_t m = (uint64_t)((1u << bits) - 1u) << sh;
@@ -298,7 +307,10 @@ __device__ __forceinline__ void row_chunk(const InT* xrow, const uint8_t* xt, in
   }
 }
 
-template <int KB, int VB, typename InT>
+// MX: the outlier-aware mixed layout (TQ_LAYOUT_MIXED): chunks ch = 0, 1 (coordinates 0..63) are
+// the outlier half with KB / VB bits, chunks 2, 3 the other half with one bit fewer; each half has
+// its own norm, codebook and power-of-two input scale (exact, as Pi is block-diagonal).
+template <int KB, int VB, typename InT, bool MX>
 __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
@@ -308,6 +320,12 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   // epilogues: thread = (tile row r = TMEM lane, 32-coordinate chunk ch)
   const int r = tid & 127, ch = tid >> 7;
   constexpr int LK = 1 << KB, LV = 1 << VB;
+  constexpr int LK2 = MX ? 1 << (KB - 1) : LK, LV2 = MX ? 1 << (VB - 1) : LV;
+  constexpr int K_ROW = MX ? 8 * (2 * KB - 1) : 16 * KB;  // packed row bytes
+  constexpr int V_ROW = MX ? 8 * (2 * VB - 1) : 16 * VB;
+  const int g = ch >> 1;  // mixed layout: half of this thread's chunk (0: outlier channels)
+  // sqrt(d_half) for u: sqrt(64) per half in the mixed layout, sqrt(128) otherwise
+  const double sqd_u = MX ? 8.0 : sqrt((double)D);
 
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // operand tiles need 1024-byte alignment
     if (tid == 0) atomicOr(&g_quantize_error, 2u);
@@ -327,6 +345,10 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   if (tid < LK - 1) s.kthr[tid] = a.kt[tid];
   if (tid < LV) s.vcent[tid] = a.vc[tid];
   if (tid < LV - 1) s.vthr[tid] = a.vt[tid];
+  if (MX && tid < LK2) s.kcent2[tid] = a.kc2[tid];
+  if (MX && tid < LK2 - 1) s.kthr2[tid] = a.kt2[tid];
+  if (MX && tid < LV2) s.vcent2[tid] = a.vc2[tid];
+  if (MX && tid < LV2 - 1) s.vthr2[tid] = a.vt2[tid];
   if (tid < TM) s.vflag[tid] = 0;
   // Pi enters as 2^8 Pi so that its fp16 lo part stays clear of the subnormal range (the hi + lo
   // pair then carries ~22 significant bits of every entry); the 2^-8 is folded into u's scale.
@@ -361,6 +383,13 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
     TK[j] = (j < LK / 2) ? s.kthr[LK / 2 - 1 + j] : INFINITY;
     TV[j] = (j < LV / 2) ? s.vthr[LV / 2 - 1 + j] : INFINITY;
   }
+  // (mixed layout: the non-outlier half's thresholds)
+  float TK2[8], TV2[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    TK2[j] = (MX && j < LK2 / 2) ? s.kthr2[LK2 / 2 - 1 + j] : INFINITY;
+    TV2[j] = (MX && j < LV2 / 2) ? s.vthr2[LV2 / 2 - 1 + j] : INFINITY;
+  }
 
   uint32_t phase = 0;
   for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, phase ^= 1) {
@@ -381,24 +410,39 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
         cp_async_wait_all();
         __syncthreads();
       }
-      double acc = 0.0;
-      float amax = 0.0f;
+      // Half membership of the eight channels 8c .. 8c + 7 (mixed layout: outlier channels).
+      auto in_o = [&](int c, int i) -> bool {
+        const int ch8 = 8 * c + i;
+        return MX && ((a.omask[ch8 >> 5] >> (ch8 & 31)) & 1u);
+      };
+      double acc = 0.0, acc2 = 0.0;  // plain: acc; mixed: acc (outlier half), acc2 (other half)
+      float amax = 0.0f, amax2 = 0.0f;
 #pragma unroll 1
       for (int c = 8 * chalf; c < 8 * chalf + 8; ++c) {
         float v8[8];
         row_chunk<InT>(xrow, xt, cr, c, clive, v8);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          acc = fma((double)v8[i], (double)v8[i], acc);
-          amax = fmaxf(amax, fabsf(v8[i]));
+          if (!MX || in_o(c, i)) {
+            acc = fma((double)v8[i], (double)v8[i], acc);
+            amax = fmaxf(amax, fabsf(v8[i]));
+          } else {
+            acc2 = fma((double)v8[i], (double)v8[i], acc2);
+            amax2 = fmaxf(amax2, fabsf(v8[i]));
+          }
         }
       }
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      int ex = 0;
-      frexpf(amax, &ex);
-      const int e = amax > 0.0f ? max(-126, min(127, 15 - ex)) : 0;
-      const float p2 = __int_as_float((e + 127) << 23);  // 2^e
+      acc2 += __shfl_xor_sync(0xffffffffu, acc2, 1);
+      amax2 = fmaxf(amax2, __shfl_xor_sync(0xffffffffu, amax2, 1));
+      auto pow2_for = [](float am) {
+        int ex = 0;
+        frexpf(am, &ex);
+        const int e = am > 0.0f ? max(-126, min(127, 15 - ex)) : 0;
+        return __int_as_float((e + 127) << 23);  // 2^e
+      };
+      const float p2 = pow2_for(amax), p2b = MX ? pow2_for(amax2) : p2;
 #pragma unroll 1
       for (int c = 8 * chalf; c < 8 * chalf + 8; ++c) {
         float v8[8];
@@ -406,7 +450,8 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
         uint32_t o[4], ol[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float x0 = v8[2 * i] * p2, x1 = v8[2 * i + 1] * p2;
+          const float s0 = (!MX || in_o(c, 2 * i)) ? p2 : p2b, s1 = (!MX || in_o(c, 2 * i + 1)) ? p2 : p2b;
+          const float x0 = v8[2 * i] * s0, x1 = v8[2 * i + 1] * s1;
           const __half2 hh = __floats2half2_rn(x0, x1);
           o[i] = *reinterpret_cast<const uint32_t*>(&hh);
           if constexpr (sizeof(InT) == 4) {
@@ -423,13 +468,19 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
         const double n = sqrt(acc);
         (cwhich == 0 ? s.nrmk : s.nrmv)[cr] = n;
         (cwhich == 0 ? s.sclk : s.sclv)[cr] =
-            n > 0.0 ? (float)(sqrt((double)D) / (n * (double)p2 * (double)PI_SCALE)) : 0.0f;
+            n > 0.0 ? (float)(sqd_u / (n * (double)p2 * (double)PI_SCALE)) : 0.0f;
+        if constexpr (MX) {
+          const double n2 = sqrt(acc2);
+          (cwhich == 0 ? s.nrmk2 : s.nrmv2)[cr] = n2;
+          (cwhich == 0 ? s.sclk2 : s.sclv2)[cr] =
+              n2 > 0.0 ? (float)(sqd_u / (n2 * (double)p2b * (double)PI_SCALE)) : 0.0f;
+        }
       }
     }
     // sign rows (and 3-bit value rows) are assembled with shared-memory atomics: clear them
     for (int i = tid; i < TM * 4; i += THREADS) reinterpret_cast<uint32_t*>(s.sst)[i] = 0u;
-    if constexpr (VB == 3)
-      for (int i = tid; i < TM * 12; i += THREADS) reinterpret_cast<uint32_t*>(s.vst)[i] = 0u;
+    if constexpr (VB == 3 || MX)  // (the mixed layout's 3-bit value half uses atomics too)
+      for (int i = tid; i < TM * V_ROW / 4; i += THREADS) reinterpret_cast<uint32_t*>(s.vst)[i] = 0u;
     if (tid == 0) {
       s.nfl = 0;
       s.nvfl = 0;
@@ -467,11 +518,22 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
     // ---- 3a. keys: codes, residual rho (fp16 hi + lo into tensor memory), ||rho||^2 ----
     // Chunk ch holds coordinates 32ch + i; for each tau its codes fill the 8 consecutive slots
     // 32 tau + 8 ch + q of coordinates 32ch + 2 tau + {0,1,8,9,16,17,24,25}[q]: one
-    // byte-aligned field of 8 * k_bits bits at byte k_bits * (4 tau + ch).
+    // byte-aligned field of 8 * k_bits bits at byte k_bits * (4 tau + ch).  Mixed layout: the
+    // half's stream starts at byte 0 (outlier half) or 8 k_bits, and the field of chunk ch holds
+    // slots 16 tau + 8 (ch & 1) + q at byte b (2 tau + (ch & 1)) of it, b the half's bit width.
+    // The residual entering the sketch is, in the mixed layout, f_g rho with
+    // f_g = sqrt(2) ||x_g|| / ||x||: sqrt(128) / ||x|| times the half's residual in the rotated
+    // basis, so that the sketch is S r in the units of the plain method.
     {
-      const float scl = s.sclk[r];
+      const bool g1 = MX && g == 1;
+      const float scl = g1 ? s.sclk2[r] : s.sclk[r];
       const bool zero = scl == 0.0f;
-      uint8_t* krow = s.kst + r * (16 * KB);
+      float fg = 1.0f;
+      if constexpr (MX) {
+        const double n0 = s.nrmk[r], n1 = s.nrmk2[r], nx = sqrt(n0 * n0 + n1 * n1);
+        fg = nx > 0.0 ? (float)(1.4142135623730951 * (g1 ? n1 : n0) / nx) : 0.0f;
+      }
+      uint8_t* krow = s.kst + r * K_ROW;
       float r2 = 0.0f;
       uint32_t yr[32];
       tmem_ld32(tmem + lane_base + COL_K + 32 * ch, yr);
@@ -479,6 +541,9 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
       uint32_t hi[16], lo[16];
       uint32_t fld[4] = {0u, 0u, 0u, 0u};
       uint32_t near = 0u;
+      const int LKg = g1 ? LK2 : LK;
+      const float* kcg = g1 ? s.kcent2 : s.kcent;
+      const int bg = g1 ? KB - 1 : KB;
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         float rr[2];
@@ -488,14 +553,16 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
           const float u = __uint_as_float(yr[ii]) * scl;
           const float aa = fabsf(u);
           float margin;
-          const int kpos = search_pos<KB>(aa, TK, margin);
-          const int idx = zero ? LK / 2 : (u >= 0.0f ? LK / 2 + kpos : LK / 2 - 1 - kpos);
-          const float rho = u - s.kcent[idx];
+          int kpos;
+          if constexpr (MX) kpos = g1 ? search_pos<KB - 1>(aa, TK2, margin) : search_pos<KB>(aa, TK, margin);
+          else kpos = search_pos<KB>(aa, TK, margin);
+          const int idx = zero ? LKg / 2 : (u >= 0.0f ? LKg / 2 + kpos : LKg / 2 - 1 - kpos);
+          const float rho = (u - kcg[idx]) * fg;
           near |= (fminf(margin, aa) < a.guard.code_k ? 1u : 0u) << ii;
           rr[e2] = rho;
           r2 = fmaf(rho, rho, r2);
           const int tau = (ii & 7) >> 1, q = ((ii >> 4) << 2) | (((ii >> 3) & 1) << 1) | (ii & 1);
-          fld[tau] |= (uint32_t)idx << (KB * q);
+          fld[tau] |= (uint32_t)idx << (bg * q);
         }
         const __half2 hh = __floats2half2_rn(rr[0], rr[1]);
         const float2 hf = __half22float2(hh);
@@ -505,15 +572,24 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
       }
 #pragma unroll
       for (int tau = 0; tau < 4; ++tau) {
-        uint8_t* dst = krow + KB * (4 * tau + ch);
-        if constexpr (KB == 4) {
-          *reinterpret_cast<uint32_t*>(dst) = fld[tau];
-        } else if constexpr (KB == 2) {
-          *reinterpret_cast<uint16_t*>(dst) = (uint16_t)fld[tau];
+        if constexpr (MX) {
+          uint8_t* dst = krow + (g1 ? 8 * KB : 0) + bg * (2 * tau + (ch & 1));
+          if (!g1 && KB == 4) {
+            *reinterpret_cast<uint32_t*>(dst) = fld[tau];
+          } else {
+            for (int bb = 0; bb < bg; ++bb) dst[bb] = (uint8_t)(fld[tau] >> (8 * bb));
+          }
         } else {
-          dst[0] = (uint8_t)fld[tau];
-          dst[1] = (uint8_t)(fld[tau] >> 8);
-          dst[2] = (uint8_t)(fld[tau] >> 16);
+          uint8_t* dst = krow + KB * (4 * tau + ch);
+          if constexpr (KB == 4) {
+            *reinterpret_cast<uint32_t*>(dst) = fld[tau];
+          } else if constexpr (KB == 2) {
+            *reinterpret_cast<uint16_t*>(dst) = (uint16_t)fld[tau];
+          } else {
+            dst[0] = (uint8_t)fld[tau];
+            dst[1] = (uint8_t)(fld[tau] >> 8);
+            dst[2] = (uint8_t)(fld[tau] >> 16);
+          }
         }
       }
       if (a.qjl) {
@@ -532,37 +608,52 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
       }
     }
     // ---- 3b. values: codes.  Coordinate 32ch + i sits at slot 16 (i % 8) + 4 ch + i / 8: chunk ch
-    //          gives lane group g a field of 4 codes at bit v_bits (16 g + 4 ch). ----
+    //          gives lane group g a field of 4 codes at bit v_bits (16 g + 4 ch).  Mixed layout:
+    //          within the half's stream (byte 0 or 8 v_bits), slot 8 (i % 8) + 4 (ch & 1) + i / 8. ----
     {
-      const float scl = s.sclv[r];
+      const bool g1 = MX && g == 1;
+      const float scl = g1 ? s.sclv2[r] : s.sclv[r];
       const bool zero = scl == 0.0f;
       uint32_t yr[32];
       tmem_ld32(tmem + lane_base + COL_V + 32 * ch, yr);
       tmem_wait_ld();
       uint32_t near = 0u;
       uint32_t f8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      const int LVg = g1 ? LV2 : LV;
+      const int bg = g1 ? VB - 1 : VB;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float u = __uint_as_float(yr[i]) * scl;
         const float aa = fabsf(u);
         float margin;
-        const int kpos = search_pos<VB>(aa, TV, margin);
-        const int idx = zero ? LV / 2 : (u >= 0.0f ? LV / 2 + kpos : LV / 2 - 1 - kpos);
+        int kpos;
+        if constexpr (MX) kpos = g1 ? search_pos<VB - 1>(aa, TV2, margin) : search_pos<VB>(aa, TV, margin);
+        else kpos = search_pos<VB>(aa, TV, margin);
+        const int idx = zero ? LVg / 2 : (u >= 0.0f ? LVg / 2 + kpos : LVg / 2 - 1 - kpos);
         near |= (fminf(margin, aa) < a.guard.code_v ? 1u : 0u) << i;
-        f8[i & 7] |= (uint32_t)idx << (VB * (i >> 3));
+        f8[i & 7] |= (uint32_t)idx << (bg * (i >> 3));
       }
-      uint8_t* vrow = s.vst + r * (16 * VB);
+      uint8_t* vrow = s.vst + r * V_ROW;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        if constexpr (VB == 4) {
-          *reinterpret_cast<uint16_t*>(vrow + 8 * g + 2 * ch) = (uint16_t)f8[g];
+      for (int gg = 0; gg < 8; ++gg) {
+        if constexpr (MX) {
+          if (!g1 && VB == 4) {
+            *reinterpret_cast<uint16_t*>(vrow + 4 * gg + 2 * (ch & 1)) = (uint16_t)f8[gg];
+          } else {  // 4 codes of bg bits at bit 8 (8 VB) + bg (8 gg + 4 (ch & 1)) of the row
+            const int P = (g1 ? 64 * VB : 0) + bg * (8 * gg + 4 * (ch & 1));
+            uint32_t* w = reinterpret_cast<uint32_t*>(vrow);
+            atomicOr(&w[P >> 5], f8[gg] << (P & 31));
+            if ((P & 31) + 4 * bg > 32) atomicOr(&w[(P >> 5) + 1], f8[gg] >> (32 - (P & 31)));
+          }
+        } else if constexpr (VB == 4) {
+          *reinterpret_cast<uint16_t*>(vrow + 8 * gg + 2 * ch) = (uint16_t)f8[gg];
         } else if constexpr (VB == 2) {
-          vrow[4 * g + ch] = (uint8_t)f8[g];
+          vrow[4 * gg + ch] = (uint8_t)f8[gg];
         } else {
-          const int P = 48 * g + 12 * ch;  // 12-bit field: may straddle two words
+          const int P = 48 * gg + 12 * ch;  // 12-bit field: may straddle two words
           uint32_t* w = reinterpret_cast<uint32_t*>(vrow);
-          atomicOr(&w[P >> 5], f8[g] << (P & 31));
-          if ((P & 31) > 20) atomicOr(&w[(P >> 5) + 1], f8[g] >> (32 - (P & 31)));
+          atomicOr(&w[P >> 5], f8[gg] << (P & 31));
+          if ((P & 31) > 20) atomicOr(&w[(P >> 5) + 1], f8[gg] >> (32 - (P & 31)));
         }
       }
       if (!(live && !zero)) near = 0u;
@@ -577,6 +668,10 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
     if (ch == 0) {
       s.kn[r] = (float)s.nrmk[r];
       s.vn[r] = (float)s.nrmv[r];
+      if constexpr (MX) {
+        s.kn2[r] = (float)s.nrmk2[r];
+        s.vn2[r] = (float)s.nrmv2[r];
+      }
     }
     tc_fence_before();
     __syncthreads();
@@ -604,18 +699,24 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
         const double part = have ? exact_dot_part<InT>(a.Pi, x, j, tid & 3) : 0.0;
         const double dot = quad_sum(part);  // all lanes take part in the shuffle
         if (!have || (tid & 3)) continue;
-        const double nn = val ? s.nrmv[rr] : s.nrmk[rr];
-        const double ud = sqrt((double)D) * dot / nn;
-        if (code_exempt_exact(ud, val ? s.vthr : s.kthr, (val ? LV : LK) - 1)) atomicAdd(&s.nexc, 1u);
+        const bool hj = MX && j >= 64;  // mixed layout: coordinate of the non-outlier half
+        const double nn = val ? (hj ? s.nrmv2[rr] : s.nrmv[rr]) : (hj ? s.nrmk2[rr] : s.nrmk[rr]);
+        const double ud = sqd_u * dot / nn;
+        const float* thr = val ? (hj ? s.vthr2 : s.vthr) : (hj ? s.kthr2 : s.kthr);
+        const int nthr = (val ? (hj ? LV2 : LV) : (hj ? LK2 : LK)) - 1;
+        if (code_exempt_exact(ud, thr, nthr)) atomicAdd(&s.nexc, 1u);
+        const uint32_t idx = (uint32_t)code_exact(ud, thr, nthr);
         if (val) {
-          const uint32_t idx = (uint32_t)code_exact(ud, s.vthr, LV - 1);
-          uint8_t* row = s.vst + rr * (16 * VB);
-          if (get_code(row, VB, v_slot_of_coord(j)) != idx) set_code(row, VB, v_slot_of_coord(j), idx);
+          uint8_t* row = s.vst + rr * V_ROW;
+          const int bits = hj ? VB - 1 : VB;
+          const int P = MX ? mixed_bit_pos(j, v_slot_of_coord_mixed(j), VB) : VB * v_slot_of_coord(j);
+          if (get_code_at(row, bits, P) != idx) set_code_at(row, bits, P, idx);
         } else {
-          const uint32_t idx = (uint32_t)code_exact(ud, s.kthr, LK - 1);
-          uint8_t* row = s.kst + rr * (16 * KB);
-          if (get_code(row, KB, k_slot_of_coord(j)) != idx) {
-            set_code(row, KB, k_slot_of_coord(j), idx);
+          uint8_t* row = s.kst + rr * K_ROW;
+          const int bits = hj ? KB - 1 : KB;
+          const int P = MX ? mixed_bit_pos(j, k_slot_of_coord_mixed(j), KB) : KB * k_slot_of_coord(j);
+          if (get_code_at(row, bits, P) != idx) {
+            set_code_at(row, bits, P, idx);
             // the residual fed to the sketch came from the other cell: redo the vector in fp64
             if (a.qjl) atomicOr(&s.vflag[rr], 1u);
           }
@@ -650,9 +751,11 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
     __syncthreads();
     if (s.err) break;
     if (tid < TM) {
-      if (a.qjl)
-        s.rn[tid] = (float)(s.nrmk[tid] * sqrt((double)(s.rho2[0][tid] + s.rho2[1][tid] + s.rho2[2][tid] +
-                                                        s.rho2[3][tid])) / sqrt((double)D));
+      if (a.qjl) {
+        const double nk = MX ? sqrt(s.nrmk[tid] * s.nrmk[tid] + s.nrmk2[tid] * s.nrmk2[tid]) : s.nrmk[tid];
+        s.rn[tid] = (float)(nk * sqrt((double)(s.rho2[0][tid] + s.rho2[1][tid] + s.rho2[2][tid] +
+                                                s.rho2[3][tid])) / sqrt((double)D));
+      }
       if (s.vflag[tid]) s.vfl[atomicAdd(&s.nvfl, 1)] = (uint8_t)tid;
     }
     __syncthreads();
@@ -665,49 +768,68 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
         const int rr = s.vfl[f];
         const unsigned int fl = s.vflag[rr];
         if (fl & 4) {  // value row
-          const double nv = s.nrmv[rr];
           const InT* vx = reinterpret_cast<const InT*>(a.v) + in_base + (int64_t)rr * a.st;
           {
             const int j = tid >> 2;
+            const bool hj = MX && j >= 64;
+            const double nv = hj ? s.nrmv2[rr] : s.nrmv[rr];
+            const float* thr = hj ? s.vthr2 : s.vthr;
+            const int nthr = (hj ? LV2 : LV) - 1;
             const double dot = quad_sum(exact_dot_part<InT>(a.Pi, vx, j, tid & 3));
             if ((tid & 3) == 0) {
-              const int idx = nv > 0.0 ? code_exact(sqrt((double)D) * dot / nv, s.vthr, LV - 1) : LV / 2;
+              const int idx = nv > 0.0 ? code_exact(sqd_u * dot / nv, thr, nthr) : (nthr + 1) / 2;
               // (a row whose near-threshold list overflowed: its coordinates are counted here)
-              if (nv > 0.0 && code_exempt_exact(sqrt((double)D) * dot / nv, s.vthr, LV - 1)) atomicAdd(&s.nexc, 1u);
-              s.fcode[v_slot_of_coord(j)] = (uint8_t)idx;
+              if (nv > 0.0 && code_exempt_exact(sqd_u * dot / nv, thr, nthr)) atomicAdd(&s.nexc, 1u);
+              s.fcode[MX ? (hj ? 64 : 0) + v_slot_of_coord_mixed(j) : v_slot_of_coord(j)] = (uint8_t)idx;
             }
           }
           __syncthreads();
-          if (tid < 4 * VB) {
+          if (tid < V_ROW / 4) {
             uint32_t word = 0;
             for (int kk = 0; kk < 32; ++kk) {
               const int P = 32 * tid + kk;
-              word |= (uint32_t)((s.fcode[P / VB] >> (P % VB)) & 1) << kk;
+              int code, bit;
+              if (MX && P >= 64 * VB) {
+                code = s.fcode[64 + (P - 64 * VB) / (VB - 1)];
+                bit = (P - 64 * VB) % (VB - 1);
+              } else {
+                code = s.fcode[P / VB];
+                bit = P % VB;
+              }
+              word |= (uint32_t)((code >> bit) & 1) << kk;
             }
-            reinterpret_cast<uint32_t*>(s.vst + rr * (16 * VB))[tid] = word;
+            reinterpret_cast<uint32_t*>(s.vst + rr * V_ROW)[tid] = word;
           }
           __syncthreads();
         }
         if (!(fl & 3)) continue;  // uniform: read from shared memory after a barrier
-        const double nk = s.nrmk[rr];
         const InT* kx = reinterpret_cast<const InT*>(a.k) + in_base + (int64_t)rr * a.st;
+        // ||x|| (mixed layout: of both halves); each coordinate's residual enters the sketch as
+        // f_g rho (f_g = sqrt(2) ||x_g|| / ||x||, 1 in the plain layout)
+        const double nk = MX ? sqrt(s.nrmk[rr] * s.nrmk[rr] + s.nrmk2[rr] * s.nrmk2[rr]) : s.nrmk[rr];
         {
           const int j = tid >> 2;
+          const bool hj = MX && j >= 64;
+          const double ng = hj ? s.nrmk2[rr] : s.nrmk[rr];
+          const float* thr = hj ? s.kthr2 : s.kthr;
+          const float* cen = hj ? s.kcent2 : s.kcent;
+          const int nthr = (hj ? LK2 : LK) - 1;
+          const double fgd = MX ? (nk > 0.0 ? 1.4142135623730951 * ng / nk : 0.0) : 1.0;
           const double dot = quad_sum(exact_dot_part<InT>(a.Pi, kx, j, tid & 3));
           double rho = 0.0;
           if ((tid & 3) == 0) {
             int idx;
-            if (nk > 0.0) {
-              const double ud = sqrt((double)D) * dot / nk;
-              idx = code_exact(ud, s.kthr, LK - 1);
-              if ((fl & 2) && code_exempt_exact(ud, s.kthr, LK - 1)) atomicAdd(&s.nexc, 1u);
-              rho = ud - (double)s.kcent[idx];
+            if (ng > 0.0) {
+              const double ud = sqd_u * dot / ng;
+              idx = code_exact(ud, thr, nthr);
+              if ((fl & 2) && code_exempt_exact(ud, thr, nthr)) atomicAdd(&s.nexc, 1u);
+              rho = (ud - (double)cen[idx]) * fgd;
             } else {
-              idx = LK / 2;
-              rho = -(double)s.kcent[idx];
+              idx = (nthr + 1) / 2;
+              rho = -(double)cen[idx] * fgd;
             }
             s.fx64[j] = rho;
-            s.fcode[k_slot_of_coord(j)] = (uint8_t)idx;
+            s.fcode[MX ? (hj ? 64 : 0) + k_slot_of_coord_mixed(j) : k_slot_of_coord(j)] = (uint8_t)idx;
           }
           double q2 = rho * rho;
           for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xffffffffu, q2, o);
@@ -730,13 +852,21 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
           }
         }
         __syncthreads();
-        if (tid < 4 * KB) {
+        if (tid < K_ROW / 4) {
           uint32_t word = 0;
           for (int kk = 0; kk < 32; ++kk) {
             const int P = 32 * tid + kk;
-            word |= (uint32_t)((s.fcode[P / KB] >> (P % KB)) & 1) << kk;
+            int code, bit;
+            if (MX && P >= 64 * KB) {
+              code = s.fcode[64 + (P - 64 * KB) / (KB - 1)];
+              bit = (P - 64 * KB) % (KB - 1);
+            } else {
+              code = s.fcode[P / KB];
+              bit = P % KB;
+            }
+            word |= (uint32_t)((code >> bit) & 1) << kk;
           }
-          reinterpret_cast<uint32_t*>(s.kst + rr * (16 * KB))[tid] = word;
+          reinterpret_cast<uint32_t*>(s.kst + rr * K_ROW)[tid] = word;
         } else if (tid >= 32 && tid < 36 && a.qjl) {
           const int w = tid - 32;
           uint32_t word = 0;
@@ -757,20 +887,36 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
 
     // ---- 6. coalesced stores of the tile's rows ----
     {
-      const uint4* src = reinterpret_cast<const uint4*>(s.kst);
-      uint4* dst = reinterpret_cast<uint4*>(a.k_codes + row0 * (16 * KB));
-      for (int i = tid; i < nt * KB; i += THREADS) dst[i] = src[i];
-      src = reinterpret_cast<const uint4*>(s.vst);
-      dst = reinterpret_cast<uint4*>(a.v_codes + row0 * (16 * VB));
-      for (int i = tid; i < nt * VB; i += THREADS) dst[i] = src[i];
+      if constexpr (MX) {  // rows of 56 bytes: 8-byte units (any row is 8-byte aligned)
+        const uint2* srk = reinterpret_cast<const uint2*>(s.kst);
+        uint2* dsk = reinterpret_cast<uint2*>(a.k_codes + row0 * K_ROW);
+        for (int i = tid; i < nt * K_ROW / 8; i += THREADS) dsk[i] = srk[i];
+        const uint2* srv = reinterpret_cast<const uint2*>(s.vst);
+        uint2* dsv = reinterpret_cast<uint2*>(a.v_codes + row0 * V_ROW);
+        for (int i = tid; i < nt * V_ROW / 8; i += THREADS) dsv[i] = srv[i];
+      } else {
+        const uint4* srk = reinterpret_cast<const uint4*>(s.kst);
+        uint4* dsk = reinterpret_cast<uint4*>(a.k_codes + row0 * K_ROW);
+        for (int i = tid; i < nt * KB; i += THREADS) dsk[i] = srk[i];
+        const uint4* srv = reinterpret_cast<const uint4*>(s.vst);
+        uint4* dsv = reinterpret_cast<uint4*>(a.v_codes + row0 * V_ROW);
+        for (int i = tid; i < nt * VB; i += THREADS) dsv[i] = srv[i];
+      }
+      const uint4* src;
+      uint4* dst;
       if (a.qjl) {
         src = reinterpret_cast<const uint4*>(s.sst);
         dst = reinterpret_cast<uint4*>(a.k_signs + row0 * 16);
         for (int i = tid; i < nt; i += THREADS) dst[i] = src[i];
       }
       for (int i = tid; i < nt; i += THREADS) {
-        a.k_norm[row0 + i] = s.kn[i];
-        a.v_norm[row0 + i] = s.vn[i];
+        if constexpr (MX) {
+          reinterpret_cast<float2*>(a.k_norm)[row0 + i] = make_float2(s.kn[i], s.kn2[i]);
+          reinterpret_cast<float2*>(a.v_norm)[row0 + i] = make_float2(s.vn[i], s.vn2[i]);
+        } else {
+          a.k_norm[row0 + i] = s.kn[i];
+          a.v_norm[row0 + i] = s.vn[i];
+        }
         if (a.qjl) a.k_rnorm[row0 + i] = s.rn[i];
       }
     }
@@ -783,15 +929,15 @@ __global__ void __launch_bounds__(THREADS, 1) quantize_kernel(QArgs a) {
   if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-template <int KB, int VB, typename InT>
+template <int KB, int VB, typename InT, bool MX = false>
 tq_status launch3(const QArgs& a, int sms, cudaStream_t stream) {
   const size_t smem = sizeof(Smem);
-  cudaError_t e = cudaFuncSetAttribute(quantize_kernel<KB, VB, InT>,
+  cudaError_t e = cudaFuncSetAttribute(quantize_kernel<KB, VB, InT, MX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
   const int64_t total = (int64_t)a.B * a.Hkv * ((a.T_new + TM - 1) / TM);
   const int grid = (int)(total < sms ? total : sms);
-  quantize_kernel<KB, VB, InT><<<grid, THREADS, smem, stream>>>(a);
+  quantize_kernel<KB, VB, InT, MX><<<grid, THREADS, smem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "quantize launch: %s", cudaGetErrorString(e));
   return TQ_OK;
@@ -901,6 +1047,14 @@ extern "C" tq_status tq_quantize(const tq_params* params, const void* k, const v
   // bands below are >= 4x those.  fp32 values enter as fp16(x) alone (relative 2^-12, ~2e-4 in u).
   a.guard = dtype == TQ_F32 ? Guards{4e-6f, 4e-3f, 3e-5f} : Guards{4e-6f, 4e-6f, 3e-5f};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cache->layout == TQ_LAYOUT_MIXED) {  // 4-bit outlier half, 3-bit other half (checked above)
+    a.kc2 = params->k_centroids_lo;
+    a.kt2 = params->k_thresholds_lo;
+    a.vc2 = params->v_centroids_lo;
+    a.vt2 = params->v_thresholds_lo;
+    for (int w = 0; w < 4; ++w) a.omask[w] = params->outlier_mask[w];
+    return dtype == TQ_F32 ? launch3<4, 4, float, true>(a, sms, s) : launch3<4, 4, __nv_bfloat16, true>(a, sms, s);
+  }
   if (dtype == TQ_BF16) {
     bool handled = false;
     st = quantize_bf16_pipeline(params, k, v, stride_b, stride_h, stride_t, T_new, t_offset, cache, sms, s,
@@ -945,4 +1099,18 @@ extern "C" long long tq_quantize_exempt_signs(void) {
   if (cudaMemcpyFromSymbol(&v, tq::g_quantize_exempt_signs, sizeof(v)) != cudaSuccess) return -1;
   const long long p = tq::pipe_exempt_signs();
   return p < 0 ? -1 : (long long)v + p;
+}
+
+extern "C" tq_status tq_debug_quantize_stall(int enable, long long wait_cycles) {
+  tq::clear_error();
+  if (enable && wait_cycles <= 0) return tq::fail(TQ_ERR_INVALID_ARG, "wait_cycles %lld must be > 0", wait_cycles);
+  tq::pipe_set_test_stall(enable, wait_cycles);
+  return TQ_OK;
+}
+
+extern "C" int tq_reset_device_errors(void) {
+  const unsigned int z = 0;
+  if (cudaMemcpyToSymbol(tq::g_quantize_error, &z, sizeof(z)) != cudaSuccess) return -1;
+  if (tq::pipe_reset_errors() != 0) return -1;
+  return tq::decode_reset_errors();
 }

@@ -30,6 +30,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -52,11 +53,13 @@ constexpr int N_CONV_WARPS = 4;
 constexpr uint32_t IDESC = idesc_f16_f32(128, 128);
 constexpr uint32_t TMEM_COLS = 512;         // two buffers x (Y_K | Y_V)
 constexpr int QCAP = 1024;                  // fixup ring entries per CTA (>= 2 tiles' worth)
+constexpr int SLOW_CAP = 64;                // key rows deferred to the cooperative end phase
 constexpr int MAX_CTAS = 160;
+static_assert(sizeof(int) == 4, "");
 constexpr int LUT_N = 128;                  // cells of the code lookup tables
 constexpr float CELL_MAGIC = 8388608.0f + 64.0f;  // 2^23 + cell offset: fma(u, alpha, .) rounds to a cell
 constexpr float PI_SCALE = 256.0f;
-constexpr long long WAIT_LIMIT = 4000000000LL;    // ~2 s of SM clock
+constexpr long long WAIT_LIMIT = 4000000000LL;    // ~2 s of SM clock (default bound of every wait)
 constexpr float C_SCALE = 0.04419417382415922f;   // sqrt(128) / 256 (u = y * C_SCALE / ||x||)
 
 __device__ unsigned int g_pipe_error;         // bit 0: a wait timed out; bit 1: smem misaligned; bit 2: no LUT
@@ -67,18 +70,17 @@ __device__ unsigned int g_pipe_code_fixups;
 // fp64 fixups, which every such case reaches: the fast path's error is far inside its guard bands).
 __device__ unsigned int g_pipe_exempt_codes;
 __device__ unsigned int g_pipe_exempt_signs;
-// Launch epoch of the fixup ring: read by every CTA at start, advanced by the last CTA to finish,
-// so consecutive launches on a stream (CUDA graph replays included) never share an epoch.
-__device__ unsigned int g_pipe_epoch;
-__device__ unsigned int g_pipe_ctas_done;
+// The fixup ring of a CTA is the row of the SM it runs on: a CTA of this kernel takes nearly all of
+// an SM's shared memory, so no two of them (of one launch, of overlapping launches, or of launches
+// on other streams) ever share an SM.  Each CTA draws a fresh generation number for its SM at
+// start; ring entries carry it in their tag, so entries left by earlier CTAs never match.
+constexpr int MAX_SMS = 256;
+__device__ unsigned int g_ring_gen[MAX_SMS];
 
-// One thread per CTA, on every exit path.
-__device__ __forceinline__ void count_cta_done() {
-  __threadfence();
-  if (atomicAdd(&g_pipe_ctas_done, 1u) == gridDim.x - 1) {  // every CTA has read the epoch
-    g_pipe_ctas_done = 0;
-    atomicAdd(&g_pipe_epoch, 1u);
-  }
+__device__ __forceinline__ uint32_t sm_id() {
+  uint32_t v;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(v));
+  return v;
 }
 
 // One queued fixup for row r of global tile `tile` (CTA-local tile number seqt).  kind 0 / 1: half
@@ -97,7 +99,7 @@ struct FixEntry {
   uint32_t pad;
   uint64_t tag;
 };
-__device__ FixEntry g_fix_ring[MAX_CTAS][QCAP];
+__device__ FixEntry g_fix_ring[MAX_SMS][QCAP];
 
 struct PArgs {
   const __nv_bfloat16* k;
@@ -122,6 +124,8 @@ struct PArgs {
   const float* vc;
   const float* vt;
   float band_code, band_sign;
+  long long wait_limit;  // bound of every wait, in SM cycles (WAIT_LIMIT unless a test shortens it)
+  int stall_first_load;  // test hook: each CTA skips its first TMA load (its waits then run out)
 };
 
 struct __align__(1024) PSmem {
@@ -157,7 +161,12 @@ struct __align__(1024) PSmem {
   unsigned int stored_seq;   // tiles in global memory (CTA-local count)
   unsigned int main_done;
   unsigned int fix_done[N_FIX];
-  uint32_t epoch;            // this launch's ring epoch
+  long long wait_limit;      // bound of every wait (SM cycles)
+  unsigned int n_slow;       // key rows queued for the cooperative fp64 re-derivation
+  uint32_t slow[SLOW_CAP][2];// (tile, row) of each
+  double cred[THREADS / 32]; // cooperative phase: warp partial sums
+  uint32_t epoch;            // this CTA's generation on its SM (ring tags)
+  uint32_t ring;             // this CTA's ring row (its SM)
   unsigned int pi_lo;        // Pi has a nonzero fp16 lo part (else its lo MMA pass is skipped)
 };
 
@@ -199,7 +208,7 @@ __device__ __forceinline__ bool pwait(PSmem& s, uint64_t* bar, uint32_t parity) 
         : "memory");
     if (done) return true;
     if (*reinterpret_cast<volatile unsigned int*>(&s.err)) return false;
-    if (clock64() - t0 > WAIT_LIMIT) {
+    if (clock64() - t0 > s.wait_limit) {
       atomicOr(&s.err, 1u);
       return false;
     }
@@ -219,7 +228,7 @@ __device__ __forceinline__ bool pwait_w(PSmem& s, uint64_t* bar, uint32_t parity
         : "r"(a), "r"(parity), "r"(100000u)
         : "memory");
     if (__any_sync(0xffffffffu, done != 0)) return true;  // the phase has completed
-    const bool stop = *reinterpret_cast<volatile unsigned int*>(&s.err) != 0 || clock64() - t0 > WAIT_LIMIT;
+    const bool stop = *reinterpret_cast<volatile unsigned int*>(&s.err) != 0 || clock64() - t0 > s.wait_limit;
     if (__any_sync(0xffffffffu, stop)) {
       if ((threadIdx.x & 31) == 0) atomicOr(&s.err, 1u);
       return false;
@@ -682,6 +691,22 @@ __device__ __forceinline__ void fix_entry(PSmem& s, const PArgs& a, const FixEnt
     }
     return;
   }
+  // The whole key vector has to be re-derived in fp64 (u, codes, rho, every sign, ||r||): that is
+  // two 128 x 128 matrix-vector products, a long chain of memory round trips for one warp, so the
+  // row goes to the cooperative phase at the end of the kernel, where all 16 warps share it.
+  unsigned int qs = 0;
+  if (lane == 0) {
+    qs = atomicAdd(&s.n_slow, 1u);
+    if (qs < SLOW_CAP) {
+      s.slow[qs][0] = E.tile;
+      s.slow[qs][1] = E.r | (vec ? 0x10000u : 0u);  // bit 16: a key code changed (||r|| too)
+    }
+  }
+  if (__shfl_sync(0xffffffffu, qs, 0) < SLOW_CAP) {
+    if (lane == 0) atomicAdd(&g_pipe_vector_fixups, 1u);
+    return;
+  }
+  // (list full: the warp does it itself)
   // Exact residual of the whole key vector (fp64): u, codes, rho.
   double r2 = 0.0;
   matvec8(a.Pi, x, [&](int j, double dot) {  // lane (4 q) receives Pi row j = j0 + q
@@ -763,36 +788,36 @@ __device__ __forceinline__ void coords(const PArgs& a, int64_t tile, int& b, int
 }
 
 // ================================================================ TMA producer (warp 12)
-__device__ __noinline__ void role_tma(const PArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                                      int n_tiles) {
+// Load L of the CTA: tile L / 2, K (L even) or V (L odd), into ring slot L % SLOTS.
+__device__ __forceinline__ void issue_load(const PArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, int L) {
   PSmem& s = smem();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  (void)tid; (void)warp; (void)lane;
-  // ================================================================ TMA producer
+  int b, h, t0, nt;
+  coords(a, tile_of(L >> 1), b, h, t0, nt);
+  const int sl = L % SLOTS;
+  mbar_arrive_expect_tx(&s.full[sl], TILE_BYTES);
+  const void* tm = (L & 1) ? (const void*)tmv : (const void*)tmk;
+  tma_load_4d(smem_u32(s.slot[sl]), tm, &s.full[sl], 0, t0, h, b);
+  tma_load_4d(smem_u32(s.slot[sl] + TILE_BYTES / 2), tm, &s.full[sl], 64, t0, h, b);
+}
+
+// Loads [first, 2 n_tiles): the first ones were issued in the prologue, before the operands were
+// staged, so that the first tile is in flight meanwhile.
+__device__ __noinline__ void role_tma(const PArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                                      int n_tiles, int first) {
+  PSmem& s = smem();
+  const int lane = threadIdx.x & 31;
   if (lane == 0) {
-    int issued = 0;
-    for (int it = 0; it < n_tiles; ++it) {
-      int b, h, t0, nt;
-      coords(a, tile_of(it), b, h, t0, nt);
-      bool ok = true;
-      for (int which = 0; which < 2 && ok; ++which) {
-        const int L = 2 * it + which, sl = L % SLOTS, u = L / SLOTS;
-        if (u >= 1 && !pwait(s, &s.empty[sl], (u - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&s.full[sl], TILE_BYTES);
-        const void* tm = which ? (const void*)tmv : (const void*)tmk;
-        tma_load_4d(smem_u32(s.slot[sl]), tm, &s.full[sl], 0, t0, h, b);
-        tma_load_4d(smem_u32(s.slot[sl] + TILE_BYTES / 2), tm, &s.full[sl], 64, t0, h, b);
-        ++issued;
-      }
-      if (!ok) break;
+    int issued = first;
+    for (int L = first; L < 2 * n_tiles; ++L) {
+      const int sl = L % SLOTS, u = L / SLOTS;
+      if (u >= 1 && !pwait(s, &s.empty[sl], (u - 1) & 1)) break;
+      issue_load(a, tmk, tmv, L);
+      ++issued;
     }
     // every load issued has landed before the CTA may exit
     for (int L = max(0, issued - SLOTS); L < issued; ++L) {
       const long long t0 = clock64();
-      while (!mbar_test(&s.full[L % SLOTS], (L / SLOTS) & 1) && clock64() - t0 < WAIT_LIMIT) {
+      while (!mbar_test(&s.full[L % SLOTS], (L / SLOTS) & 1) && clock64() - t0 < s.wait_limit) {
       }
     }
   }
@@ -836,6 +861,10 @@ __device__ __noinline__ void role_mma(const PArgs& a, uint32_t tmem, int n_tiles
   __syncwarp();
 }
 
+// Programmatic dependent launch: a quantize launch may start while the previous one (a chunk of
+// the same stream) finishes; every thread waits for it to complete before its first global store.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t fix_tag(const PSmem& s, unsigned int k) {
   return ((uint64_t)s.epoch << 32) | (uint64_t)(k + 1u);
 }
@@ -849,14 +878,14 @@ __device__ __forceinline__ void push_fix(PSmem& s, const PArgs& a, const FixEntr
     const unsigned int m = slot - QCAP;
     const long long tw = clock64();
     while (ld_acq(&s.fix_done[m % N_FIX]) <= m / N_FIX) {
-      if (clock64() - tw > WAIT_LIMIT || *reinterpret_cast<volatile unsigned int*>(&s.err)) {
+      if (clock64() - tw > s.wait_limit || *reinterpret_cast<volatile unsigned int*>(&s.err)) {
         atomicOr(&s.err, 1u);
         break;
       }
       __nanosleep(200);
     }
   }
-  FixEntry* dst = &g_fix_ring[blockIdx.x][slot % QCAP];
+  FixEntry* dst = &g_fix_ring[s.ring][slot % QCAP];
   dst->tile = E.tile;
   dst->r = E.r;
   dst->kind = E.kind;
@@ -981,6 +1010,7 @@ __device__ __noinline__ void role_conv(const PArgs& a, uint32_t tmem, int n_tile
     }
     // ---- the epilogue has staged the codes of tile ut: copy the tile out ----
     if (!pwait_w(s, &s.fw, ut & 1)) break;
+    if (ut == 0) wait_prior_grid();
     if (r < nt && (smk[0] | smk[1] | smk[2] | smk[3])) {
       FixEntry E;
       E.tile = (uint32_t)tile;
@@ -1166,12 +1196,13 @@ __device__ __noinline__ void role_epi(const PArgs& a, uint32_t tmem, int n_tiles
 template <int KB, int VB>
 __device__ __noinline__ void role_fix(const PArgs& a) {
   PSmem& s = smem();
+  wait_prior_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int w = warp - W_FIX;
   unsigned int k = (unsigned)w, seen = 0, done_count = 0;
   long long t_last = clock64();
   while (true) {
-    const FixEntry* src = &g_fix_ring[blockIdx.x][k % QCAP];
+    const FixEntry* src = &g_fix_ring[s.ring][k % QCAP];
     const unsigned int stored = ld_acq(&s.stored_seq);
     if (*reinterpret_cast<const volatile uint64_t*>(&src->tag) == fix_tag(s, k)) {
       __threadfence_block();
@@ -1195,11 +1226,117 @@ __device__ __noinline__ void role_fix(const PArgs& a) {
     if (stored != seen) {
       seen = stored;
       t_last = clock64();
-    } else if (clock64() - t_last > WAIT_LIMIT) {
+    } else if (clock64() - t_last > s.wait_limit) {
       atomicOr(&s.err, 1u);
       break;
     }
     __nanosleep(500);
+  }
+}
+
+// Cooperative fp64 re-derivation of the deferred key rows, by all 512 threads once every role has
+// finished (the rows are in global memory; no other fixup touches them any more).  Per row: the
+// exact norm; u_j = sqrt(128) (Pi x)_j / ||x|| by four threads per coordinate, then its code and
+// rho_j; (S rho)_l by four threads per sketch row; then the row's codes, signs and ||r||.
+template <int KB, int VB>
+__device__ __noinline__ void coop_slow_rows(const PArgs& a) {
+  PSmem& s = smem();
+  constexpr int LK = 1 << KB;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = tid & 3, j = tid >> 2;  // quarter of a dot product, coordinate / sketch row
+  const double sqd = sqrt((double)D);
+  const int n = min((int)s.n_slow, SLOW_CAP);
+  double* x = s.frho[0];
+  double* rho = s.frho[1];
+  for (int i = 0; i < n; ++i) {
+    const uint32_t tile = s.slow[i][0];
+    const int r = (int)(s.slow[i][1] & 0xffffu);
+    const bool code_changed = (s.slow[i][1] >> 16) != 0;
+    const int bh = (int)(tile / (uint32_t)a.tiles_per_bh);
+    const int t = (int)(tile % (uint32_t)a.tiles_per_bh) * TM + r;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const int64_t in_off = (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)t * a.st;
+    const int64_t row = ((int64_t)b * a.Hkv + h) * a.T_cap + a.t_offset + t;
+    // 1. the input row in fp64 and ||x||^2 (warps 0 and 1)
+    if (tid < 64) {
+      const uint32_t w2 = reinterpret_cast<const uint32_t*>(a.k + in_off)[tid];
+      const double x0 = (double)__uint_as_float(w2 << 16), x1 = (double)__uint_as_float(w2 & 0xffff0000u);
+      x[2 * tid] = x0;
+      x[2 * tid + 1] = x1;
+      const double ss = warp_sum(fma(x0, x0, x1 * x1));
+      if (lane == 0) s.cred[warp] = ss;
+    }
+    __syncthreads();
+    const double nk = sqrt(s.cred[0] + s.cred[1]);
+    // 2. exact u, code and rho of coordinate j
+    {
+      const float4* pr = reinterpret_cast<const float4*>(a.Pi + j * D + 32 * q);
+      double acc = 0.0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 p = pr[k];
+        const double* xv = x + 32 * q + 4 * k;
+        acc = fma((double)p.x, xv[0], acc);
+        acc = fma((double)p.y, xv[1], acc);
+        acc = fma((double)p.z, xv[2], acc);
+        acc = fma((double)p.w, xv[3], acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      double r2 = 0.0;
+      if (q == 0) {
+        const double u = nk > 0.0 ? sqd * acc / nk : 0.0;
+        const uint32_t code = nk > 0.0 ? code_lut(u, s.klut, s.alpha_k) : (uint32_t)(LK / 2);
+        const double rh = u - (double)s.kcent[code];
+        rho[j] = rh;
+        s.fcode[0][k_slot_of_coord(j)] = (uint8_t)code;
+        r2 = rh * rh;
+      }
+      r2 = warp_sum(r2);
+      __syncthreads();  // every thread has read x and cred[0..1]
+      if (lane == 0) s.cred[warp] = r2;
+    }
+    __syncthreads();
+    // 3. exact sketch value of row j, and its sign bit
+    {
+      const float4* sr = reinterpret_cast<const float4*>(a.S + j * D + 32 * q);
+      double acc = 0.0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 p = sr[k];
+        const double* rv = rho + 32 * q + 4 * k;
+        acc = fma((double)p.x, rv[0], acc);
+        acc = fma((double)p.y, rv[1], acc);
+        acc = fma((double)p.z, rv[2], acc);
+        acc = fma((double)p.w, rv[3], acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (q == 0) {
+        s.fsign[0][sign_bit_of_row(j)] = acc >= 0.0 ? 1 : 0;
+        if (fabs(acc) <= kExemptSignBand) atomicAdd(&g_pipe_exempt_signs, 1u);
+      }
+    }
+    __syncthreads();
+    // 4. the row's codes, signs and ||r||
+    if (tid < 4 * KB) {
+      uint32_t word = 0;
+      for (int kk = 0; kk < 32; ++kk) {
+        const int P = 32 * tid + kk;
+        word |= (uint32_t)((s.fcode[0][P / KB] >> (P % KB)) & 1) << kk;
+      }
+      reinterpret_cast<uint32_t*>(a.k_codes + row * (16 * KB))[tid] = word;
+    } else if (tid >= 32 && tid < 36) {
+      const int w = tid - 32;
+      uint32_t word = 0;
+      for (int kk = 0; kk < 32; ++kk) word |= (uint32_t)s.fsign[0][32 * w + kk] << kk;
+      reinterpret_cast<uint32_t*>(a.k_signs + row * 16)[w] = word;
+    } else if (tid == 64 && code_changed) {  // (otherwise the fast ||r||, from the same codes, stays)
+      double q2 = 0.0;
+      for (int w = 0; w < THREADS / 32; ++w) q2 += s.cred[w];
+      a.k_rnorm[row] = (float)(nk * sqrt(q2) / sqd);
+    }
+    __syncthreads();  // scratch reused by the next row
   }
 }
 
@@ -1209,15 +1346,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                          const __grid_constant__ CUtensorMap tmv) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   PSmem& s = *reinterpret_cast<PSmem*>(smem_raw);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int LK = 1 << KB, LV = 1 << VB;
   if ((smem_u32(smem_raw) & 1023u) != 0) {
-    if (tid == 0) {
-      atomicOr(&g_pipe_error, 2u);
-      count_cta_done();
-    }
+    if (tid == 0) atomicOr(&g_pipe_error, 2u);
     return;
   }
+  // the next quantize launch of this stream may start its prologue and loads now (it waits for
+  // this grid before its first global store)
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int n_tiles = (int)((a.total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
 
   // ---- prologue ----
@@ -1244,12 +1381,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     s.q_tail = 0;
     s.stored_seq = 0;
     s.main_done = 0;
-    s.epoch = *reinterpret_cast<volatile unsigned int*>(&g_pipe_epoch);
+    const uint32_t smid = sm_id();
+    s.ring = smid < MAX_SMS ? smid : 0u;
+    s.epoch = atomicAdd(&g_ring_gen[s.ring], 1u) + 1u;
+    if (smid >= MAX_SMS) s.err |= 8u;  // (never on sm_100: 148 SMs)
     s.pi_lo = 0;
+    s.n_slow = 0;
+    s.wait_limit = a.wait_limit;
     for (int i = 0; i < N_FIX; ++i) s.fix_done[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   __syncthreads();
+  // the first tile's K and V (and the next K) start loading before the operands are staged
+  const int pre = min(SLOTS, 2 * n_tiles);
+  if (warp == W_TMA && lane == 0 && s.err == 0)
+    for (int L = a.stall_first_load ? 1 : 0; L < pre; ++L) issue_load(a, &tmk, &tmv, L);
   if (tid < LK) s.kcent[tid] = a.kc[tid];
   if (tid < LK - 1) s.kthr[tid] = a.kt[tid];
   if (tid < LV) s.vcent[tid] = a.vc[tid];
@@ -1264,17 +1410,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (s.err & 4u) {  // no usable cell width for this codebook (never for Lloyd-Max grids of 2..4 bits)
-    if (tid == 0) {
-      atomicOr(&g_pipe_error, 4u);
-      count_cta_done();
-    }
+  if (s.err & 12u) {  // no usable cell width for this codebook (never for Lloyd-Max grids of 2..4
+                      // bits), or an SM number outside the ring table (never on sm_100)
+    if (warp == W_TMA && lane == 0)  // loads issued above land before the CTA exits
+      for (int L = 0; L < (s.err & 8u ? 0 : pre); ++L) {
+        const long long t0 = clock64();
+        while (!mbar_test(&s.full[L % SLOTS], 0) && clock64() - t0 < s.wait_limit) {
+        }
+      }
+    if (tid == 0) atomicOr(&g_pipe_error, s.err & 12u);
     if (warp == W_MMA) tmem_dealloc(s.tmem_base, TMEM_COLS);
     return;
   }
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == W_TMA) role_tma(a, &tmk, &tmv, n_tiles);
+  if (warp == W_TMA) role_tma(a, &tmk, &tmv, n_tiles, pre);
   else if (warp == W_MMA) role_mma(a, tmem, n_tiles);
   else if (warp < N_CONV_WARPS) role_conv<KB, VB>(a, tmem, n_tiles);
   else if (warp >= W_EPI && warp < W_EPI + N_EPI_WARPS) role_epi<KB, VB>(a, tmem, n_tiles);
@@ -1283,14 +1433,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0) {
-    if (s.err) atomicOr(&g_pipe_error, s.err);
-    count_cta_done();
+  if (s.n_slow && !s.err) {
+    wait_prior_grid();
+    coop_slow_rows<KB, VB>(a);
   }
+  if (tid == 0 && s.err) atomicOr(&g_pipe_error, s.err);
   if (warp == W_MMA) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // ---------------------------------------------------------------------------------------------
+// Test hook (tq_debug_quantize_stall): host-side settings read at each launch.
+std::atomic<int> g_test_stall{0};
+std::atomic<long long> g_test_wait_cycles{0};
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1334,8 +1489,19 @@ tq_status launch_kv(const PArgs& a, const CUtensorMap& mk, const CUtensorMap& mv
   cudaError_t err = cudaFuncSetAttribute(quantize_pipe_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(err));
-  quantize_pipe_kernel<KB, VB><<<grid, THREADS, smem, stream>>>(a, mk, mv);
-  err = cudaGetLastError();
+  // programmatic dependent launch: when the previous kernel of the stream is a quantize launch
+  // (consecutive chunks), this one's prologue and first loads overlap its tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, quantize_pipe_kernel<KB, VB>, a, mk, mv);
   if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "quantize launch: %s", cudaGetErrorString(err));
   return TQ_OK;
 }
@@ -1384,6 +1550,9 @@ tq_status quantize_bf16_pipeline(const tq_params* p, const void* k, const void* 
   // |S rho| error <= 8e-6 measured.  The bands are wider.
   a.band_code = 4e-6f;
   a.band_sign = 3e-5f;
+  const long long wl = g_test_wait_cycles.load();
+  a.wait_limit = wl > 0 ? wl : WAIT_LIMIT;
+  a.stall_first_load = g_test_stall.load() ? 1 : 0;
   const int grid = (int)std::min<int64_t>(a.total_tiles, std::min(sms, MAX_CTAS));
   *handled = true;
   const int kb = c->k_bits, vb = c->v_bits;
@@ -1415,6 +1584,14 @@ long long pipe_code_fixups() {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_pipe_code_fixups, sizeof(v)) != cudaSuccess) return -1;
   return v;
+}
+void pipe_set_test_stall(int enable, long long wait_cycles) {
+  g_test_stall = enable ? 1 : 0;
+  g_test_wait_cycles = enable ? wait_cycles : 0;
+}
+int pipe_reset_errors() {
+  const unsigned int z = 0;
+  return cudaMemcpyToSymbol(g_pipe_error, &z, sizeof(z)) == cudaSuccess ? 0 : -1;
 }
 long long pipe_exempt_codes() {
   unsigned int v = 0;

@@ -107,8 +107,26 @@ tq_status tq_build_codebook(int bits, int max_iter, double tol, float* centroids
  */
 tq_status tq_build_hadamard_rotation(uint64_t seed, float* Pi);
 
+/* Cache layouts (tq_cache.layout). */
+enum { TQ_LAYOUT_PLAIN = 0, TQ_LAYOUT_MIXED = 1 };
+
 /* Caller-owned packed cache (device pointers; see the layout above).  k_signs and k_rnorm may
- * be NULL when qjl_m == 0. */
+ * be NULL when qjl_m == 0.
+ *
+ * layout = TQ_LAYOUT_MIXED: outlier-aware mixed precision.  Source: tproger.ru, section on
+ * TheTom's llama.cpp fork (turbo3 = 3.5-bit KV quantization, 4.6x vs FP16); ai-manual.ru M5 Max
+ * KV-cache benchmark (per-layer outlier-aware 3/4-bit quantization).  The channels split into an
+ * outlier half O (tq_params.outlier_mask, 64 channels) coded with k_bits / v_bits and the other
+ * half R coded with one bit less; each half is rotated on its own (tq_params.Pi must be the block
+ * rotation: rows 0..63 act only on the outlier channels, rows 64..127 only on the others), has its
+ * own norm and codebook (tq_params.*_lo for half R), u_g = sqrt(64) (Pi x)_g / ||x_g||.  QJL acts
+ * on the whole residual r = Pi x - khat (khat_g = ||x_g|| / 8 * c_g[idx_g]): k_rnorm = ||r||, and
+ * a sign bit is 1 when (S r)_l >= 0.  Supported: k_bits = v_bits = 4 (halves of 4 and 3 bits).
+ *   k_codes row: the half-O bit stream (64 codes of k_bits bits; coordinate 16a + 8h + 2t + e at
+ *     slot 16t + 4a + 2h + e), then the half-R stream (64 codes of k_bits - 1 bits, coordinate
+ *     64 + 16a + 8h + 2t + e at slot 16t + 4a + 2h + e): 8 (2 k_bits - 1) bytes.
+ *   v_codes row: likewise with value slots (coordinate 64g' + 8n + g at slot 8g + n of half g').
+ *   k_norm, v_norm: float [.., 2] = (||x_O||, ||x_R||). */
 typedef struct {
   int B, Hkv, T_cap, head_dim, k_bits, v_bits, qjl_m;
   uint8_t* k_codes;
@@ -117,6 +135,7 @@ typedef struct {
   float* k_rnorm;
   uint8_t* v_codes;
   float* v_norm;
+  int layout;  /* TQ_LAYOUT_PLAIN or TQ_LAYOUT_MIXED */
 } tq_cache;
 
 /* Per-layer constants (device pointers, caller-owned, fp32 unless stated).
@@ -138,6 +157,14 @@ typedef struct {
   const float* v_centroids;
   const float* v_thresholds;
   const double* S_Pi;
+  /* TQ_LAYOUT_MIXED only (ignored otherwise): codebooks of the non-outlier half (one bit fewer),
+   * device fp32 like the ones above, and the outlier channels (bit c of outlier_mask[c / 32] set
+   * for channel c in O; exactly 64 bits set). */
+  const float* k_centroids_lo;
+  const float* k_thresholds_lo;
+  const float* v_centroids_lo;
+  const float* v_thresholds_lo;
+  uint32_t outlier_mask[4];
 } tq_params;
 
 /*
@@ -200,8 +227,25 @@ long long tq_quantize_exempt_codes(void);
 long long tq_quantize_exempt_signs(void);
 
 /*
+ * Clear the error bits that tq_quantize_device_errors and tq_decode_device_errors report (host;
+ * synchronizes with the device).  Returns 0, or -1 if the device could not be reached.
+ */
+int tq_reset_device_errors(void);
+
+/*
+ * Test hook for the failure handling of tq_quantize (bf16 inputs): while enabled, every CTA of a
+ * launch skips its first tile load and every wait of the kernel gives up after `wait_cycles` SM
+ * cycles instead of about two seconds.  The waits then run out one after another, the kernel
+ * records bit 0 in tq_quantize_device_errors, releases its tensor memory and returns; the cache
+ * rows of that launch are not valid.  enable = 0 restores normal operation.  Host-side setting,
+ * read at each launch; not for concurrent use with other callers of tq_quantize.
+ * Errors: TQ_ERR_INVALID_ARG (enable with wait_cycles <= 0).
+ */
+tq_status tq_debug_quantize_stall(int enable, long long wait_cycles);
+
+/*
  * Bytes of device workspace tq_decode_attn needs for these sizes on the current device
- * (split-K partials plus the rotated queries).  Returns 0 on invalid sizes.
+ * (the split-K partials).  Returns 0 on invalid sizes.
  */
 size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_len);
 

@@ -148,13 +148,14 @@ def compare_full_cache(w: W.Workload, cache: tq.Cache, K: torch.Tensor, V: torch
     return total
 
 
-def exemption_free_inputs(w: W.Workload, spare: int = 64):
+def exemption_free_inputs(w: W.Workload, spare: int = 64, mixed=None):
     """K, V of the workload's recipe ([B, Hkv, T, 128], input dtype, CPU) in which no vector has a
     coordinate within the code band of a threshold or a sketch value within the sign band of 0:
     the recipe is drawn with T + spare tokens and, per (batch, kv-head), the first T vectors whose
     K and V are both free of exempt cases are kept (about 0.3% of vectors are skipped).  On such
     inputs the cache has exactly one correct value, so a GPU-written cache and the decode over it
-    can be compared with the oracle without exceptions."""
+    can be compared with the oracle without exceptions.  mixed = (outlier channels, block
+    rotation): the exemptions of the mixed layout instead."""
     big = w.scaled(T=w.T + spare)
     K = W.make_kv(big, "k")
     V = W.make_kv(big, "v")
@@ -163,9 +164,15 @@ def exemption_free_inputs(w: W.Workload, spare: int = 64):
     Vo = torch.empty_like(Ko)
     for b in range(w.B):
         for h in range(w.Hkv):
-            kq = O.quantize_vectors(K[b, h].double().numpy(), Pi, w.k_bits, S)
-            vq = O.quantize_vectors(V[b, h].double().numpy(), Pi, w.v_bits, None)
-            bad = O.code_exempt(kq["u"], w.k_bits).any(1) | O.code_exempt(vq["u"], w.v_bits).any(1)
+            if mixed is None:
+                kq = O.quantize_vectors(K[b, h].double().numpy(), Pi, w.k_bits, S)
+                vq = O.quantize_vectors(V[b, h].double().numpy(), Pi, w.v_bits, None)
+                bad = O.code_exempt(kq["u"], w.k_bits).any(1) | O.code_exempt(vq["u"], w.v_bits).any(1)
+            else:
+                oc, P = mixed
+                kq = O.quantize_vectors_mixed(K[b, h].double().numpy(), P, oc, 4, 3, S)
+                vq = O.quantize_vectors_mixed(V[b, h].double().numpy(), P, oc, 4, 3, None)
+                bad = O.code_exempt_mixed(kq["u"], 4, 3).any(1) | O.code_exempt_mixed(vq["u"], 4, 3).any(1)
             if S is not None:
                 bad |= (np.abs(kq["sproj"]) <= O.SIGN_BAND).any(1)
             keep = np.flatnonzero(~bad)[: w.T]
@@ -173,6 +180,51 @@ def exemption_free_inputs(w: W.Workload, spare: int = 64):
             Ko[b, h] = K[b, h, torch.as_tensor(keep)]
             Vo[b, h] = V[b, h, torch.as_tensor(keep)]
     return Ko, Vo
+
+
+def mixed_setup(w: W.Workload):
+    """Constants of the outlier-aware mixed layout for a workload: outlier channels from its
+    scale draw, the block rotation of those channels, the sketch."""
+    oc = W.outlier_channels_for(w)
+    return oc, W.make_block_rotation(1000 + w.seed, oc), W.qjl_for(w)
+
+
+def compare_rows_mixed(w: W.Workload, cache: tq.Cache, kx, vx, bi, hi, ti, oc, P) -> dict:
+    """compare_rows for the mixed layout (4-bit outlier half, 3-bit other half): codes, signs,
+    both norms of each row and ||r|| against the oracle's mixed quantization."""
+    S = W.qjl_for(w)
+    kx, vx = np.asarray(kx, np.float64), np.asarray(vx, np.float64)
+    kq = O.quantize_vectors_mixed(kx, P, oc, 4, 3, S)
+    vq = O.quantize_vectors_mixed(vx, P, oc, 4, 3, None)
+    dev = cache.k_codes.device
+    ib, ih, it = (torch.as_tensor(np.asarray(x), device=dev) for x in (bi, hi, ti))
+    g = lambda t: t[ib, ih, it].cpu().numpy()
+    out = {"vectors": int(kx.shape[0]), "coords": int(2 * kx.shape[0] * 128)}
+    for name, q, codes, slot in (("k", kq, g(cache.k_codes), O.k_slot_of_coord_mixed),
+                                 ("v", vq, g(cache.v_codes), O.v_slot_of_coord_mixed)):
+        ex = O.code_exempt_mixed(q["u"], 4, 3)
+        got = O.unpack_codes_mixed(codes, 4, 3, slot)
+        diff = got != q["idx"]
+        assert not (diff & ~ex).any(), f"{name} codes differ outside the exemption band at {np.argwhere(diff & ~ex)[:5]}"
+        clean = ~ex.any(1)
+        assert np.array_equal(codes[clean], O.pack_codes_mixed(q["idx"], 4, 3, slot)[clean])
+        out[name + "_exempt"] = int(ex.sum())
+        out[name + "_mismatch_in_band"] = int(diff.sum())
+        norms = g(cache.k_norm if name == "k" else cache.v_norm)
+        assert ulp_distance_f32(norms[:, 0], q["n_O"].astype(np.float32)).max() <= NORM_ULP
+        assert ulp_distance_f32(norms[:, 1], q["n_R"].astype(np.float32)).max() <= NORM_ULP
+    k_ex = O.code_exempt_mixed(kq["u"], 4, 3)
+    s_ex = O.sign_exempt(kq["sproj"], k_ex)
+    signs = O.unpack_signs(g(cache.k_signs))
+    sd = signs != kq["signs"]
+    assert not (sd & ~s_ex).any(), f"sign bits differ outside the exemption band at {np.argwhere(sd & ~s_ex)[:5]}"
+    rn = g(cache.k_rnorm).astype(np.float64)
+    clean = ~k_ex.any(1)
+    err = np.abs(rn - kq["rnorm"])[clean]
+    assert (err <= 1e-5 * kq["rnorm"][clean] + 1e-30).all(), (err / np.maximum(kq["rnorm"][clean], 1e-30)).max()
+    out["exempt_codes"] = out["k_exempt"] + out["v_exempt"]
+    out["exempt_signs"] = int(s_ex.sum())
+    return out
 
 
 def attention_errors(got: np.ndarray, ref: np.ndarray):
@@ -202,5 +254,6 @@ def oracle_cache_arrays(w: W.Workload, Kh, Vh, T_cap=None):
 
 __all__ = ["ATTN_MAX_ABS", "ATTN_REL_L2", "EXEMPT_FRACTION_MAX", "ulp_distance_f32", "gpu_inputs",
            "params_for", "compare_rows", "compare_quantized", "compare_full_cache", "merge_counts",
+           "mixed_setup", "compare_rows_mixed",
            "exemption_free_inputs", "attention_errors", "assert_attention_close",
            "oracle_cache_arrays", "math", "torch"]

@@ -115,7 +115,7 @@ def test_workspace_size():
     c = fake_cache()
     L = tq.lib()
     n = L.tq_decode_workspace_size(1, 8, ctypes.byref(c), 64)
-    assert n >= 4 * (2 * 8 * 128 + 8 * 130)
+    assert n >= 4 * 8 * 132  # at least one (max, sum, pad, pad, o[128]) partial per query head
     assert L.tq_decode_workspace_size(1, 7, ctypes.byref(c), 64) == 0
     assert L.tq_decode_workspace_size(1, 8, None, 64) == 0
     big = L.tq_decode_workspace_size(4, 32, ctypes.byref(fake_cache(B=4, Hkv=8, T_cap=131072)), 131072)
@@ -152,3 +152,11 @@ def test_sketch_rotation_and_hadamard_builder_argument_errors():
     assert L.tq_sketch_rotation(FAKE, FAKE, 0, FAKE, None) == tq.TQ_ERR_INVALID_ARG
     assert L.tq_build_hadamard_rotation(1, None) == tq.TQ_ERR_INVALID_ARG
     assert quantize_status(params=fake_params(S_Pi=FAKE + 8)) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_debug_quantize_stall_argument_check():
+    """The failure-handling test hook refuses a non-positive wait limit (no device needed)."""
+    L = tq.lib()
+    assert L.tq_debug_quantize_stall(1, 0) == tq.TQ_ERR_INVALID_ARG
+    assert "wait_cycles" in tq.last_error()
+    assert L.tq_debug_quantize_stall(0, 0) == tq.TQ_OK

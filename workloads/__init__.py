@@ -60,6 +60,7 @@ class Workload:
     chunk: int  # streaming-quantize chunk length (tokens); T = one chunk
     head_dim: int = HEAD_DIM
     rotation: str = "haar"  # "haar" (dense Haar-random) | "hadamard" (D1 H D2 H D3 / d)
+    layout: str = "plain"   # "plain" | "mixed" (outlier half at k_bits / v_bits, the rest one bit fewer)
 
     @property
     def group(self) -> int:
@@ -81,11 +82,15 @@ class Workload:
         )
 
     # compressed bytes per token per kv-head (codes + signs + norms)
+    def _code_bytes(self, bits: int) -> int:
+        return 8 * (2 * bits - 1) if self.layout == "mixed" else 16 * bits
+
     def k_row_bytes(self) -> int:
-        return 16 * self.k_bits + (16 + 4 if self.qjl_m else 0) + 4
+        nb = 8 if self.layout == "mixed" else 4
+        return self._code_bytes(self.k_bits) + (16 + 4 if self.qjl_m else 0) + nb
 
     def v_row_bytes(self) -> int:
-        return 16 * self.v_bits + 4
+        return self._code_bytes(self.v_bits) + (8 if self.layout == "mixed" else 4)
 
     def decode_bytes(self, seq_len: Optional[int] = None) -> int:
         T = self.T if seq_len is None else seq_len
@@ -204,6 +209,8 @@ def outlier_channels_for(w: Workload, count: int = HEAD_DIM // 2) -> np.ndarray:
 
 
 def rotation_for(w: Workload) -> np.ndarray:
+    if w.layout == "mixed":
+        return make_block_rotation(1000 + w.seed, outlier_channels_for(w), w.head_dim)
     if w.rotation == "hadamard":
         return make_hadamard_rotation(1000 + w.seed, w.head_dim)
     assert w.rotation == "haar", w.rotation
