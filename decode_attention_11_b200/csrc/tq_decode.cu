@@ -7,16 +7,17 @@
 // Softmax and the value sum also run in the rotated basis; one final o = Pi^T o' per head.
 //
 // Kernels (on the caller's stream; merge is a programmatic dependent of split):
-//   split   one persistent CTA per SM over an even share of all (unit, token) pairs.  At the start of
-//           each segment the CTA computes q' = Pi q and sq = S q' of the unit's heads in fp32 (shared
-//           memory).  A producer warp streams stages of the packed cache into a ring of
-//           shared-memory slots with bulk copies (mbarrier completion); 11 (7 for groups of 5-8
-//           heads) consumer warps take 16 tokens each per stage: codes become fp16 pairs through a
-//           lane-replicated shared-memory table (one permute + one load per two coordinates), and
-//           m16n8k16 tensor-core MMAs compute q'.khat, the QJL sign dot (sign bits placed in fp16
-//           mantissas by a shift and one logic op, B rows pre-scaled to match) and P.vhat (P split
-//           into fp16 hi + lo).  Online softmax runs in log2 units; each segment ends with one
-//           (max, sum, o'[128]) partial per head.
+//   split   one persistent CTA per SM over an even share of all (unit, token) pairs.  Up front the
+//           CTA computes q' = Pi q and sq = S q' of the heads of its first four segments in fp32
+//           (shared memory), while a producer warp already streams stages of the packed cache into
+//           a ring of shared-memory slots with bulk copies (mbarrier completion).  11 (7 for groups
+//           of 5-8 heads) consumer warps take 16 tokens each per stage: codes become fp16 pairs
+//           through a lane-replicated shared-memory table (one permute + one load per two
+//           coordinates), and m16n8k16 tensor-core MMAs compute q'.khat, the QJL sign dot (sign bits
+//           placed in fp16 mantissas by a shift and one logic op, B rows pre-scaled to match) and
+//           P.vhat (P split into fp16 hi + lo).  Online softmax runs in log2 units; at a segment's
+//           end every consumer warp writes its own (max, sum, o'[128]) partial per head, so no
+//           barrier stops the CTA between segments.
 //   merge   one CTA per (batch, query head): log-sum-exp merge of the head's partials, then
 //           o = Pi^T o'.
 #include <cuda_bf16.h>
@@ -156,6 +157,7 @@ struct Shape {
   static constexpr int ST = 16 * NW;        // tokens per stage
 };
 constexpr int NS_MAX = 8;                   // ring slots
+constexpr int NSEG_PRE = 2;                 // segments whose query prep is computed in one pass
 constexpr int MIN_TOK_PER_CTA = 256;        // fewer CTAs than SMs below this much work each
 constexpr int CTRL_BYTES = 256;             // mbarriers, slot offsets, flags (end of dynamic smem)
 constexpr long long WAIT_LIMIT = 4000000000LL;  // ~2 s of SM clock per wait
@@ -194,7 +196,7 @@ __device__ unsigned int g_decode_error;  // bit 0: a wait timed out; bit 1: shar
 // table, the 3-bit halves two more 64-entry tables.
 template <int KB, int VB, bool QJL, int NB, bool MX = false>
 struct Layout {
-  static constexpr int NW = Shape<NB>::NW, ST = Shape<NB>::ST, HGN = 4 * NB;
+  static constexpr int ST = Shape<NB>::ST, HGN = 4 * NB;
   static constexpr int K_ROW = MX ? 8 * (2 * KB - 1) : 16 * KB;
   static constexpr int V_ROW = MX ? 8 * (2 * VB - 1) : 16 * VB;
   static constexpr int NORM = MX ? 8 : 4;  // norm bytes per token
@@ -212,10 +214,14 @@ struct Layout {
   static constexpr int V_TBL = kPacked ? 0 : (1 << (2 * VB)) * 128;
   static constexpr int TBL_BYTES = kPacked ? 65536 : K_TBL + V_TBL;
   static constexpr int TBL2_BYTES = MX ? 2 * 64 * 128 : 0;  // 3-bit K and V pair tables
-  // per-warp (max, sum) and o' of the 4 NB heads, for the merge of the warps at a segment's end
-  static constexpr int MERGE_BYTES_W = 4 * (NW * HGN * 2 + NW * HGN * D);
-  static constexpr int PREP_BYTES = 4 * 3 * HGN * D;  // query prep at a segment's start
-  static constexpr int MERGE_BYTES = MERGE_BYTES_W > PREP_BYTES ? MERGE_BYTES_W : PREP_BYTES;
+  // query prep of NSEG_PRE segments: q' and S q' of their heads (the raw q is staged in the
+  // latter), 64 codebook floats, the MMA B fragments of every lane ([segment][n-block][word / 4]
+  // [lane][word % 4], 32 words) and (fK, fQ, Kh, 2^-e) per head
+  static constexpr int FRAG_WORDS = NSEG_PRE * NB * 32 * 32;
+  static constexpr int PREP_BYTES = 4 * (2 * NSEG_PRE * HGN * D + 64 + FRAG_WORDS + NSEG_PRE * HGN * 4);
+  // the merge of the warps at the CTA's last segment end, one n-block at a time, in ring memory:
+  // (max, sum) and o' of four heads per warp
+  static constexpr int MERGE_BYTES = 4 * (Shape<NB>::NW * 4 * 2 + Shape<NB>::NW * 4 * D);
   static_assert(STAGE_BYTES % 16 == 0 && OFF_SG % 16 == 0 && OFF_VC % 16 == 0 && OFF_NK % 16 == 0,
                 "bulk-copy granularity");
   static_assert(MX || (K_ROW % 16 == 0 && V_ROW % 16 == 0), "bulk-copy granularity");
@@ -229,7 +235,8 @@ struct Ctrl {
   uint32_t stage_off[NS_MAX];  // byte offsets of the ring slots from the start of dynamic smem
   uint32_t tbl_addr;           // shared-window address of the pair tables
   uint32_t tbl2_addr;          // mixed layout: the 3-bit pair tables
-  uint32_t merge_off;
+  uint32_t prep_off;
+  uint32_t merge_off;          // the warps' merge area at the CTA's end (inside the ring)
   int ns;
   unsigned int err;
 };
@@ -386,8 +393,10 @@ __device__ __forceinline__ uint32_t v_pair(const PairLut<KB, VB>& L, const VPair
 }
 
 // Shared-memory plan, computed by one thread: the pair tables (at a 64 KB boundary for the packed
-// tables), the warp-merge area and as many ring slots as fit around them.  ns = 0 when the slots
-// do not fit (never with the 227 KB of an sm_100 CTA).
+// tables) split the rest into two free regions; the most ring slots (up to NS_MAX) are placed
+// first-fit such that the query-prep area (and the mixed layout's second tables) still fit around
+// them.  The warps' merge at the CTA's end goes into adjacent ring slots.  ns = 0 when nothing
+// fits (never with the 227 KB of an sm_100 CTA).
 template <int KB, int VB, bool QJL, int NB, bool MX>
 __device__ void plan_smem(unsigned char* smem, int dyn, Ctrl& c) {
   using Lay = Layout<KB, VB, QJL, NB, MX>;
@@ -395,41 +404,47 @@ __device__ void plan_smem(unsigned char* smem, int dyn, Ctrl& c) {
   const uint32_t end = base + (uint32_t)dyn - CTRL_BYTES;
   const uint32_t tbl = Lay::kPacked ? ((base + 0xFFFFu) & ~0xFFFFu) : base;
   c.tbl_addr = tbl;
-  // free regions: [base, tbl) and [tbl + TBL_BYTES, end)
-  uint32_t r0 = base, r0e = tbl, r1 = tbl + Lay::TBL_BYTES, r1e = end;
-  if (r1 > end) {
-    c.ns = 0;
+  c.ns = 0;
+  if (tbl + Lay::TBL_BYTES > end) return;
+  for (int ns = NS_MAX; ns >= 2; --ns) {
+    // free regions: [base, tbl) and [tbl + TBL_BYTES, end)
+    uint32_t r0 = base, r0e = tbl, r1 = tbl + Lay::TBL_BYTES, r1e = end;
+    auto take = [&](uint32_t bytes, uint32_t& off) -> bool {
+      if (r0e - r0 >= bytes) {
+        off = r0 - base;
+        r0 += bytes;
+        return true;
+      }
+      if (r1e - r1 >= bytes) {
+        off = r1 - base;
+        r1 += bytes;
+        return true;
+      }
+      return false;
+    };
+    bool ok = true;
+    for (int i = 0; i < ns && ok; ++i) ok = take(Lay::STAGE_BYTES, c.stage_off[i]);
+    uint32_t off = 0;
+    ok = ok && take(Lay::PREP_BYTES, off);
+    c.prep_off = off;
+    if (ok && Lay::TBL2_BYTES) {
+      ok = take(Lay::TBL2_BYTES, off);
+      c.tbl2_addr = base + off;
+    }
+    if (!ok) continue;
+    // the warps' merge at the CTA's end reuses ring memory: a run of adjacent slots large enough
+    c.merge_off = 0xFFFFFFFFu;
+    for (int k = 0; k < ns && c.merge_off == 0xFFFFFFFFu; ++k) {
+      uint32_t run = Lay::STAGE_BYTES;
+      for (int i = k + 1; i < ns && run < (uint32_t)Lay::MERGE_BYTES &&
+                          c.stage_off[i] == c.stage_off[i - 1] + Lay::STAGE_BYTES; ++i)
+        run += Lay::STAGE_BYTES;
+      if (run >= (uint32_t)Lay::MERGE_BYTES) c.merge_off = c.stage_off[k];
+    }
+    if (c.merge_off == 0xFFFFFFFFu) continue;
+    c.ns = ns;
     return;
   }
-  auto take = [&](uint32_t bytes, uint32_t& off) -> bool {
-    if (r0e - r0 >= bytes) {
-      off = r0 - base;
-      r0 += bytes;
-      return true;
-    }
-    if (r1e - r1 >= bytes) {
-      off = r1 - base;
-      r1 += bytes;
-      return true;
-    }
-    return false;
-  };
-  uint32_t off = 0;
-  if (!take(Lay::MERGE_BYTES, off)) {
-    c.ns = 0;
-    return;
-  }
-  c.merge_off = off;
-  if (Lay::TBL2_BYTES) {
-    if (!take(Lay::TBL2_BYTES, off)) {
-      c.ns = 0;
-      return;
-    }
-    c.tbl2_addr = base + off;
-  }
-  int ns = 0;
-  while (ns < NS_MAX && take(Lay::STAGE_BYTES, off)) c.stage_off[ns++] = off;
-  c.ns = ns >= 2 ? ns : 0;
 }
 
 template <int KB, int VB, bool QJL, int NB, bool MX>
@@ -525,16 +540,248 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
   }
 
   // ================================================================ consumers (warps 0 .. NW-1)
-  // Pair tables: entry e = lo | hi << b -> half2(c[lo], c[hi]), four lane replicas per 16-byte store.
+  // Prologue: q' = Pi q and sq = S q' of the heads of the CTA's first NSEG_PRE segments (fp32, the
+  // prep area [NSEG_PRE][HGN][D] each; the raw q is staged where sq goes) and the pair tables.
+  // Every global load it needs is issued first, so they share one memory round trip: the
+  // thread's half-row of Pi (task (row, half) = (tid / 2, tid % 2)), its share of the queries and
+  // one codebook entry; S is prefetched into L2 and read after the first pass.  Tasks tid + 32 NW,
+  // ... (seven consumer warps: warp 0 takes the last 32) load their rows when they get to them; the
+  // two halves of a row are always in one warp.
+  float* qpm = reinterpret_cast<float*>(smem + ctl.prep_off);
+  float* sqm = qpm + NSEG_PRE * HGN * D;
+  float* cbs = sqm + NSEG_PRE * HGN * D;  // [64]: c_K at 0, c_V at 16, mixed layout c_K lo at 32, c_V lo at 40
+  float4 m4[16];
+  int nhs[NSEG_PRE];  // heads of each segment of the chunk (0 past the CTA's range)
+  constexpr int QPT = (NSEG_PRE * HGN * D + NW * 32 - 1) / (NW * 32);  // query values per thread
+  // segments of the chunk starting at fc: heads and query offsets
+  auto chunk_info = [&](int64_t fc, int64_t (&qbase)[NSEG_PRE]) {
+    int64_t f = fc;
+#pragma unroll
+    for (int si = 0; si < NSEG_PRE; ++si) {
+      nhs[si] = 0;
+      qbase[si] = 0;
+      if (f < f_end) {
+        const int64_t u = f / L;
+        const int64_t t0 = f - u * L;
+        f += (L - t0 < f_end - f) ? L - t0 : f_end - f;
+        const int bk = (int)(u / a.hgroups), hg = (int)(u % a.hgroups);
+        const int b = bk / a.Hkv, h0 = (bk % a.Hkv) * a.g + hg * HG;
+        nhs[si] = min(HG, a.g - hg * HG);
+        qbase[si] = ((int64_t)b * a.Hq + h0) * D;
+      }
+    }
+  };
+  auto load_q = [&](const int64_t (&qbase)[NSEG_PRE], int i) -> float {
+    const int si = i / (HGN * D), hh = (i / D) % HGN, d = i % D;
+    const int64_t qi = qbase[si] + hh * D + d;
+    return a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[qi])
+                    : reinterpret_cast<const float*>(a.q)[qi];
+  };
+  auto q_live = [&](int i) { return (i % (HGN * D)) / D < nhs[i / (HGN * D)]; };
+  auto prep_pass = [&](const float* M, const float* vin, float* vout) {
+    for (int task = tid; task < 2 * D; task += NW * 32) {  // whole warps
+      const int row = task >> 1, half = task & 1;
+      if (task != tid) {
+        const float4* mr = reinterpret_cast<const float4*>(M + row * D + 64 * half);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) m4[k] = __ldg(mr + k);
+      }
+#pragma unroll 1
+      for (int si = 0; si < NSEG_PRE; ++si) {
+#pragma unroll 1
+        for (int hh = 0; hh < nhs[si]; ++hh) {
+          const float4* v4 = reinterpret_cast<const float4*>(vin + (si * HGN + hh) * D + 64 * half);
+          float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 16; k += 2) {
+            const float4 x = v4[k], y = v4[k + 1];
+            acc0 = fmaf(m4[k].x, x.x, acc0);
+            acc1 = fmaf(m4[k + 1].x, y.x, acc1);
+            acc0 = fmaf(m4[k].y, x.y, acc0);
+            acc1 = fmaf(m4[k + 1].y, y.y, acc1);
+            acc0 = fmaf(m4[k].z, x.z, acc0);
+            acc1 = fmaf(m4[k + 1].z, y.z, acc1);
+            acc0 = fmaf(m4[k].w, x.w, acc0);
+            acc1 = fmaf(m4[k + 1].w, y.w, acc1);
+          }
+          float acc = acc0 + acc1;
+          acc += __shfl_xor_sync(FULL, acc, 1);
+          if (half == 0) vout[(si * HGN + hh) * D + row] = acc;
+        }
+      }
+    }
+  };
+  auto prep_passes = [&]() {  // raw q staged in sqm (and a barrier since)
+    prep_pass(a.Pi, sqm, qpm);
+    consumers_sync<NW>();
+    if constexpr (QJL) {
+      if (tid < 2 * D) {
+        const float4* sr = reinterpret_cast<const float4*>(a.S + (tid >> 1) * D + 64 * (tid & 1));
+#pragma unroll
+        for (int k = 0; k < 16; ++k) m4[k] = __ldg(sr + k);
+      }
+      prep_pass(a.S, qpm, sqm);
+      consumers_sync<NW>();
+    }
+  };
+  // B operands of the main loop's MMAs, built once per chunk for all consumer warps.  Column gq of
+  // n-block nb = head 4 nb + gq / 2, part gq % 2 (0: fp16 hi, 1: fp16 lo); k-step kk holds
+  // k = 16kk + 2t, +1 (reg 0), +8, +9 (reg 1) of lane (gq, t).  Word 2kk + r of a lane holds the q'
+  // fragment (kk, r), word 16 + 2kk + r the S q' one.  Each head is scaled by a power of two 2^-e
+  // so that q' and 16 S q' stay far inside fp16 range.
+  uint32_t* frg = reinterpret_cast<uint32_t*>(cbs + 64);
+  float4* hcon = reinterpret_cast<float4*>(frg + Lay::FRAG_WORDS);  // [NSEG_PRE][HGN]
+  auto prep_frags = [&]() {
+    // per head: the scale, then the QJL constant Kh = -C - 0.5 sum_k sq_k 2^-e with C the sum of the
+    // fp16 parts of the pre-scaled S q' (sum_l sq_l (2 b_l - 1) = 2 (D_hi + D_lo + Kh) in the MMA)
+    for (int hx = warp; hx < NSEG_PRE * HGN; hx += NW) {  // warp-uniform
+      const int si = hx / HGN, hh = hx % HGN;
+      if (hh >= nhs[si]) {
+        if (lane == 0) hcon[hx] = make_float4(a.sK, a.sQ, 0.0f, 1.0f);
+        continue;
+      }
+      const float* qp = qpm + hx * D;
+      const float* sp = sqm + hx * D;
+      float mx = 0.0f;
+#pragma unroll
+      for (int k = lane; k < D; k += 32)
+        mx = fmaxf(mx, fmaxf(fabsf(qp[k]), QJL ? 16.0f * fabsf(sp[k]) : 0.0f));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+      // 2^-e with mx 2^-e < 2^14 (e >= 0); inf / nan stay inf / nan
+      const int ex = (mx < 16384.0f || !(mx < INFINITY)) ? 0 : ((__float_as_int(mx) >> 23) & 255) - 127 - 13;
+      const float dn = __int_as_float((127 - ex) << 23);
+      float ch = 0.0f, sh = 0.0f;
+      if constexpr (QJL) {
+#pragma unroll
+        for (int k = lane; k < D; k += 32) {
+          const float scl = (float)(16 >> ((k >> 3) & 3));  // sgn_scale of the k-step pair
+          const float v = sp[k] * dn * scl;
+          const float hi = __half2float(__float2half_rn(v));
+          const float lo = __half2float(__float2half_rn(v - hi));
+          ch += hi + lo;
+          sh += (hi + lo) * (1.0f / scl);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          ch += __shfl_xor_sync(FULL, ch, o);
+          sh += __shfl_xor_sync(FULL, sh, o);
+        }
+      }
+      if (lane == 0) {
+        const float up = __int_as_float((127 + ex) << 23);
+        hcon[hx] = make_float4(a.sK * up, a.sQ * up, -ch - 0.5f * sh, dn);
+      }
+    }
+    consumers_sync<NW>();
+    for (int i = tid; i < Lay::FRAG_WORDS; i += NW * 32) {
+      const int word = ((i >> 7) & 7) * 4 + (i & 3), ln = (i >> 2) & 31;
+      const int nb = (i >> 10) % NB, si = i / (1024 * NB);
+      const int kk = (word >> 1) & 7, r = word & 1, sq = word >> 4;
+      const int hh = 4 * nb + (ln >> 3), tt = ln & 3;
+      const bool lo = (ln >> 2) & 1;
+      uint32_t v = 0u;
+      if (hh < nhs[si] && (!sq || QJL)) {
+        const float* src = (sq ? sqm : qpm) + (si * HGN + hh) * D + 16 * kk + 8 * r + 2 * tt;
+        const float f = hcon[si * HGN + hh].w * (sq ? sgn_scale(2 * kk + r) : 1.0f);
+        float h0, l0, h1, l1;
+        split_half(src[0] * f, h0, l0);
+        split_half(src[1] * f, h1, l1);
+        v = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
+      }
+      frg[i] = v;
+    }
+    consumers_sync<NW>();
+  };
+  // A later chunk (a CTA whose range holds more than NSEG_PRE segments: short contexts) comes in the
+  // middle of the stream, where every consumer warp is at the same segment boundary and the loop
+  // state holds registers: there the matrix rows are read 16 values at a time.
+  auto prep_chunk = [&](int64_t fc) {
+    int64_t qbase[NSEG_PRE];
+    chunk_info(fc, qbase);
+#pragma unroll 1
+    for (int i = tid; i < NSEG_PRE * HGN * D; i += NW * 32)
+      if (q_live(i)) sqm[i] = load_q(qbase, i);
+    consumers_sync<NW>();
+#pragma unroll 1
+    for (int pass = 0; pass < (QJL ? 2 : 1); ++pass) {
+      const float* vin = pass ? qpm : sqm;
+      float* vout = pass ? sqm : qpm;
+#pragma unroll 1
+      for (int task = tid; task < 2 * D; task += NW * 32) {  // whole warps
+        const int row = task >> 1, half = task & 1;
+        const float4* mr = reinterpret_cast<const float4*>((pass ? a.S : a.Pi) + row * D + 64 * half);
+#pragma unroll 1
+        for (int si2 = 0; si2 < NSEG_PRE; ++si2) {
+#pragma unroll 1
+          for (int hh = 0; hh < nhs[si2]; ++hh) {
+            const float4* v4 = reinterpret_cast<const float4*>(vin + (si2 * HGN + hh) * D + 64 * half);
+            float acc = 0.0f;
+#pragma unroll 1
+            for (int k0 = 0; k0 < 16; k0 += 4) {
+#pragma unroll
+              for (int k = k0; k < k0 + 4; ++k) {
+                const float4 mm = __ldg(mr + k), x = v4[k];
+                acc = fmaf(mm.x, x.x, acc);
+                acc = fmaf(mm.y, x.y, acc);
+                acc = fmaf(mm.z, x.z, acc);
+                acc = fmaf(mm.w, x.w, acc);
+              }
+            }
+            acc += __shfl_xor_sync(FULL, acc, 1);
+            if (half == 0) vout[(si2 * HGN + hh) * D + row] = acc;
+          }
+        }
+      }
+      consumers_sync<NW>();
+    }
+    prep_frags();
+  };
+
   Lut lut;
   {
+    // ---- issue the loads
+    int64_t qbase[NSEG_PRE];
+    chunk_info(f_begin, qbase);
+    float qr[QPT];
+#pragma unroll
+    for (int k = 0; k < QPT; ++k) {
+      const int i = tid + k * NW * 32;
+      qr[k] = (i < NSEG_PRE * HGN * D && q_live(i)) ? load_q(qbase, i) : 0.0f;
+    }
+    if (tid < 2 * D) {
+      const float4* pr = reinterpret_cast<const float4*>(a.Pi + (tid >> 1) * D + 64 * (tid & 1));
+#pragma unroll
+      for (int k = 0; k < 16; ++k) m4[k] = __ldg(pr + k);
+      if constexpr (QJL) {
+        const float* sr = a.S + (tid >> 1) * D + 64 * (tid & 1);
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(sr));
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(sr + 32));
+      }
+    }
+    float cbv = 0.0f;
+    if (tid < 16) cbv = tid < (1 << KB) ? a.kc[tid] : 0.0f;
+    else if (tid < 32) cbv = tid - 16 < (1 << VB) ? a.vc[tid - 16] : 0.0f;
+    else if (MX && tid < 40) cbv = a.kc2[tid - 32];
+    else if (MX && tid < 48) cbv = a.vc2[tid - 40];
+    // ---- stage them in shared memory
+#pragma unroll
+    for (int k = 0; k < QPT; ++k) {
+      const int i = tid + k * NW * 32;
+      if (i < NSEG_PRE * HGN * D) sqm[i] = qr[k];
+    }
+    if (tid < 64) cbs[tid] = cbv;
+    consumers_sync<NW>();
+
+    // ---- pair tables: entry e = lo | hi << b -> half2(c[lo], c[hi]), four lane replicas per
+    // 16-byte store
     const uint32_t tbl = ctl.tbl_addr;
     unsigned char* tp = smem + (tbl - smem_u32(smem));
     if constexpr (Lut::kPacked) {
       for (int i = tid; i < 256 * 2 * 8; i += NW * 32) {  // (entry, half, group of four lanes)
         const int e = i >> 4, half = (i >> 3) & 1, q4 = i & 7;
-        const float* cb = half ? a.vc : a.kc;
-        const uint32_t v = pack_half2(__ldg(cb + (e & 15)), __ldg(cb + (e >> 4)));
+        const float* cb = cbs + 16 * half;
+        const uint32_t v = pack_half2(cb[e & 15], cb[e >> 4]);
         *reinterpret_cast<uint4*>(tp + e * 256 + half * 128 + 16 * q4) = make_uint4(v, v, v, v);
       }
       lut.rk = tbl | (4u * lane);
@@ -543,8 +790,8 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         unsigned char* tp2 = smem + (ctl.tbl2_addr - smem_u32(smem));
         for (int i = tid; i < 2 * 64 * 8; i += NW * 32) {  // (table, entry, group of four lanes)
           const int isv = i >> 9, e = (i >> 3) & 63, q4 = i & 7;
-          const float* cb = isv ? a.vc2 : a.kc2;
-          const uint32_t v = pack_half2(__ldg(cb + (e & 7)), __ldg(cb + (e >> 3)));
+          const float* cb = cbs + 32 + 8 * isv;
+          const uint32_t v = pack_half2(cb[e & 7], cb[e >> 3]);
           *reinterpret_cast<uint4*>(tp2 + isv * 8192 + e * 128 + 16 * q4) = make_uint4(v, v, v, v);
         }
         lut.rk2 = ctl.tbl2_addr + 4u * lane;
@@ -556,26 +803,29 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         const int j = isv ? i - Lay::K_TBL / 16 : i;
         const int e = j >> 3;
         const int bits = isv ? VB : KB;
-        const float* cb = isv ? a.vc : a.kc;
-        const uint32_t v = pack_half2(__ldg(cb + (e & ((1 << bits) - 1))), __ldg(cb + (e >> bits)));
+        const float* cb = cbs + (isv ? 16 : 0);
+        const uint32_t v = pack_half2(cb[e & ((1 << bits) - 1)], cb[e >> bits]);
         *reinterpret_cast<uint4*>(tp + 16 * i) = make_uint4(v, v, v, v);
       }
       lut.rk = tbl + 4u * lane;
       lut.rv = tbl + Lay::K_TBL + 4u * lane;
     }
   }
-  consumers_sync<NW>();
+  prep_passes();  // (its barriers also order the table stores before the first lookup)
+  prep_frags();
   // the merge kernel may launch now; its CTAs wait for this grid to finish before reading
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   const int gq = lane >> 2, t = lane & 3;
-  float* mrg = reinterpret_cast<float*>(smem + ctl.merge_off);
-  float* mw = mrg;                 // [NW][HGN]
-  float* lw = mw + NW * HGN;       // [NW][HGN]
-  float* ow = lw + NW * HGN;       // [NW][HGN][D]
   int slot = 0;
   uint32_t phase = 0;  // parity of the ring round being consumed
-  for (int64_t f = f_begin; f < f_end;) {
+  int si = 0;          // this segment's index in the prep chunk
+  for (int64_t f = f_begin; f < f_end; ++si) {
+    if (si == NSEG_PRE) {  // the next chunk (every consumer warp is at this segment boundary)
+      consumers_sync<NW>();  // the previous chunk's q' / S q' are read
+      prep_chunk(f);
+      si = 0;
+    }
     const int64_t u = f / L;
     const int t0 = (int)(f - u * L);
     const int t1 = (int)(L < t0 + (f_end - f) ? L : t0 + (f_end - f));
@@ -585,114 +835,28 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
     const int h0 = kvh * a.g + hg * HG;
     const int nh = min(HG, a.g - hg * HG);
 
-    // ---- query prep for this unit's heads (the merge area is free at a segment's start):
-    // q' = Pi q, then sq = S q', fp32, into shared memory.  Thread (i, half) sums 64 of the 128
-    // products of output row i for every head, reading its half-row of Pi (S) once.
-    float* qsm = mrg;             // [HGN][D] query vectors
-    float* qpm = qsm + HGN * D;   // [HGN][D] q'
-    float* sqm = qpm + HGN * D;   // [HGN][D] S q'
-    for (int i = tid; i < nh * D; i += NW * 32) {
-      const int64_t qi = ((int64_t)b * a.Hq + h0 + i / D) * D + i % D;
-      qsm[i] = a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[qi])
-                        : reinterpret_cast<const float*>(a.q)[qi];
-    }
-    consumers_sync<NW>();
-    for (int pass = 0; pass < (QJL ? 2 : 1); ++pass) {
-      const float* Mtx = pass ? a.S : a.Pi;
-      const float* vin = pass ? qpm : qsm;
-      float* vout = pass ? sqm : qpm;
-      for (int task = tid; task < 2 * D; task += NW * 32) {  // 32 NW is a multiple of 32: pairs stay in a warp
-        const int row = task >> 1, half = task & 1;
-        const float4* mr = reinterpret_cast<const float4*>(Mtx + row * D + 64 * half);
-        float4 m4[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) m4[k] = __ldg(mr + k);
-        for (int hh = 0; hh < nh; ++hh) {
-          const float4* v4 = reinterpret_cast<const float4*>(vin + hh * D + 64 * half);
-          float acc = 0.0f;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float4 x = v4[k];
-            acc = fmaf(m4[k].x, x.x, acc);
-            acc = fmaf(m4[k].y, x.y, acc);
-            acc = fmaf(m4[k].z, x.z, acc);
-            acc = fmaf(m4[k].w, x.w, acc);
-          }
-          acc += __shfl_xor_sync(FULL, acc, 1);
-          if (half == 0) vout[hh * D + row] = acc;
-        }
-      }
-      consumers_sync<NW>();
-    }
-
-    // ---- B operands of this unit's heads.  Column gq of n-block nb = head 4 nb + gq / 2, part
-    // gq % 2 (0: fp16 hi, 1: fp16 lo); k-step kk holds k = 16kk + 2t, +1 (reg 0), +8, +9 (reg 1).
-    // Each head is scaled by a power of two 2^-e so that q' and 16 S q' stay far inside fp16 range.
+    // ---- B operands and per-head constants of this segment (built by prep_frags)
     uint32_t bq[NB][8][2], bsq[NB][8][2];
     float fK[NB], fQ[NB], Kh[NB];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      const int hh = 4 * nb + (gq >> 1);
-      const bool live = hh < nh;
-      const bool lo = gq & 1;
-      const float* qp = qpm + (live ? hh : 0) * D;
-      const float* sp = sqm + (live ? hh : 0) * D;
-      float qv[8][2][2], sv[8][2][2];
-      float mx = 0.0f;
+      const uint4* fp = reinterpret_cast<const uint4*>(frg) + (si * NB + nb) * 8 * 32 + lane;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
+      for (int w4 = 0; w4 < 8; ++w4) {
+        const uint4 v = fp[w4 * 32];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int k = 16 * kk + 8 * r + 2 * t + e;
-            qv[kk][r][e] = live ? qp[k] : 0.0f;
-            sv[kk][r][e] = (live && QJL) ? sp[k] : 0.0f;
-            mx = fmaxf(mx, fmaxf(fabsf(qv[kk][r][e]), 16.0f * fabsf(sv[kk][r][e])));
-          }
-      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));  // both parts of the head
-      // 2^-e with mx 2^-e < 2^14 (e >= 0); inf / nan stay inf / nan
-      const int ex = (mx < 16384.0f || !(mx < INFINITY)) ? 0 : ((__float_as_int(mx) >> 23) & 255) - 127 - 13;
-      const float dn = __int_as_float((127 - ex) << 23);  // 2^-ex
-      float csum = 0.0f, ssum = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          float hx, lx, hy, ly;
-          split_half(qv[kk][r][0] * dn, hx, lx);
-          split_half(qv[kk][r][1] * dn, hy, ly);
-          bq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
-          if constexpr (QJL) {
-            const float scl = sgn_scale(2 * kk + r);
-            split_half(sv[kk][r][0] * dn * scl, hx, lx);
-            split_half(sv[kk][r][1] * dn * scl, hy, ly);
-            bsq[nb][kk][r] = lo ? pack_half2(lx, ly) : pack_half2(hx, hy);
-            const float p0 = lo ? lx : hx, p1 = lo ? ly : hy;  // this lane's column values
-            csum += p0 + p1;
-            ssum += (p0 + p1) * (1.0f / scl);
-          } else {
-            bsq[nb][kk][r] = 0u;
-          }
+        for (int j = 0; j < 4; ++j) {
+          const int word = 4 * w4 + j;
+          if (word < 16) bq[nb][word >> 1][word & 1] = wv[j];
+          else bsq[nb][(word >> 1) & 7][word & 1] = wv[j];
         }
-      // column sums over the four lanes of the column, then per head (hi + lo columns) for the
-      // score layout, where lane (gq, t) holds head 4 nb + t
-      csum += __shfl_xor_sync(FULL, csum, 1);
-      csum += __shfl_xor_sync(FULL, csum, 2);
-      ssum += __shfl_xor_sync(FULL, ssum, 1);
-      ssum += __shfl_xor_sync(FULL, ssum, 2);
-      const float ch = __shfl_sync(FULL, csum, 8 * t) + __shfl_sync(FULL, csum, 8 * t + 4);
-      const float sh = __shfl_sync(FULL, ssum, 8 * t) + __shfl_sync(FULL, ssum, 8 * t + 4);
-      const int ext = __shfl_sync(FULL, ex, 8 * t);
-      const float up = __int_as_float((127 + ext) << 23);  // 2^e of head 4 nb + t
-      fK[nb] = a.sK * up;
-      fQ[nb] = a.sQ * up;
-      Kh[nb] = -ch - 0.5f * sh;  // sum_l sq_l (2 b_l - 1) = 2 (D_hi + D_lo + Kh)
+      }
+      const float4 hc = hcon[si * HGN + 4 * nb + t];
+      fK[nb] = hc.x;
+      fQ[nb] = hc.y;
+      Kh[nb] = hc.z;
     }
-
-    consumers_sync<NW>();  // q' / S q' are read; the merge at this segment's end reuses the area
 
     // Output accumulators: n-block nb, dim block db: (dim 16db + gq, head 4nb + t) hi/lo in [0]/[1],
     // (dim 16db + 8 + gq) in [2]/[3].
@@ -946,70 +1110,104 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       }
     }
 
-    // ---- merge the NW warps: one (max, sum, o') partial per head of this segment ----
+    // ---- partials.  Per head, slots 0 .. pmax-1 hold one (max, sum, o') partial per CTA that ends
+    // inside the head's unit (slot j: the CTA's index among the unit's CTAs), and slots pmax ..
+    // pmax + NW - 1 the per-warp partials of the one CTA that streams the unit's last token and
+    // goes on to the next unit.  So a segment that is not the CTA's last costs no barrier, and
+    // the CTA's last one merges its warps through the (then free) ring memory.
+    const int64_t hstride = (int64_t)(a.pmax + NW) * PART;
+    if (f < f_end) {
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int hh = 4 * nb + t;
-      float lq = l_run[nb];
-      lq += __shfl_xor_sync(FULL, lq, 4);
-      lq += __shfl_xor_sync(FULL, lq, 8);
-      lq += __shfl_xor_sync(FULL, lq, 16);
-      if (gq == 0) {
-        mw[warp * HGN + hh] = m_run[nb];
-        lw[warp * HGN + hh] = lq;
-      }
-      float* o = ow + (warp * HGN + hh) * D;
+      for (int nb = 0; nb < NB; ++nb) {
+        const int hh = 4 * nb + t;
+        float lq = l_run[nb];
+        lq += __shfl_xor_sync(FULL, lq, 4);
+        lq += __shfl_xor_sync(FULL, lq, 8);
+        lq += __shfl_xor_sync(FULL, lq, 16);
+        if (hh < nh) {
+          float* dst = a.part + ((int64_t)b * a.Hq + h0 + hh) * hstride + (a.pmax + warp) * PART;
+          if (gq == 0) {
+            dst[0] = m_run[nb];
+            dst[1] = lq;
+          }
 #pragma unroll
-      for (int db = 0; db < 8; ++db) {
-        o[16 * db + gq] = oacc[nb][db][0] + oacc[nb][db][1];
-        o[16 * db + 8 + gq] = oacc[nb][db][2] + oacc[nb][db][3];
-      }
-    }
-    consumers_sync<NW>();
-    {
-      const int j = c - part_cta_of(a.ntot, a.ctas, u * L);  // partial slot of this CTA in unit u
-      for (int idx = tid; idx < nh * D; idx += NW * 32) {
-        const int r = idx / D, dd = idx % D;
-        float M = -1e30f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w * HGN + r]);
-        float Ls = 0.0f, O = 0.0f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const float fw = ex2(mw[w * HGN + r] - M);
-          Ls = fmaf(fw, lw[w * HGN + r], Ls);
-          O = fmaf(fw, ow[(w * HGN + r) * D + dd], O);
-        }
-        float* dst = a.part + (((int64_t)b * a.Hq + h0 + r) * a.pmax + j) * PART;
-        dst[4 + dd] = O;
-        if (dd == 0) {
-          dst[0] = M;
-          dst[1] = Ls;
+          for (int db = 0; db < 8; ++db) {
+            dst[4 + 16 * db + gq] = oacc[nb][db][0] + oacc[nb][db][1];
+            dst[4 + 16 * db + 8 + gq] = oacc[nb][db][2] + oacc[nb][db][3];
+          }
         }
       }
+    } else {
+      const int j = c - part_cta_of(a.ntot, a.ctas, u * L);
+      float* mw = reinterpret_cast<float*>(smem + ctl.merge_off);  // [NW][4]
+      float* lw = mw + NW * 4;                                       // [NW][4]
+      float* ow = lw + NW * 4;                                       // [NW][4][D]
+      consumers_sync<NW>();  // every warp is past its last stage: the ring is free
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float lq = l_run[nb];
+        lq += __shfl_xor_sync(FULL, lq, 4);
+        lq += __shfl_xor_sync(FULL, lq, 8);
+        lq += __shfl_xor_sync(FULL, lq, 16);
+        if (gq == 0) {
+          mw[warp * 4 + t] = m_run[nb];
+          lw[warp * 4 + t] = lq;
+        }
+        float* o = ow + (warp * 4 + t) * D;
+#pragma unroll
+        for (int db = 0; db < 8; ++db) {
+          o[16 * db + gq] = oacc[nb][db][0] + oacc[nb][db][1];
+          o[16 * db + 8 + gq] = oacc[nb][db][2] + oacc[nb][db][3];
+        }
+        consumers_sync<NW>();
+        for (int idx = tid; idx < 4 * D; idx += NW * 32) {
+          const int r = idx / D, dd = idx % D;
+          if (4 * nb + r < nh) {
+            float M = -1e30f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w * 4 + r]);
+            float Ls = 0.0f, O = 0.0f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+              const float fw = ex2(mw[w * 4 + r] - M);
+              Ls = fmaf(fw, lw[w * 4 + r], Ls);
+              O = fmaf(fw, ow[(w * 4 + r) * D + dd], O);
+            }
+            float* dst = a.part + ((int64_t)b * a.Hq + h0 + 4 * nb + r) * hstride + (int64_t)j * PART;
+            dst[4 + dd] = O;
+            if (dd == 0) {
+              dst[0] = M;
+              dst[1] = Ls;
+            }
+          }
+        }
+        if (nb + 1 < NB) consumers_sync<NW>();  // the area is reused by the next n-block
+      }
     }
-    consumers_sync<NW>();  // the merge area is reused by the next segment
   }
   if (tid == 0 && *reinterpret_cast<volatile unsigned int*>(&ctl.err)) atomicOr(&g_decode_error, 1u);
 }
 
 // ------------------------------------------------------------------------------------------ merge
 
-// One 512-thread CTA per (batch, query head), a programmatic dependent of the split kernel: it
-// waits for the split grid, merges the head's partials (one per CTA that streamed part of the
-// head's unit) by log-sum-exp and writes o = Pi^T o'.  Thread (d, q), d = tid % 128 and
-// q = tid / 128, takes the partials s = q (mod 4) of dimension d with a running maximum, so all of
-// its loads issue at once (one L2 round trip); the four quarters are then combined per dimension.
-// The un-rotation gives thread (i, q) the rows 32q .. 32q + 31 of Pi, loaded before the wait.
-constexpr int MERGE_THREADS = 4 * D;
+// One 1024-thread CTA per (batch, query head), a programmatic dependent of the split kernel: it
+// waits for the split grid, merges the head's partials (see the split kernel's end) by
+// log-sum-exp and writes o = Pi^T o'.  Thread (d, q),
+// d = tid % 128 and q = tid / 128, takes the partials s = q (mod 8) of dimension d with a running
+// maximum; its loads do not depend on one another, so they issue together.  The eight groups are
+// then combined per dimension.  The un-rotation gives thread (i, q) the rows 16q .. 16q + 15 of Pi,
+// loaded before the wait.
+constexpr int MERGE_GROUPS = 8;
+constexpr int MERGE_THREADS = MERGE_GROUPS * D;
+constexpr int MERGE_ROWS = D / MERGE_GROUPS;
 
 // (The partials are written by the still-running split grid: they are read with ld.global.cg,
 // through L2 only, never through the non-coherent read-only path.)
 __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part, const float* __restrict__ Pi,
                                                               float* __restrict__ out, int Hq, int g, int Hkv,
                                                               int hgroups, int64_t seq_len, int64_t ntot, int ctas,
-                                                              int pmax) {
-  __shared__ float mq[4][D], lq[4][D], oq[4][D], ob[D];
+                                                              int pmax, int nw) {
+  __shared__ float mq[MERGE_GROUPS][D], lq[MERGE_GROUPS][D], oq[MERGE_GROUPS][D], ob[D];
   const int tid = threadIdx.x, d = tid % D, q = tid / D;
   const int64_t bh = blockIdx.x;
   if (seq_len == 0) {  // empty context: the output is zero (no split grid ran)
@@ -1017,20 +1215,24 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
     return;
   }
   // Pi is an input, not an output of split: its rows load while the split grid finishes
-  float pj[32];
+  float pj[MERGE_ROWS];
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) pj[jj] = __ldg(Pi + (32 * q + jj) * D + d);
+  for (int jj = 0; jj < MERGE_ROWS; ++jj) pj[jj] = __ldg(Pi + (MERGE_ROWS * q + jj) * D + d);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int b = (int)(bh / Hq), h = (int)(bh % Hq);
   const int64_t u = ((int64_t)b * Hkv + h / g) * hgroups + (h % g) / HG;
   const int first = part_cta_of(ntot, ctas, u * seq_len);
-  const int S = part_cta_of(ntot, ctas, u * seq_len + seq_len - 1) - first + 1;
-  const float* p = part + bh * pmax * PART;
+  const int last = part_cta_of(ntot, ctas, u * seq_len + seq_len - 1);
+  // the last CTA wrote per-warp partials (slots pmax ..) when its range goes on past the unit
+  const bool past = part_start(ntot, ctas, last + 1) > (u + 1) * seq_len;
+  const int S = last - first + (past ? nw : 1);
+  const float* p = part + bh * (pmax + nw) * PART;
   float M = -1e30f, Ls = 0.0f, O = 0.0f;
 #pragma unroll 4
-  for (int s2 = q; s2 < S; s2 += 4) {
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p + (int64_t)s2 * PART));
-    const float o = __ldcg(p + (int64_t)s2 * PART + 4 + d);
+  for (int s2 = q; s2 < S; s2 += MERGE_GROUPS) {
+    const int slot = s2 < last - first ? s2 : (past ? pmax + s2 - (last - first) : s2);
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p + (int64_t)slot * PART));
+    const float o = __ldcg(p + (int64_t)slot * PART + 4 + d);
     const float Mn = fmaxf(M, ml.x);
     const float a0 = ex2(M - Mn), a1 = ex2(ml.x - Mn);
     Ls = fmaf(a1, ml.y, Ls * a0);
@@ -1042,10 +1244,12 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
   oq[q][d] = O;
   __syncthreads();
   if (tid < D) {
-    const float Mx = fmaxf(fmaxf(mq[0][d], mq[1][d]), fmaxf(mq[2][d], mq[3][d]));
+    float Mx = mq[0][d];
+#pragma unroll
+    for (int k = 1; k < MERGE_GROUPS; ++k) Mx = fmaxf(Mx, mq[k][d]);
     float Lt = 0.0f, Ot = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < MERGE_GROUPS; ++k) {
       const float w = ex2(mq[k][d] - Mx);
       Lt = fmaf(w, lq[k][d], Lt);
       Ot = fmaf(w, oq[k][d], Ot);
@@ -1053,13 +1257,18 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const float* part,
     ob[d] = Lt > 0.0f ? Ot / Lt : 0.0f;
   }
   __syncthreads();
-  // o_i = sum_j Pi[j][i] o'_j, thread (i = d, q) over rows 32q .. 32q + 31
+  // o_i = sum_j Pi[j][i] o'_j, thread (i = d, q) over rows MERGE_ROWS q ..
   float r = 0.0f;
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) r = fmaf(pj[jj], ob[32 * q + jj], r);
+  for (int jj = 0; jj < MERGE_ROWS; ++jj) r = fmaf(pj[jj], ob[MERGE_ROWS * q + jj], r);
   mq[q][d] = r;  // (the combine above has read mq: a barrier separates them)
   __syncthreads();
-  if (tid < D) out[bh * D + d] = mq[0][d] + mq[1][d] + mq[2][d] + mq[3][d];
+  if (tid < D) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int k = 0; k < MERGE_GROUPS; ++k) acc += mq[k][d];
+    out[bh * D + d] = acc;
+  }
 }
 
 // ------------------------------------------------------------------------------------------ host
@@ -1111,8 +1320,14 @@ Plan make_plan(int B, int Hq, int Hkv, int seq_len, int sms) {
   return p;
 }
 
-// Workspace: the partials [B*Hq][pmax][132] fp32.
-size_t workspace_bytes(int B, int Hq, const Plan& p) { return sizeof(float) * (size_t)B * Hq * p.pmax * PART; }
+// Consumer warps of a split CTA for groups of g query heads per kv-head.
+int split_warps(int g) { return g <= 4 ? Shape<1>::NW : Shape<2>::NW; }
+
+// Workspace: the partials [B*Hq][pmax + NW][132] fp32: one per CTA that ends inside the head's
+// unit, plus one per consumer warp of the CTA that streams past the unit's end.
+size_t workspace_bytes(int B, int Hq, int g, const Plan& p) {
+  return sizeof(float) * (size_t)B * Hq * (p.pmax + split_warps(g)) * PART;
+}
 
 template <int KB, int VB, bool QJL, int NB, bool MX>
 tq_status launch_split_nb(const DArgs& a, cudaStream_t stream) {
@@ -1130,7 +1345,7 @@ tq_status launch_split_nb(const DArgs& a, cudaStream_t stream) {
   return TQ_OK;
 }
 
-// One n-block of four heads when a group has at most four query heads, else two.
+// One n-block of four heads when a group has at most four query heads, else two (split_warps).
 template <int KB, int VB, bool QJL, bool MX = false>
 tq_status launch_split(const DArgs& a, cudaStream_t stream) {
   return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1, MX>(a, stream) : launch_split_nb<KB, VB, QJL, 2, MX>(a, stream);
@@ -1162,7 +1377,7 @@ extern "C" size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache,
   using namespace tq;
   if (!cache || B < 1 || Hq < 1 || cache->Hkv < 1 || Hq % cache->Hkv || seq_len < 0) return 0;
   const Plan p = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
-  return workspace_bytes(B, Hq, p);
+  return workspace_bytes(B, Hq, Hq / cache->Hkv, p);
 }
 
 namespace tq {
@@ -1196,7 +1411,7 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
     return fail(TQ_ERR_INVALID_ARG, "q / out / workspace must be 16-byte aligned");
   const int B = cache->B;
   const Plan plan = make_plan(B, Hq, cache->Hkv, seq_len, device_sms());
-  const size_t need = workspace_bytes(B, Hq, plan);
+  const size_t need = workspace_bytes(B, Hq, Hq / cache->Hkv, plan);
   if (ws_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
 
@@ -1257,7 +1472,8 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   cfg.attrs = attr;
   cfg.numAttrs = seq_len > 0 ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, merge_kernel, (const float*)ws, params->Pi, out, Hq, g,
-                         cache->Hkv, plan.hgroups, (int64_t)seq_len, plan.ntot, plan.ctas, plan.pmax);
+                         cache->Hkv, plan.hgroups, (int64_t)seq_len, plan.ntot, plan.ctas, plan.pmax,
+                         split_warps(g));
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
@@ -1305,7 +1521,7 @@ extern "C" tq_status tq_decode_step(const tq_params* params, const void* k_new, 
 namespace tq {
 namespace {
 
-constexpr size_t kStaticWorkspaceBytes = (size_t)4 << 20;  // 4 MiB
+constexpr size_t kStaticWorkspaceBytes = (size_t)16 << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
 
 constexpr int kMaxDevices = 64;

@@ -244,8 +244,9 @@ int tq_reset_device_errors(void);
 tq_status tq_debug_quantize_stall(int enable, long long wait_cycles);
 
 /*
- * Bytes of device workspace tq_decode_attn needs for these sizes on the current device
- * (the split-K partials).  Returns 0 on invalid sizes.
+ * Bytes of device workspace tq_decode_attn needs for these sizes on the current device: the
+ * split-K partials, one (max, sum, o'[128]) record of 132 floats per query head for every consumer
+ * warp of every CTA that streams part of the head's tokens.  Returns 0 on invalid sizes.
  */
 size_t tq_decode_workspace_size(int B, int Hq, const tq_cache* cache, int seq_len);
 
@@ -307,7 +308,7 @@ tq_status tq_decode_step(const tq_params* params, const void* k_new, const void*
  * runtimes that fix their device footprint at start-up and forbid later cudaMalloc, and plug-in
  * hosts that pass a library only the tensors of one call.  Same arguments and results as
  * tq_decode_attn without `workspace`/`workspace_bytes`: the scratch lives in a file-scope device
- * array of tq_decode_static_workspace_limit() bytes (4 MiB) that every GPU loading the library
+ * array of tq_decode_static_workspace_limit() bytes (16 MiB) that every GPU loading the library
  * holds until the process exits.  The function itself calls no cudaMalloc or cudaFree.
  *
  *   - Sizes whose scratch (tq_decode_workspace_size) exceeds the limit are rejected with

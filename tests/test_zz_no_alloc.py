@@ -58,7 +58,7 @@ def test_static_decode_matches_workspace_decode_two_calls():
 
 def test_static_decode_rejects_sizes_above_the_limit():
     limit = tq.decode_static_workspace_limit()
-    assert limit == 4 << 20
+    assert limit == 16 << 20
     w, params, cache, q = _setup("llama3_8b_32k", T=256, B=1, Hkv=8, Hq=32)
     # a cache description whose split-K scratch exceeds the limit (never dereferenced)
     big = cache.as_c()
