@@ -166,7 +166,16 @@ constexpr long long WAIT_LIMIT = 4000000000LL;  // ~2 s of SM clock per wait
 __host__ __device__ inline int64_t part_start(int64_t N, int C, int c) { return (int64_t)c * N / C; }
 __host__ __device__ inline int part_cta_of(int64_t N, int C, int64_t f) { return (int)(((f + 1) * C - 1) / N); }
 
+// Shared-memory plan of a split CTA: absolute shared-window addresses (tables) and offsets from
+// the start of dynamic shared memory (the rest), for dynamic shared memory starting at `base`.
+struct SmemPlan {
+  uint32_t base, tbl, tbl2, prep_off, merge_off;
+  int ns;
+  uint32_t stage_off[NS_MAX];
+};
+
 struct DArgs {
+  SmemPlan plan;  // computed on the host for the usual base of dynamic shared memory
   int B, Hq, Hkv, g, hgroups, T_cap, seq_len;
   int units, ctas, pmax, dyn_smem;
   int64_t ntot;  // units * seq_len
@@ -392,59 +401,68 @@ __device__ __forceinline__ uint32_t v_pair(const PairLut<KB, VB>& L, const VPair
   else return L.v(p.template index<NU>());
 }
 
-// Shared-memory plan, computed by one thread: the pair tables (at a 64 KB boundary for the packed
-// tables) split the rest into two free regions; the most ring slots (up to NS_MAX) are placed
-// first-fit such that the query-prep area (and the mixed layout's second tables) still fit around
-// them.  The warps' merge at the CTA's end goes into adjacent ring slots.  ns = 0 when nothing
-// fits (never with the 227 KB of an sm_100 CTA).
+// Shared-memory plan: the pair tables (at a 64 KB boundary for the packed tables) split the rest
+// into two free regions; the most ring slots (up to NS_MAX) are placed first-fit such that the
+// query-prep area (and the mixed layout's second tables) still fit around them.  The warps' merge
+// at the CTA's end goes into adjacent ring slots.  ns = 0 when nothing fits (never with the 227 KB
+// of an sm_100 CTA).  The host computes it once per launch for the usual start of dynamic shared
+// memory; a CTA whose dynamic shared memory starts elsewhere computes its own.
+struct Regions {
+  uint32_t base, r0, r0e, r1, r1e;
+  __host__ __device__ bool take(uint32_t bytes, uint32_t& off) {
+    if (r0e - r0 >= bytes) {
+      off = r0 - base;
+      r0 += bytes;
+      return true;
+    }
+    if (r1e - r1 >= bytes) {
+      off = r1 - base;
+      r1 += bytes;
+      return true;
+    }
+    return false;
+  }
+};
+
 template <int KB, int VB, bool QJL, int NB, bool MX>
-__device__ void plan_smem(unsigned char* smem, int dyn, Ctrl& c) {
+__host__ __device__ void plan_layout(uint32_t base, int dyn, SmemPlan& p) {
   using Lay = Layout<KB, VB, QJL, NB, MX>;
-  const uint32_t base = smem_u32(smem);
   const uint32_t end = base + (uint32_t)dyn - CTRL_BYTES;
   const uint32_t tbl = Lay::kPacked ? ((base + 0xFFFFu) & ~0xFFFFu) : base;
-  c.tbl_addr = tbl;
-  c.ns = 0;
+  p.base = base;
+  p.tbl = tbl;
+  p.tbl2 = 0;
+  p.ns = 0;
   if (tbl + Lay::TBL_BYTES > end) return;
   for (int ns = NS_MAX; ns >= 2; --ns) {
-    // free regions: [base, tbl) and [tbl + TBL_BYTES, end)
-    uint32_t r0 = base, r0e = tbl, r1 = tbl + Lay::TBL_BYTES, r1e = end;
-    auto take = [&](uint32_t bytes, uint32_t& off) -> bool {
-      if (r0e - r0 >= bytes) {
-        off = r0 - base;
-        r0 += bytes;
-        return true;
-      }
-      if (r1e - r1 >= bytes) {
-        off = r1 - base;
-        r1 += bytes;
-        return true;
-      }
-      return false;
-    };
+    Regions r{base, base, tbl, tbl + (uint32_t)Lay::TBL_BYTES, end};  // [base, tbl) and [tbl + TBL, end)
     bool ok = true;
-    for (int i = 0; i < ns && ok; ++i) ok = take(Lay::STAGE_BYTES, c.stage_off[i]);
-    uint32_t off = 0;
-    ok = ok && take(Lay::PREP_BYTES, off);
-    c.prep_off = off;
+    for (int i = 0; i < ns && ok; ++i) ok = r.take(Lay::STAGE_BYTES, p.stage_off[i]);
+    ok = ok && r.take(Lay::PREP_BYTES, p.prep_off);
     if (ok && Lay::TBL2_BYTES) {
-      ok = take(Lay::TBL2_BYTES, off);
-      c.tbl2_addr = base + off;
+      uint32_t off = 0;
+      ok = r.take(Lay::TBL2_BYTES, off);
+      p.tbl2 = base + off;
     }
     if (!ok) continue;
     // the warps' merge at the CTA's end reuses ring memory: a run of adjacent slots large enough
-    c.merge_off = 0xFFFFFFFFu;
-    for (int k = 0; k < ns && c.merge_off == 0xFFFFFFFFu; ++k) {
+    p.merge_off = 0xFFFFFFFFu;
+    for (int k = 0; k < ns && p.merge_off == 0xFFFFFFFFu; ++k) {
       uint32_t run = Lay::STAGE_BYTES;
       for (int i = k + 1; i < ns && run < (uint32_t)Lay::MERGE_BYTES &&
-                          c.stage_off[i] == c.stage_off[i - 1] + Lay::STAGE_BYTES; ++i)
+                          p.stage_off[i] == p.stage_off[i - 1] + Lay::STAGE_BYTES; ++i)
         run += Lay::STAGE_BYTES;
-      if (run >= (uint32_t)Lay::MERGE_BYTES) c.merge_off = c.stage_off[k];
+      if (run >= (uint32_t)Lay::MERGE_BYTES) p.merge_off = p.stage_off[k];
     }
-    if (c.merge_off == 0xFFFFFFFFu) continue;
-    c.ns = ns;
+    if (p.merge_off == 0xFFFFFFFFu) continue;
+    p.ns = ns;
     return;
   }
+}
+
+// 64-bit division that takes the 32-bit path when both operands fit (every realistic size).
+__device__ __forceinline__ int64_t div_s(int64_t x, int64_t y) {
+  return (x <= 0x7fffffff && y <= 0x7fffffff) ? (int64_t)((uint32_t)x / (uint32_t)y) : x / y;
 }
 
 template <int KB, int VB, bool QJL, int NB, bool MX>
@@ -460,7 +478,15 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
   const int64_t L = a.seq_len;
 
   if (tid == 0) {
-    plan_smem<KB, VB, QJL, NB, MX>(smem, a.dyn_smem, ctl);
+    SmemPlan p;
+    if (smem_u32(smem) == a.plan.base) p = a.plan;
+    else plan_layout<KB, VB, QJL, NB, MX>(smem_u32(smem), a.dyn_smem, p);
+    ctl.tbl_addr = p.tbl;
+    ctl.tbl2_addr = p.tbl2;
+    ctl.prep_off = p.prep_off;
+    ctl.merge_off = p.merge_off;
+    ctl.ns = p.ns;
+    for (int i = 0; i < p.ns; ++i) ctl.stage_off[i] = p.stage_off[i];
     ctl.err = 0;
     for (int i = 0; i < ctl.ns; ++i) {
       mbar_init_(&ctl.full[i], 1 + 32);  // producer's expect_tx + the noinc arrivals of its 32 lanes
@@ -477,13 +503,15 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
 
   if (warp == NW) {
     // ================================================================ producer
+    // the consumers' prologue loads go to memory first (named barrier 2, arrived at by them)
+    asm volatile("bar.sync 2, %0;\n" ::"n"((NW + 1) * 32) : "memory");
     int it = 0, issued = 0, slot = 0, round = 0;  // stage count, ring slot, times round the ring
     for (int64_t f = f_begin; f < f_end;) {
-      const int64_t u = f / L;
+      const int64_t u = div_s(f, L);
       const int t0 = (int)(f - u * L);
       const int t1 = (int)(L < t0 + (f_end - f) ? L : t0 + (f_end - f));
       f += t1 - t0;
-      const int bk = (int)(u / a.hgroups);  // b * Hkv + kv-head
+      const int bk = (int)div_s(u, a.hgroups);  // b * Hkv + kv-head
       const int64_t rowb = (int64_t)bk * a.T_cap;
       for (int s0 = t0; s0 < t1; s0 += ST, ++it) {
         const int cur = slot, cur_round = round;  // this stage's slot, and its earlier uses
@@ -541,16 +569,13 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
 
   // ================================================================ consumers (warps 0 .. NW-1)
   // Prologue: q' = Pi q and sq = S q' of the heads of the CTA's first NSEG_PRE segments (fp32, the
-  // prep area [NSEG_PRE][HGN][D] each; the raw q is staged where sq goes) and the pair tables.
+  // prep area [NSEG_PRE][HGN][D] each; the raw q is staged where sq goes), then the pair tables.
   // Every global load it needs is issued first, so they share one memory round trip: the
-  // thread's half-row of Pi (task (row, half) = (tid / 2, tid % 2)), its share of the queries and
-  // one codebook entry; S is prefetched into L2 and read after the first pass.  Tasks tid + 32 NW,
-  // ... (seven consumer warps: warp 0 takes the last 32) load their rows when they get to them; the
-  // two halves of a row are always in one warp.
+  // thread's rows of Pi and S (see prologue_pass), its share of the queries and one codebook
+  // entry.  The producer starts its copies once the consumers have these loads (named barrier 2).
   float* qpm = reinterpret_cast<float*>(smem + ctl.prep_off);
   float* sqm = qpm + NSEG_PRE * HGN * D;
   float* cbs = sqm + NSEG_PRE * HGN * D;  // [64]: c_K at 0, c_V at 16, mixed layout c_K lo at 32, c_V lo at 40
-  float4 m4[16];
   int nhs[NSEG_PRE];  // heads of each segment of the chunk (0 past the CTA's range)
   constexpr int QPT = (NSEG_PRE * HGN * D + NW * 32 - 1) / (NW * 32);  // query values per thread
   // segments of the chunk starting at fc: heads and query offsets
@@ -561,10 +586,10 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       nhs[si] = 0;
       qbase[si] = 0;
       if (f < f_end) {
-        const int64_t u = f / L;
+        const int64_t u = div_s(f, L);
         const int64_t t0 = f - u * L;
         f += (L - t0 < f_end - f) ? L - t0 : f_end - f;
-        const int bk = (int)(u / a.hgroups), hg = (int)(u % a.hgroups);
+        const int bk = (int)div_s(u, a.hgroups), hg = (int)(u - (int64_t)bk * a.hgroups);
         const int b = bk / a.Hkv, h0 = (bk % a.Hkv) * a.g + hg * HG;
         nhs[si] = min(HG, a.g - hg * HG);
         qbase[si] = ((int64_t)b * a.Hq + h0) * D;
@@ -578,50 +603,45 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
                     : reinterpret_cast<const float*>(a.q)[qi];
   };
   auto q_live = [&](int i) { return (i % (HGN * D)) / D < nhs[i / (HGN * D)]; };
-  auto prep_pass = [&](const float* M, const float* vin, float* vout) {
-    for (int task = tid; task < 2 * D; task += NW * 32) {  // whole warps
-      const int row = task >> 1, half = task & 1;
-      if (task != tid) {
-        const float4* mr = reinterpret_cast<const float4*>(M + row * D + 64 * half);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) m4[k] = __ldg(mr + k);
-      }
+  // Prologue pass: eight lanes per matrix row, lane (row, e) holding the 16-byte chunks e, e + 8,
+  // e + 16, e + 24 of the row, so that each load instruction of a warp reads four whole 128-byte
+  // lines; warp w takes rows 4w + r + 4 NW j in round j.  A row's dot product is summed over its
+  // eight lanes.
+  constexpr int PR = (D + 4 * NW - 1) / (4 * NW);  // rounds
+  auto prologue_pass = [&](const float4 (&r4)[PR][4], const float* vin, float* vout) {
+    const int e = lane & 7;
 #pragma unroll 1
-      for (int si = 0; si < NSEG_PRE; ++si) {
+    for (int si = 0; si < NSEG_PRE; ++si) {
 #pragma unroll 1
-        for (int hh = 0; hh < nhs[si]; ++hh) {
-          const float4* v4 = reinterpret_cast<const float4*>(vin + (si * HGN + hh) * D + 64 * half);
-          float acc0 = 0.0f, acc1 = 0.0f;
+      for (int hh = 0; hh < nhs[si]; ++hh) {
+        const float4* v4 = reinterpret_cast<const float4*>(vin + (si * HGN + hh) * D) + e;
+        float4 x[4];
 #pragma unroll
-          for (int k = 0; k < 16; k += 2) {
-            const float4 x = v4[k], y = v4[k + 1];
-            acc0 = fmaf(m4[k].x, x.x, acc0);
-            acc1 = fmaf(m4[k + 1].x, y.x, acc1);
-            acc0 = fmaf(m4[k].y, x.y, acc0);
-            acc1 = fmaf(m4[k + 1].y, y.y, acc1);
-            acc0 = fmaf(m4[k].z, x.z, acc0);
-            acc1 = fmaf(m4[k + 1].z, y.z, acc1);
-            acc0 = fmaf(m4[k].w, x.w, acc0);
-            acc1 = fmaf(m4[k + 1].w, y.w, acc1);
+        for (int k = 0; k < 4; ++k) x[k] = v4[8 * k];
+#pragma unroll
+        for (int j = 0; j < PR; ++j) {
+          const int row = 4 * warp + (lane >> 3) + 4 * NW * j;
+          if (4 * NW * j + 4 * warp < D) {  // warp-uniform: this round has rows for the warp
+            float c0 = 0.0f, c1 = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; k += 2) {
+              c0 = fmaf(r4[j][k].x, x[k].x, c0);
+              c1 = fmaf(r4[j][k + 1].x, x[k + 1].x, c1);
+              c0 = fmaf(r4[j][k].y, x[k].y, c0);
+              c1 = fmaf(r4[j][k + 1].y, x[k + 1].y, c1);
+              c0 = fmaf(r4[j][k].z, x[k].z, c0);
+              c1 = fmaf(r4[j][k + 1].z, x[k + 1].z, c1);
+              c0 = fmaf(r4[j][k].w, x[k].w, c0);
+              c1 = fmaf(r4[j][k + 1].w, x[k + 1].w, c1);
+            }
+            float acc = c0 + c1;
+            acc += __shfl_xor_sync(FULL, acc, 1);
+            acc += __shfl_xor_sync(FULL, acc, 2);
+            acc += __shfl_xor_sync(FULL, acc, 4);
+            if (e == 0 && row < D) vout[(si * HGN + hh) * D + row] = acc;
           }
-          float acc = acc0 + acc1;
-          acc += __shfl_xor_sync(FULL, acc, 1);
-          if (half == 0) vout[(si * HGN + hh) * D + row] = acc;
         }
       }
-    }
-  };
-  auto prep_passes = [&]() {  // raw q staged in sqm (and a barrier since)
-    prep_pass(a.Pi, sqm, qpm);
-    consumers_sync<NW>();
-    if constexpr (QJL) {
-      if (tid < 2 * D) {
-        const float4* sr = reinterpret_cast<const float4*>(a.S + (tid >> 1) * D + 64 * (tid & 1));
-#pragma unroll
-        for (int k = 0; k < 16; ++k) m4[k] = __ldg(sr + k);
-      }
-      prep_pass(a.S, qpm, sqm);
-      consumers_sync<NW>();
     }
   };
   // B operands of the main loop's MMAs, built once per chunk for all consumer warps.  Column gq of
@@ -749,14 +769,16 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       const int i = tid + k * NW * 32;
       qr[k] = (i < NSEG_PRE * HGN * D && q_live(i)) ? load_q(qbase, i) : 0.0f;
     }
-    if (tid < 2 * D) {
-      const float4* pr = reinterpret_cast<const float4*>(a.Pi + (tid >> 1) * D + 64 * (tid & 1));
+    float4 m4[PR][4], s4[PR][4];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) m4[k] = __ldg(pr + k);
-      if constexpr (QJL) {
-        const float* sr = a.S + (tid >> 1) * D + 64 * (tid & 1);
-        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(sr));
-        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(sr + 32));
+    for (int j = 0; j < PR; ++j) {
+      const int row = 4 * warp + (lane >> 3) + 4 * NW * j;
+      const float4* pr = reinterpret_cast<const float4*>(a.Pi + (row < D ? row : 0) * D) + (lane & 7);
+      const float4* sr = reinterpret_cast<const float4*>(a.S + (row < D ? row : 0) * D) + (lane & 7);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        m4[j][k] = __ldg(pr + 8 * k);
+        if constexpr (QJL) s4[j][k] = __ldg(sr + 8 * k);
       }
     }
     float cbv = 0.0f;
@@ -764,6 +786,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
     else if (tid < 32) cbv = tid - 16 < (1 << VB) ? a.vc[tid - 16] : 0.0f;
     else if (MX && tid < 40) cbv = a.kc2[tid - 32];
     else if (MX && tid < 48) cbv = a.vc2[tid - 40];
+    asm volatile("bar.arrive 2, %0;\n" ::"n"((NW + 1) * 32) : "memory");  // the producer may start
     // ---- stage them in shared memory
 #pragma unroll
     for (int k = 0; k < QPT; ++k) {
@@ -772,6 +795,13 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
     }
     if (tid < 64) cbs[tid] = cbv;
     consumers_sync<NW>();
+    // ---- q' = Pi q, then sq = S q'
+    prologue_pass(m4, sqm, qpm);
+    consumers_sync<NW>();
+    if constexpr (QJL) {
+      prologue_pass(s4, qpm, sqm);
+      consumers_sync<NW>();
+    }
 
     // ---- pair tables: entry e = lo | hi << b -> half2(c[lo], c[hi]), four lane replicas per
     // 16-byte store
@@ -811,8 +841,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       lut.rv = tbl + Lay::K_TBL + 4u * lane;
     }
   }
-  prep_passes();  // (its barriers also order the table stores before the first lookup)
-  prep_frags();
+  prep_frags();  // (its barriers also order the table stores before the first lookup)
   // the merge kernel may launch now; its CTAs wait for this grid to finish before reading
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
@@ -826,11 +855,11 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       prep_chunk(f);
       si = 0;
     }
-    const int64_t u = f / L;
+    const int64_t u = div_s(f, L);
     const int t0 = (int)(f - u * L);
     const int t1 = (int)(L < t0 + (f_end - f) ? L : t0 + (f_end - f));
     f += t1 - t0;
-    const int bk = (int)(u / a.hgroups), hg = (int)(u % a.hgroups);
+    const int bk = (int)div_s(u, a.hgroups), hg = (int)(u - (int64_t)bk * a.hgroups);
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
     const int h0 = kvh * a.g + hg * HG;
     const int nh = min(HG, a.g - hg * HG);
@@ -1330,7 +1359,11 @@ size_t workspace_bytes(int B, int Hq, int g, const Plan& p) {
 }
 
 template <int KB, int VB, bool QJL, int NB, bool MX>
-tq_status launch_split_nb(const DArgs& a, cudaStream_t stream) {
+tq_status launch_split_nb(const DArgs& a0, cudaStream_t stream) {
+  DArgs a = a0;
+  // dynamic shared memory usually starts right after the per-block reserved bytes
+  plan_layout<KB, VB, QJL, NB, MX>((uint32_t)device_attr(cudaDevAttrReservedSharedMemoryPerBlock, 1024),
+                                   a.dyn_smem, a.plan);
   cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        a.dyn_smem);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
@@ -1435,6 +1468,7 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
     a.pmax = plan.pmax;
     a.ntot = plan.ntot;
     a.dyn_smem = split_dyn_smem();
+    // (a.plan is filled per layout at launch)
     // k-hat = ||k|| / sqrt(128) c (mixed layout: ||k_g|| / sqrt(64) c_g of each half)
     a.sK = (float)((double)sc * 1.4426950408889634 / sqrt(cache->layout == TQ_LAYOUT_MIXED ? 64.0 : (double)D));
     a.sQ = cache->qjl_m ? (float)((double)sc * 1.4426950408889634 * 2.0 * sqrt(M_PI / 2.0) / cache->qjl_m)
