@@ -451,7 +451,7 @@ def run_gpu(args, w):
         "roofline": roof_q if dominant == "tq_quantize" else roof_d,
         "roofline_decode": roof_d, "roofline_quantize": roof_q,
         "cpu_baseline": cb, "e2e": e2e,
-        "gpu_launches": args.steps * (n_chunks + 3),
+        "gpu_launches": args.steps * (n_chunks + 2),
         "quantize_fp64_fixups": {"coords": tq.quantize_code_fixups(), "key_vectors": tq.quantize_vector_fixups(),
                                  "calls": (args.warmup + args.steps) * n_chunks},
         "clocks": clk.summary(),

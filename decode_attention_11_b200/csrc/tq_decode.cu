@@ -1430,6 +1430,7 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
                                     const tq_cache* cache, int seq_len, float scale, float* out,
                                     void* workspace, size_t ws_bytes, void* stream) {
   using namespace tq;
+  const NvtxRange nvtx_range("tq_decode_attn");
   clear_error();
   tq_status st = check_cache(cache);
   if (st != TQ_OK) return st;
@@ -1519,6 +1520,7 @@ extern "C" tq_status tq_decode_step(const tq_params* params, const void* k_new, 
                                     int t, float scale, float* out, void* workspace, size_t workspace_bytes,
                                     void* stream) {
   using namespace tq;
+  const NvtxRange nvtx_range("tq_decode_step");
   clear_error();
   tq_status st = check_cache(cache);
   if (st != TQ_OK) return st;
@@ -1589,6 +1591,7 @@ extern "C" tq_status tq_decode_attn_static(const tq_params* params, const void* 
                                            int Hq, const tq_cache* cache, int seq_len,
                                            float scale, float* out, void* stream) {
   using namespace tq;
+  const NvtxRange nvtx_range("tq_decode_attn_static");
   clear_error();
   if (!cache) return fail(TQ_ERR_INVALID_ARG, "cache is NULL");
   const size_t need = tq_decode_workspace_size(cache->B, Hq, cache, seq_len);

@@ -7,6 +7,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tq_internal.h"
 
 namespace tq {
@@ -24,6 +26,9 @@ tq_status fail(tq_status st, const char* fmt, ...) {
 }
 
 void clear_error() { g_last_error.clear(); }
+
+NvtxRange::NvtxRange(const char* name) { nvtxRangePushA(name); }
+NvtxRange::~NvtxRange() { nvtxRangePop(); }
 
 tq_status check_cache(const tq_cache* c) {
   if (!c) return fail(TQ_ERR_INVALID_ARG, "cache is NULL");

@@ -22,6 +22,14 @@ constexpr int kQjlRows = 128;
 constexpr double kExemptCodeBand = 1e-6;
 constexpr double kExemptSignBand = 1e-5;
 
+// NVTX range around an entry point (header-only NVTX 3: a no-op unless a profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name);
+  ~NvtxRange();
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Thread-local error detail; returns `st` so callers can `return fail(...)`.
 tq_status fail(tq_status st, const char* fmt, ...);
 void clear_error();

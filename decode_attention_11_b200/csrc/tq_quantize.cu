@@ -8,17 +8,19 @@
 // scale bits) and "Step 2: QJL" (one extra bit per sketch row makes the inner-product error
 // unbiased).
 //
-// One persistent 256-thread CTA per SM works on 128-token tiles of one (batch, kv-head):
-//   1. cp.async brings the bf16 K and V tiles into shared memory in the UMMA 128-byte-swizzle
-//      layout; each thread converts one row in place to fp16 (exact for bf16 input) and sums
-//      its squares in fp64 (the stored norm).
+// This general kernel serves fp32 inputs and the outlier-aware mixed layout (TQ_LAYOUT_MIXED, any
+// input type); bf16 inputs in the plain layout go to the pipelined kernel of tq_quantize_pipe.cu.
+// One persistent 512-thread CTA per SM works on 128-token tiles of one (batch, kv-head):
+//   1. cp.async brings the K and V tiles into shared memory in the UMMA 128-byte-swizzle layout
+//      (fp32 as fp16 hi + lo); each thread converts one row and sums its squares in fp64 (the
+//      stored norm; one norm per half in the mixed layout).
 //   2. One thread issues tcgen05.mma: Y_K = X_K Pi^T and Y_V = X_V Pi^T with Pi split into fp16
-//      hi + lo (about 22 significant bits), accumulated in fp32 tensor memory (fp32 keys also
-//      enter as fp16 hi + lo).
-//   3. Warpgroup 0 reads Y_K row by row: u = sqrt(d) y / ||x||, code by a branch-free binary
-//      search of the thresholds, residual rho = u - c[code] written as fp16 hi + lo for the next
-//      MMA; warpgroup 1 does the same for Y_V (codes only).
-//   4. tcgen05.mma: S rho for the QJL sign bits; warpgroup 1 packs the signs.
+//      hi + lo (about 22 significant bits; the lo pass is skipped when Pi is exact in fp16),
+//      accumulated in fp32 tensor memory.
+//   3. The epilogue warps read Y row by row in 32-coordinate chunks: u = sqrt(d) y / ||x||, code
+//      by a branch-free binary search of the thresholds (each half its own codebook and scale in
+//      the mixed layout), residual rho = u - c[code] written as fp16 hi + lo for the next MMA.
+//   4. tcgen05.mma: S rho for the QJL sign bits, packed by the epilogue.
 // Exactness: codes and sign bits equal those of the float64 definition.  Any coordinate whose
 // fast value lies within a guard band of a decision boundary (a threshold; 0 for a sign) is
 // re-derived in fp64 from the original inputs, leaving only values within ~1e-15 of a boundary.
@@ -995,6 +997,7 @@ extern "C" tq_status tq_quantize(const tq_params* params, const void* k, const v
                                  int64_t stride_b, int64_t stride_h, int64_t stride_t, int T_new,
                                  int t_offset, const tq_cache* cache, void* stream) {
   using namespace tq;
+  const NvtxRange nvtx_range("tq_quantize");
   clear_error();
   tq_status st = check_cache(cache);
   if (st != TQ_OK) return st;

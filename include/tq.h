@@ -187,9 +187,10 @@ tq_status tq_sketch_rotation(const float* Pi, const float* S, int qjl_m, double*
  *   T_new       >= 0 (0 enqueues nothing);  0 <= t_offset, t_offset + T_new <= cache->T_cap
  * Output bits are those of the float64 definition except where a rotated coordinate lies within
  * about 1e-15 of a threshold (the kernel re-derives near-boundary cases in fp64).
- * TQ_BF16 calls on one device share a file-scope device queue of those fp64 re-derivations:
- * calls whose device work may overlap (different streams without ordering, or host threads
- * racing on one device) corrupt each other's results; order them on one stream.
+ * Calls may run concurrently on different streams: the TQ_BF16 kernel keeps its queue of fp64
+ * re-derivations per SM, a CTA of it occupies an SM's shared memory alone, and each CTA tags its
+ * entries with a generation number drawn at its start.  Consecutive calls on one stream overlap
+ * as programmatic dependent launches (the next call's set-up runs during the previous call's tail).
  * Errors: TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA.
  */
 tq_status tq_quantize(const tq_params* params, const void* k, const void* v, int dtype,

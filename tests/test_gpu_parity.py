@@ -178,8 +178,9 @@ def test_decode_parity_small(name):
 
 
 def test_decode_ignores_workspace_contents():
-    """The workspace's previous contents never change the result: filled with 0x00, 0xFF and 0x5A
-    bytes, and reused across back-to-back calls on one stream."""
+    """The workspace's previous contents never change the result: filled with 0x00, 0xFF (NaN as
+    fp32) and 0x5A bytes, and reused across back-to-back calls on one stream.  Every output element
+    is written: the output buffer starts as NaN."""
     w = small("llama3_8b_32k")
     K, V, Kh, Vh = gpu_inputs(w)
     q = W.make_queries(w).cuda()
@@ -193,8 +194,10 @@ def test_decode_ignores_workspace_contents():
     for fill in (0x00, 0xFF, 0x5A):
         ws.fill_(fill)
         for _ in range(3):
-            outs.append(tq.decode_attn(params, q, cache, w.T, workspace=ws))
+            out = torch.full((w.B, w.Hq, 128), float("nan"), dtype=torch.float32, device="cuda")
+            outs.append(tq.decode_attn(params, q, cache, w.T, out=out, workspace=ws))
     torch.cuda.synchronize()
+    assert all(bool(torch.isfinite(o).all()) for o in outs)
     for out in outs:
         assert_attention_close(out.cpu().numpy(), ref)
 
