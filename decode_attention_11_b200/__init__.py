@@ -40,8 +40,8 @@ EXPORTED = ("tq_status_string", "tq_last_error", "tq_version", "tq_build_codeboo
             "tq_quantize_code_fixups", "tq_quantize_exempt_codes", "tq_quantize_exempt_signs",
             "tq_decode_workspace_size", "tq_decode_attn", "tq_decode_attn_static",
             "tq_decode_static_workspace_limit", "tq_sketch_rotation", "tq_build_hadamard_rotation",
-            "tq_decode_step", "tq_decode_device_errors", "tq_reset_device_errors",
-            "tq_debug_quantize_stall")
+            "tq_decode_step", "tq_decode_step_fused", "tq_decode_device_errors",
+            "tq_reset_device_errors", "tq_debug_quantize_stall")
 
 
 class TqError(RuntimeError):
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
     L.tq_debug_quantize_stall.argtypes = [ctypes.c_int, ctypes.c_longlong]
     L.tq_decode_device_errors.restype = ctypes.c_int
     L.tq_decode_device_errors.argtypes = []
+    L.tq_decode_step_fused.restype = ctypes.c_int
+    L.tq_decode_step_fused.argtypes = [ctypes.POINTER(_Cache), ctypes.c_int, ctypes.c_int]
     L.tq_decode_workspace_size.restype = ctypes.c_size_t
     L.tq_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cache),
                                            ctypes.c_int]
@@ -375,6 +377,15 @@ def decode_device_errors() -> int:
     return int(lib().tq_decode_device_errors())
 
 
+def decode_step_fused(cache: Cache, Hq: int, t: int) -> bool:
+    """Whether decode_step at row t runs as one fused decode launch (see tq_decode_step_fused)."""
+    c = cache.as_c()
+    r = int(lib().tq_decode_step_fused(ctypes.byref(c), Hq, t))
+    if r < 0:
+        raise ValueError(f"invalid sizes Hq={Hq} t={t}")
+    return r == 1
+
+
 def decode_workspace_size(B: int, Hq: int, cache: Cache, seq_len: int) -> int:
     c = cache.as_c()
     return int(lib().tq_decode_workspace_size(int(B), int(Hq), ctypes.byref(c), int(seq_len)))
@@ -459,7 +470,7 @@ __all__ = [
     "decode_attn_static", "decode_static_workspace_limit",
     "quantize_vector_fixups", "quantize_code_fixups", "quantize_exempt_codes", "quantize_exempt_signs",
     "decode_workspace_size", "decode_attn", "decode_device_errors", "reset_device_errors",
-    "debug_quantize_stall",
+    "debug_quantize_stall", "decode_step", "decode_step_fused",
     "TQ_OK", "TQ_ERR_INVALID_ARG", "TQ_ERR_UNSUPPORTED", "TQ_ERR_NO_CONVERGENCE",
     "TQ_ERR_WORKSPACE", "TQ_ERR_CUDA", "TQ_F32", "TQ_BF16", "TQ_LAYOUT_PLAIN", "TQ_LAYOUT_MIXED",
 ]

@@ -196,6 +196,13 @@ struct DArgs {
   const float* Pi;  // [128 x 128]
   const float* S;   // [128 x 128] (QJL)
   float* part;
+  // Decode step (step = 1): row seq_len - 1 of every unit is quantized in the kernel from k_new /
+  // v_new ([B, Hkv, 128], fp32 or bf16) in fp64, written to the cache and attended.
+  int step, kv_bf16;
+  const void* k_new;
+  const void* v_new;
+  const float* kt;  // thresholds of the codebooks
+  const float* vt;
 };
 
 __device__ unsigned int g_decode_error;  // bit 0: a wait timed out; bit 1: shared memory too small
@@ -227,7 +234,12 @@ struct Layout {
   // latter), 64 codebook floats, the MMA B fragments of every lane ([segment][n-block][word / 4]
   // [lane][word % 4], 32 words) and (fK, fQ, Kh, 2^-e) per head
   static constexpr int FRAG_WORDS = NSEG_PRE * NB * 32 * 32;
-  static constexpr int PREP_BYTES = 4 * (2 * NSEG_PRE * HGN * D + 64 + FRAG_WORDS + NSEG_PRE * HGN * 4);
+  static constexpr int PREP_WORDS = 2 * NSEG_PRE * HGN * D + 64 + FRAG_WORDS + NSEG_PRE * HGN * 4;
+  // decode step: the packed new row (key codes 16, signs 4, value codes 16, norms 4 words); its
+  // scratch (8 * 2D + 4 * 2D + 32 bytes) lives in the B-fragment area
+  static constexpr int STEP_BYTES = 4 * 40;
+  static_assert(4 * FRAG_WORDS >= 8 * 2 * D + 4 * 2 * D + 8 * 4, "step scratch");
+  static constexpr int PREP_BYTES = 4 * PREP_WORDS + STEP_BYTES;
   // the merge of the warps at the CTA's last segment end, one n-block at a time, in ring memory:
   // (max, sum) and o' of four heads per warp
   static constexpr int MERGE_BYTES = 4 * (Shape<NB>::NW * 4 * 2 + Shape<NB>::NW * 4 * D);
@@ -465,7 +477,118 @@ __device__ __forceinline__ int64_t div_s(int64_t x, int64_t y) {
   return (x <= 0x7fffffff && y <= 0x7fffffff) ? (int64_t)((uint32_t)x / (uint32_t)y) : x / y;
 }
 
-template <int KB, int VB, bool QJL, int NB, bool MX>
+// Decode step, by the consumer warps of a CTA whose range ends a unit: the unit's new key and value
+// (k_new / v_new) quantized in fp64 exactly as the definition reads -- n = ||x||,
+// u = sqrt(d) Pi x / n, idx = #{t_i <= u}, rho = u - c[idx], ||r|| = n ||rho|| / sqrt(d), sign
+// bits of S rho -- packed into `row` (key codes [0,16), signs [16,20), value codes [20,36), norms
+// [36,39) words) and, for the unit's first head group, written into cache row seq_len - 1.
+// Matrix rows are read eight lanes per row as in the prologue.  Kept out of line: its registers
+// must not weigh on the main loop.
+template <int KB, int VB, bool QJL, int NB>
+__device__ __noinline__ void quantize_step_row(const DArgs& a, float* x, double* y, double* nrm, uint32_t* row,
+                                      const float* cbs, int64_t bk, int hg, int64_t L) {
+  constexpr int NW = Shape<NB>::NW, PR = (D + 4 * NW - 1) / (4 * NW);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, e = lane & 7;
+  for (int i = tid; i < 2 * D; i += NW * 32) {  // i < D: key element i; D <= i: value element i - D
+    const void* src = i < D ? a.k_new : a.v_new;
+    const int64_t off = bk * D + (i % D);
+    x[i] = a.kv_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(src)[off])
+                     : reinterpret_cast<const float*>(src)[off];
+  }
+  if (tid < 40) row[tid] = 0u;
+  consumers_sync<NW>();
+  // vout[v][r] = sum_k M[r][k] vin[v][k] in fp64 (vin: fp32 at vf or fp64 at vd), nv vectors
+  auto matvec = [&](const float* M, const float* vf, const double* vd, double* vout, int nv) {
+    for (int j = 0; j < PR; ++j) {
+      const int r = 4 * warp + (lane >> 3) + 4 * NW * j;
+      if (4 * NW * j + 4 * warp >= D) break;  // warp-uniform
+      const float4* mr = reinterpret_cast<const float4*>(M + r * D) + e;
+      float4 m[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m[k] = __ldg(mr + 8 * k);
+      for (int v = 0; v < nv; ++v) {
+        double acc = 0.0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c0 = v * D + 4 * (e + 8 * k);
+          acc = fma((double)m[k].x, vd ? vd[c0] : (double)vf[c0], acc);
+          acc = fma((double)m[k].y, vd ? vd[c0 + 1] : (double)vf[c0 + 1], acc);
+          acc = fma((double)m[k].z, vd ? vd[c0 + 2] : (double)vf[c0 + 2], acc);
+          acc = fma((double)m[k].w, vd ? vd[c0 + 3] : (double)vf[c0 + 3], acc);
+        }
+        acc += __shfl_xor_sync(FULL, acc, 1);
+        acc += __shfl_xor_sync(FULL, acc, 2);
+        acc += __shfl_xor_sync(FULL, acc, 4);
+        if (e == 0) vout[v * D + r] = acc;
+      }
+    }
+  };
+  auto sumsq = [&](const float* vf, const double* vd) -> double {  // one warp, fixed order
+    double acc = 0.0;
+    for (int k = 0; k < D / 32; ++k) {
+      const double v = vd ? vd[lane + 32 * k] : (double)vf[lane + 32 * k];
+      acc = fma(v, v, acc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+    return acc;
+  };
+  matvec(a.Pi, x, nullptr, y, 2);  // y = Pi k, Pi v
+  if (warp < 2) {
+    const double ss = sumsq(x + D * warp, nullptr);
+    if (lane == 0) nrm[warp] = sqrt(ss);
+  }
+  consumers_sync<NW>();
+  for (int i = tid; i < 2 * D; i += NW * 32) {  // coordinate i % D of the key (i < D) or the value
+    const bool isv = i >= D;
+    const int j = i % D;
+    const double n = nrm[isv ? 1 : 0];
+    const double u = n > 0.0 ? sqrt((double)D) * y[i] / n : 0.0;
+    const int bits = isv ? VB : KB;
+    const float* th = isv ? a.vt : a.kt;
+    int idx = 0;
+    for (int c = 0; c < (1 << bits) - 1; ++c) idx += u >= (double)th[c] ? 1 : 0;
+    if (!isv) y[j] = u - (double)cbs[idx];  // rho, in place of this thread's own y element
+    const int bit = bits * (isv ? v_slot_of_coord(j) : k_slot_of_coord(j));
+    uint32_t* w = row + (isv ? 20 : 0);
+    atomicOr(w + (bit >> 5), (uint32_t)idx << (bit & 31));
+    if ((bit & 31) + bits > 32) atomicOr(w + (bit >> 5) + 1, (uint32_t)idx >> (32 - (bit & 31)));
+  }
+  consumers_sync<NW>();
+  if constexpr (QJL) {
+    matvec(a.S, nullptr, y, y + D, 1);  // S rho, over the value's y (read before the barrier)
+    if (warp == 0) {
+      const double rr = sumsq(nullptr, y);
+      if (lane == 0) nrm[2] = nrm[0] * sqrt(rr) / sqrt((double)D);
+    }
+    consumers_sync<NW>();
+    for (int l = tid; l < kQjlRows; l += NW * 32) {
+      const int bit = sign_bit_of_row(l);
+      if (y[D + l] >= 0.0) atomicOr(row + 16 + (bit >> 5), 1u << (bit & 31));
+    }
+  }
+  if (tid == 0) {
+    reinterpret_cast<float*>(row)[36] = (float)nrm[0];
+    reinterpret_cast<float*>(row)[37] = QJL ? (float)nrm[2] : 0.0f;
+    reinterpret_cast<float*>(row)[38] = (float)nrm[1];
+  }
+  consumers_sync<NW>();  // the packed row is complete
+  if (hg == 0 && warp == 0) {  // one copy of the row into the cache
+    constexpr int K_ROW = 16 * KB, V_ROW = 16 * VB;
+    const int64_t r = bk * a.T_cap + L - 1;
+    if (lane < K_ROW / 4) reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.k_codes) + r * K_ROW)[lane] = row[lane];
+    if (lane < V_ROW / 4) reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.v_codes) + r * V_ROW)[lane] = row[20 + lane];
+    if (QJL && lane < 4) reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.k_signs) + r * 16)[lane] = row[16 + lane];
+    if (lane == 0) {
+      const_cast<float*>(a.k_norm)[r] = reinterpret_cast<const float*>(row)[36];
+      if (QJL) const_cast<float*>(a.k_rnorm)[r] = reinterpret_cast<const float*>(row)[37];
+      const_cast<float*>(a.v_norm)[r] = reinterpret_cast<const float*>(row)[38];
+    }
+  }
+}
+
+// STEP: the decode-step variant (a separate instantiation, so that plain decode carries none of it).
+template <int KB, int VB, bool QJL, int NB, bool MX, bool STEP>
 __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __grid_constant__ DArgs a) {
   using Lay = Layout<KB, VB, QJL, NB, MX>;
   using Lut = PairLut<KB, VB>;
@@ -513,6 +636,9 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       f += t1 - t0;
       const int bk = (int)div_s(u, a.hgroups);  // b * Hkv + kv-head
       const int64_t rowb = (int64_t)bk * a.T_cap;
+      // decode step: this segment ends its unit, whose last row is the new token, quantized by
+      // the consumers in the prologue; the producer writes it into the stage itself
+      const bool step_seg = STEP && !MX && t1 == L;
       for (int s0 = t0; s0 < t1; s0 += ST, ++it) {
         const int cur = slot, cur_round = round;  // this stage's slot, and its earlier uses
         if (++slot == ns) {
@@ -525,6 +651,38 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         const int ntok = min(ST, t1 - s0);
         const int64_t row0 = rowb + s0;
         unsigned char* st = smem + ctl.stage_off[cur];
+        if (STEP && step_seg && s0 + ntok == t1) {  // the stage with the new row (its last one)
+          const int nb = ntok - 1;          // rows copied from the cache
+          if (lane == 0 && nb > 0) {
+            if constexpr (!MX) {
+              bulk_g2s(st + Lay::OFF_KC, a.k_codes + row0 * Lay::K_ROW, nb * Lay::K_ROW, &ctl.full[cur]);
+              if constexpr (QJL) bulk_g2s(st + Lay::OFF_SG, a.k_signs + row0 * 16, nb * 16, &ctl.full[cur]);
+              bulk_g2s(st + Lay::OFF_VC, a.v_codes + row0 * Lay::V_ROW, nb * Lay::V_ROW, &ctl.full[cur]);
+            }
+          }
+          for (int i = lane; i < nb; i += 32) {
+            cp_async4(st + Lay::OFF_NK + 4 * i, a.k_norm + row0 + i, 4);
+            if constexpr (QJL) cp_async4(st + Lay::OFF_RN + 4 * i, a.k_rnorm + row0 + i, 4);
+            cp_async4(st + Lay::OFF_NV + 4 * i, a.v_norm + row0 + i, 4);
+          }
+          // wait (once) until the consumers have the packed row
+          asm volatile("bar.sync 3, %0;\n" ::"n"((NW + 1) * 32) : "memory");
+          const uint32_t* row = reinterpret_cast<const uint32_t*>(smem + ctl.prep_off + 4 * Lay::PREP_WORDS);
+          const int p = nb;
+          if (lane < Lay::K_ROW / 4) reinterpret_cast<uint32_t*>(st + Lay::OFF_KC + p * Lay::K_ROW)[lane] = row[lane];
+          if (QJL && lane < 4) reinterpret_cast<uint32_t*>(st + Lay::OFF_SG + p * 16)[lane] = row[16 + lane];
+          if (lane < Lay::V_ROW / 4) reinterpret_cast<uint32_t*>(st + Lay::OFF_VC + p * Lay::V_ROW)[lane] = row[20 + lane];
+          if (lane == 0) {
+            reinterpret_cast<float*>(st + Lay::OFF_NK)[p] = reinterpret_cast<const float*>(row)[36];
+            if (QJL) reinterpret_cast<float*>(st + Lay::OFF_RN)[p] = reinterpret_cast<const float*>(row)[37];
+            reinterpret_cast<float*>(st + Lay::OFF_NV)[p] = reinterpret_cast<const float*>(row)[38];
+          }
+          __syncwarp();  // (the lanes' stores are ordered before lane 0's release arrive)
+          if (lane == 0) mbar_expect_tx_(&ctl.full[cur], (uint32_t)(nb * Lay::TX_PER_TOKEN));
+          cp_async_arrive_noinc(&ctl.full[cur]);
+          issued = it + 1;
+          continue;
+        }
         if (lane == 0) {
           mbar_expect_tx_(&ctl.full[cur], (uint32_t)(ntok * Lay::TX_PER_TOKEN));
           if constexpr (!MX)
@@ -644,6 +802,17 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
       }
     }
   };
+  // Decode step: the new key / value of the CTA's segment that ends its unit (at most one; the
+  // host keeps the step on this path only then), quantized in fp64 exactly as the definition
+  // reads (norm, u = sqrt(d) Pi x / n, idx = #{t_i <= u}, rho = u - c[idx], ||r|| and the signs
+  // of S rho), so that no guard band is needed.  The matrix rows are the prologue's registers.
+  // Scratch of the step in the B-fragment area, which prep_frags fills only afterwards: y (fp64
+  // [2][D]: Pi k, Pi v; then rho, S rho), the new vectors (fp32 [2][D]) and the fp64 norms; the
+  // packed row stays until its stage is patched.
+  double* sty = reinterpret_cast<double*>(cbs + 64);
+  float* stx = reinterpret_cast<float*>(sty + 2 * D);
+  double* stn = reinterpret_cast<double*>(stx + 2 * D);
+  uint32_t* strow = reinterpret_cast<uint32_t*>(smem + ctl.prep_off + 4 * Lay::PREP_WORDS);  // [0,16) K codes, [16,20) signs, [20,36) V codes, [36,39) norms
   // B operands of the main loop's MMAs, built once per chunk for all consumer warps.  Column gq of
   // n-block nb = head 4 nb + gq / 2, part gq % 2 (0: fp16 hi, 1: fp16 lo); k-step kk holds
   // k = 16kk + 2t, +1 (reg 0), +8, +9 (reg 1) of lane (gq, t).  Word 2kk + r of a lane holds the q'
@@ -781,6 +950,21 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         if constexpr (QJL) s4[j][k] = __ldg(sr + 8 * k);
       }
     }
+    // decode step: the segment of this CTA that ends its unit (its last token is the new one)
+    int64_t step_bk = -1;  // b * Hkv + kv-head of that unit, -1: none
+    int step_hg = 0;
+    if constexpr (STEP && !MX) {
+      for (int64_t f = f_begin; f < f_end;) {
+        const int64_t u = div_s(f, L);
+        const int64_t t0 = f - u * L;
+        const int64_t len = (L - t0 < f_end - f) ? L - t0 : f_end - f;
+        if (t0 + len == L) {
+          step_bk = div_s(u, a.hgroups);
+          step_hg = (int)(u - step_bk * a.hgroups);
+        }
+        f += len;
+      }
+    }
     float cbv = 0.0f;
     if (tid < 16) cbv = tid < (1 << KB) ? a.kc[tid] : 0.0f;
     else if (tid < 32) cbv = tid - 16 < (1 << VB) ? a.vc[tid - 16] : 0.0f;
@@ -801,6 +985,14 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
     if constexpr (QJL) {
       prologue_pass(s4, qpm, sqm);
       consumers_sync<NW>();
+    }
+    // ---- decode step: the new row of this CTA's unit end (its scratch is the B-fragment area,
+    // which prep_frags fills only afterwards)
+    if constexpr (STEP) {
+      if (step_bk >= 0) {
+        quantize_step_row<KB, VB, QJL, NB>(a, stx, sty, stn, strow, cbs, step_bk, step_hg, L);
+        asm volatile("bar.arrive 3, %0;\n" ::"n"((NW + 1) * 32) : "memory");  // the producer may place it
+      }
     }
 
     // ---- pair tables: entry e = lo | hi << b -> half2(c[lo], c[hi]), four lane replicas per
@@ -1358,13 +1550,13 @@ size_t workspace_bytes(int B, int Hq, int g, const Plan& p) {
   return sizeof(float) * (size_t)B * Hq * (p.pmax + split_warps(g)) * PART;
 }
 
-template <int KB, int VB, bool QJL, int NB, bool MX>
+template <int KB, int VB, bool QJL, int NB, bool MX, bool STEP>
 tq_status launch_split_nb(const DArgs& a0, cudaStream_t stream) {
   DArgs a = a0;
   // dynamic shared memory usually starts right after the per-block reserved bytes
   plan_layout<KB, VB, QJL, NB, MX>((uint32_t)device_attr(cudaDevAttrReservedSharedMemoryPerBlock, 1024),
                                    a.dyn_smem, a.plan);
-  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(split_kernel<KB, VB, QJL, NB, MX, STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        a.dyn_smem);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
   // an ordinary launch: the cache it reads may come from the kernel just before (tq_quantize)
@@ -1373,7 +1565,7 @@ tq_status launch_split_nb(const DArgs& a0, cudaStream_t stream) {
   cfg.blockDim = dim3(Shape<NB>::THREADS);
   cfg.dynamicSmemBytes = a.dyn_smem;
   cfg.stream = stream;
-  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL, NB, MX>, a);
+  e = cudaLaunchKernelEx(&cfg, split_kernel<KB, VB, QJL, NB, MX, STEP>, a);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "split launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
@@ -1381,7 +1573,13 @@ tq_status launch_split_nb(const DArgs& a0, cudaStream_t stream) {
 // One n-block of four heads when a group has at most four query heads, else two (split_warps).
 template <int KB, int VB, bool QJL, bool MX = false>
 tq_status launch_split(const DArgs& a, cudaStream_t stream) {
-  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1, MX>(a, stream) : launch_split_nb<KB, VB, QJL, 2, MX>(a, stream);
+  if constexpr (!MX) {
+    if (a.step)
+      return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1, false, true>(a, stream)
+                      : launch_split_nb<KB, VB, QJL, 2, false, true>(a, stream);
+  }
+  return a.g <= 4 ? launch_split_nb<KB, VB, QJL, 1, MX, false>(a, stream)
+                  : launch_split_nb<KB, VB, QJL, 2, MX, false>(a, stream);
 }
 
 template <int KB, bool QJL>
@@ -1426,12 +1624,48 @@ extern "C" int tq_decode_device_errors(void) {
   return (int)v;
 }
 
+namespace tq {
+namespace {
+// The new token of a fused decode step: [B, Hkv, 128] key and value of kv_dtype.
+struct StepIn {
+  const void* k_new;
+  const void* v_new;
+  int kv_dtype;
+};
+
+// A decode step runs fused (the new row quantized inside the split kernel) when every CTA's range
+// holds at most NSEG_PRE segments and at most one unit end: the prologue then computes the one new
+// row the CTA needs.  Other sizes (short contexts over many units) take quantize + decode.
+bool step_fusable(const Plan& p, int64_t L) {
+  if (p.ctas <= 0 || L <= 0) return false;
+  for (int c = 0; c < p.ctas; ++c) {
+    const int64_t f0 = part_start(p.ntot, p.ctas, c), f1 = part_start(p.ntot, p.ctas, c + 1);
+    if (f1 <= f0) continue;
+    if ((f1 - 1) / L - f0 / L + 1 > NSEG_PRE || f1 / L - f0 / L > 1) return false;
+  }
+  return true;
+}
+
+tq_status decode_impl(const tq_params* params, const void* q, int q_dtype, int Hq, const tq_cache* cache,
+                      int seq_len, float scale, float* out, void* workspace, size_t ws_bytes, void* stream,
+                      const StepIn* step);
+}  // namespace
+}  // namespace tq
+
 extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, int Hq,
                                     const tq_cache* cache, int seq_len, float scale, float* out,
                                     void* workspace, size_t ws_bytes, void* stream) {
   using namespace tq;
   const NvtxRange nvtx_range("tq_decode_attn");
   clear_error();
+  return decode_impl(params, q, q_dtype, Hq, cache, seq_len, scale, out, workspace, ws_bytes, stream, nullptr);
+}
+
+namespace tq {
+namespace {
+tq_status decode_impl(const tq_params* params, const void* q, int q_dtype, int Hq, const tq_cache* cache,
+                      int seq_len, float scale, float* out, void* workspace, size_t ws_bytes, void* stream,
+                      const StepIn* step) {
   tq_status st = check_cache(cache);
   if (st != TQ_OK) return st;
   st = check_params(params, cache);
@@ -1489,6 +1723,12 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
     a.Pi = params->Pi;
     a.S = params->S;
     a.part = ws;
+    a.step = step ? 1 : 0;
+    a.kv_bf16 = step && step->kv_dtype == TQ_BF16 ? 1 : 0;
+    a.k_new = step ? step->k_new : nullptr;
+    a.v_new = step ? step->v_new : nullptr;
+    a.kt = params->k_thresholds;
+    a.vt = params->v_thresholds;
     const bool mixed = cache->layout == TQ_LAYOUT_MIXED;
     st = cache->qjl_m ? dispatch<true>(cache->k_bits, cache->v_bits, mixed, a, s)
                       : dispatch<false>(cache->k_bits, cache->v_bits, mixed, a, s);
@@ -1512,9 +1752,20 @@ extern "C" tq_status tq_decode_attn(const tq_params* params, const void* q, int 
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
+}  // namespace
+}  // namespace tq
 
 // One decode step: append the new token (tq_quantize with T_new = 1), then attend over t + 1
 // tokens.  The decode arguments are checked first so that an invalid call enqueues nothing.
+extern "C" int tq_decode_step_fused(const tq_cache* cache, int Hq, int t) {
+  using namespace tq;
+  if (!cache || cache->Hkv < 1 || Hq < 1 || Hq % cache->Hkv || t < 0 || t >= cache->T_cap) return -1;
+  return cache->layout == TQ_LAYOUT_PLAIN &&
+                 step_fusable(make_plan(cache->B, Hq, cache->Hkv, t + 1, device_sms()), (int64_t)t + 1)
+             ? 1
+             : 0;
+}
+
 extern "C" tq_status tq_decode_step(const tq_params* params, const void* k_new, const void* v_new,
                                     int kv_dtype, const void* q, int q_dtype, int Hq, const tq_cache* cache,
                                     int t, float scale, float* out, void* workspace, size_t workspace_bytes,
@@ -1535,6 +1786,17 @@ extern "C" tq_status tq_decode_step(const tq_params* params, const void* k_new, 
   const size_t need = tq_decode_workspace_size(cache->B, Hq, cache, t + 1);
   if (workspace_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  if (cache->layout == TQ_LAYOUT_PLAIN &&
+      step_fusable(make_plan(cache->B, Hq, cache->Hkv, t + 1, device_sms()), (int64_t)t + 1)) {
+    // one launch sequence: the split kernel quantizes row t itself (fp64), writes it and attends
+    if (!k_new || !v_new) return fail(TQ_ERR_INVALID_ARG, "k_new / v_new is NULL");
+    if (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16) return fail(TQ_ERR_UNSUPPORTED, "kv_dtype %d", kv_dtype);
+    const size_t es = kv_dtype == TQ_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) % es)
+      return fail(TQ_ERR_INVALID_ARG, "k_new / v_new not aligned to their element size");
+    const StepIn in{k_new, v_new, kv_dtype};
+    return decode_impl(params, q, q_dtype, Hq, cache, t + 1, scale, out, workspace, workspace_bytes, stream, &in);
+  }
   const int64_t sh = kHeadDim, sb = (int64_t)cache->Hkv * kHeadDim;
   st = tq_quantize(params, k_new, v_new, kv_dtype, sb, sh, kHeadDim, 1, t, cache, stream);
   if (st != TQ_OK) return st;

@@ -282,9 +282,11 @@ int tq_decode_device_errors(void);
 
 /*
  * One autoregressive decode step: compress the new token's K and V into cache row t of every
- * (batch, kv-head), then attend q over rows [0, t].  Enqueues tq_quantize (T_new = 1) and
- * tq_decode_attn (seq_len = t + 1) back to back on `stream`, so one CUDA graph can hold a whole
- * step (the graph is specific to t).
+ * (batch, kv-head), then attend q over rows [0, t].  Fused where tq_decode_step_fused says so:
+ * the decode kernel quantizes row t itself (fp64, so the row equals the float64 definition's
+ * except within ~1e-15 of a threshold or of 0), writes it into the cache and attends over it in
+ * the same launch; otherwise tq_quantize (T_new = 1) and tq_decode_attn (seq_len = t + 1) are
+ * enqueued back to back.  Either way one CUDA graph can hold a whole step (specific to t).
  * Source: ai-manual.ru MLX port, section "who needs this right now" (the method serves text
  * generation with autoregressive decoding); ai-news.ru overview, paragraph on the speed figures
  * (quantization is paid per token on top of attention).
@@ -299,6 +301,15 @@ int tq_decode_device_errors(void);
 tq_status tq_decode_step(const tq_params* params, const void* k_new, const void* v_new, int kv_dtype,
                          const void* q, int q_dtype, int Hq, const tq_cache* cache, int t, float scale,
                          float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Whether tq_decode_step runs fused for these sizes on the current device: 1 when the split
+ * kernel quantizes the new row itself (in fp64, exactly as the definition reads), writes it into
+ * the cache and attends over it, all in one decode launch; 0 when the call is tq_quantize followed
+ * by tq_decode_attn (the mixed layout, or short contexts over many units, where a CTA's range
+ * holds more than two segments or more than one unit end).  -1 on invalid sizes.  Host only.
+ */
+int tq_decode_step_fused(const tq_cache* cache, int Hq, int t);
 
 /*
  * tq_decode_attn_static -- decode attention that allocates nothing and takes no workspace.

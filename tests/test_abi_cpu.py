@@ -160,3 +160,19 @@ def test_debug_quantize_stall_argument_check():
     assert L.tq_debug_quantize_stall(1, 0) == tq.TQ_ERR_INVALID_ARG
     assert "wait_cycles" in tq.last_error()
     assert L.tq_debug_quantize_stall(0, 0) == tq.TQ_OK
+
+
+def test_decode_step_fused_choice():
+    """Where the decode step runs as one fused launch (host logic, the 148-SM plan without a GPU):
+    long contexts yes; many short units (a CTA's range crossing several units) and the mixed
+    layout no; invalid sizes -1."""
+    L = tq.lib()
+    long_ctx = fake_cache(B=1, Hkv=8, T_cap=32768)
+    assert L.tq_decode_step_fused(ctypes.byref(long_ctx), 32, 32767) == 1
+    assert L.tq_decode_step_fused(ctypes.byref(long_ctx), 32, 4000) == 1
+    short = fake_cache(B=8, Hkv=8, T_cap=64)
+    assert L.tq_decode_step_fused(ctypes.byref(short), 32, 10) == 0
+    mixed = fake_cache(B=1, Hkv=8, T_cap=32768, k_bits=4, v_bits=4, layout=tq.TQ_LAYOUT_MIXED)
+    assert L.tq_decode_step_fused(ctypes.byref(mixed), 32, 32767) == 0
+    assert L.tq_decode_step_fused(ctypes.byref(long_ctx), 30, 100) == -1
+    assert L.tq_decode_step_fused(ctypes.byref(long_ctx), 32, 32768) == -1

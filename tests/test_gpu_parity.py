@@ -319,13 +319,24 @@ def test_quantize_then_decode_end_to_end():
     assert rel_qjl < 1.0 and rel_mse < 1.0
 
 
-@pytest.mark.parametrize("name", ["llama3_8b_32k", "moe_1m"])
+STEP_CASES = {
+    "llama3_8b_32k": {},                                    # bf16, 4 heads per kv-head: fused
+    "moe_1m": {},                                           # bf16, 4-bit, 8 heads per kv-head: fused
+    "single_head_4k": {},                                   # fp32, 16 heads: two head groups, fused
+    "many_short_units": dict(base="llama3_8b_32k", T=40, B=4, Hkv=8, Hq=16),  # quantize + decode
+}
+
+
+@pytest.mark.parametrize("name", list(STEP_CASES))
 def test_decode_step_appends_and_attends(name):
     """Autoregressive use: the first tokens by one tq_quantize, then one tq_decode_step per new
-    token (bf16 K/V rows written at row t, then attention over rows 0..t).  Every step's output is
-    compared with the oracle's decode over the oracle's cache of the tokens so far, and the whole
-    GPU-written cache with the oracle's quantization (inputs free of exempt cases)."""
-    w = small(name)
+    token (K/V rows written at row t, then attention over rows 0..t), fused into the decode launch
+    where tq_decode_step_fused says so.  Every step's output is compared with the oracle's decode
+    over the oracle's cache of the tokens so far, and the whole GPU-written cache with the oracle's
+    quantization (inputs free of exempt cases)."""
+    over = dict(STEP_CASES[name])
+    base = over.pop("base", name)
+    w = W.CONFIGS[base].scaled(**over) if over else small(name)
     params = params_for(w)
     K, V, Kh, Vh = _clean_gpu_inputs(w)
     T0 = w.T - 5
@@ -333,6 +344,8 @@ def test_decode_step_appends_and_attends(name):
     tq.quantize(params, K[:, :, :T0], V[:, :, :T0], cache)
     q0 = W.make_queries(w)
     _, oc = oracle_cache_arrays(w, Kh, Vh)
+    fused = [tq.decode_step_fused(cache, w.Hq, t) for t in range(T0, w.T)]
+    assert all(fused) if name != "many_short_units" else not any(fused), fused
     for t in range(T0, w.T):
         q = q0 * (1.0 + 0.25 * (t - T0))
         out = tq.decode_step(params, K[:, :, t].contiguous(), V[:, :, t].contiguous(), q.cuda(), cache, t)
