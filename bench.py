@@ -37,12 +37,14 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 def source_digest(rel: str) -> str:
-    """Digest of a kernel source with comments and blank lines removed, so that a change to the
-    comments alone keeps a capture valid."""
+    """Digest of a kernel source with comments, blank lines and the debug-build blocks
+    (``#ifdef TQ_DEBUG`` ... ``#endif``, compiled out of the library that is timed) removed, so that
+    a change to those alone keeps a capture valid."""
     import hashlib
     import re
     with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
         text = f.read()
+    text = re.sub(r"^[ \t]*#ifdef TQ_DEBUG\b.*?^[ \t]*#endif[^\n]*\n", "", text, flags=re.S | re.M)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
@@ -413,6 +415,38 @@ def run_gpu(args, w):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / e_steps}
 
+    # one autoregressive step at the last row (tq_decode_step: row T-1 written again from the same
+    # K/V, then attention over all T rows), replayed from a CUDA graph like the ops above, L2 flushed
+    # before each replay; reported beside the metric, outside its timed region
+    kn, vn = K[:, :, w.T - 1].contiguous(), V[:, :, w.T - 1].contiguous()
+
+    def dstep():
+        tq.decode_step(params, kn, vn, q, cache, w.T - 1, out=out, workspace=ws)
+
+    run_s = dstep
+    if not args.no_graph:
+        with torch.cuda.stream(side):
+            dstep()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        gs = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gs):
+            dstep()
+        run_s = gs.replay
+    s_ms = []
+    for i in range(args.warmup + max(3, args.steps)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_s()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            s_ms.append(e0.elapsed_time(e1))
+    decode_step = {"ms": sorted(s_ms)[len(s_ms) // 2], "t": w.T - 1,
+                   "fused": tq.decode_step_fused(cache, w.Hq, w.T - 1),
+                   "what": "append row T-1 (quantize) + attend over T rows, one tq_decode_step call"}
+
     if world > 1:
         torch.distributed.barrier()
     if rank != 0:
@@ -452,6 +486,7 @@ def run_gpu(args, w):
         "roofline_decode": roof_d, "roofline_quantize": roof_q,
         "cpu_baseline": cb, "e2e": e2e,
         "gpu_launches": args.steps * (n_chunks + 2),
+        "decode_step": decode_step,
         "quantize_fp64_fixups": {"coords": tq.quantize_code_fixups(), "key_vectors": tq.quantize_vector_fixups(),
                                  "calls": (args.warmup + args.steps) * n_chunks},
         "clocks": clk.summary(),

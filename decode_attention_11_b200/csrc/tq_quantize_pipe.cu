@@ -1091,7 +1091,9 @@ __device__ __noinline__ void role_epi(const PArgs& a, uint32_t tmem, int n_tiles
     uint32_t kf[2][4];
     {
       const float ska = sk * alpha_k;
-#pragma unroll
+      // one copy of the chunk code (not two): the eight epilogue warps share the SM's instruction
+      // cache with four other roles, and the rolled loop measured 7% faster at 128K x 4
+#pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const uint32_t col = tb + 64 * e + 32 * cc;
         uint32_t y[32], hi[16], lo[16];
