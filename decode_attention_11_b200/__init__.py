@@ -21,7 +21,10 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
+# TQ_DEBUG=1 selects the build with the decode kernel's device-side bounds checks
+# (python -m decode_attention_11_b200.build --debug)
+LIB_PATH = os.path.join(_HERE, "libtq_b200_debug.so" if os.environ.get("TQ_DEBUG") == "1"
+                        else "libtq_b200.so")
 
 TQ_OK = 0
 TQ_ERR_INVALID_ARG = 1
@@ -74,12 +77,14 @@ _lib: Optional[ctypes.CDLL] = None
 
 
 def lib() -> ctypes.CDLL:
-    """Load libtq_b200.so (raises if it is missing: there is no other implementation)."""
+    """Load libtq_b200.so, or libtq_b200_debug.so under TQ_DEBUG=1 (raises if it is missing:
+    there is no other implementation)."""
     global _lib
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} not built; run `python -m decode_attention_11_b200.build`")
+        raise RuntimeError(f"{LIB_PATH} not built; run `python -m decode_attention_11_b200.build`"
+                           + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
     L = ctypes.CDLL(LIB_PATH)
     L.tq_status_string.restype = ctypes.c_char_p
     L.tq_status_string.argtypes = [ctypes.c_int]

@@ -205,7 +205,9 @@ struct DArgs {
   const float* vt;
 };
 
-__device__ unsigned int g_decode_error;  // bit 0: a wait timed out; bit 1: shared memory too small
+// bit 0: a wait timed out; bit 1: shared memory too small; bit 2 (TQ_DEBUG builds): a stage's rows
+// or slot out of range; bit 3 (TQ_DEBUG): a partial slot out of range
+__device__ unsigned int g_decode_error;
 
 // MX: the outlier-aware mixed layout (TQ_LAYOUT_MIXED, KB = VB = 4): rows of 56 bytes (a 4-bit
 // outlier half, then a 3-bit half) and two norms per token; the 4-bit halves use the packed pair
@@ -651,6 +653,20 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         const int ntok = min(ST, t1 - s0);
         const int64_t row0 = rowb + s0;
         unsigned char* st = smem + ctl.stage_off[cur];
+#ifdef TQ_DEBUG
+        // debug build: the stage's cache rows and its ring slot lie inside their arrays; otherwise
+        // nothing is copied, the error is recorded and every wait of the CTA gives up
+        if (ntok <= 0 || row0 < 0 || row0 + ntok > (int64_t)a.B * a.Hkv * a.T_cap ||
+            ctl.stage_off[cur] + (uint32_t)Lay::STAGE_BYTES > (uint32_t)(a.dyn_smem - CTRL_BYTES)) {
+          if (lane == 0) {
+            atomicOr(&g_decode_error, 4u);
+            atomicOr(&ctl.err, 1u);
+          }
+          // the consumers' arrival on the new-row barrier still needs its partner
+          if (STEP && step_seg && s0 + ntok == t1) asm volatile("bar.sync 3, %0;\n" ::"n"((NW + 1) * 32) : "memory");
+          continue;
+        }
+#endif
         if (STEP && step_seg && s0 + ntok == t1) {  // the stage with the new row (its last one)
           const int nb = ntok - 1;          // rows copied from the cache
           if (lane == 0 && nb > 0) {
@@ -1345,6 +1361,12 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         lq += __shfl_xor_sync(FULL, lq, 4);
         lq += __shfl_xor_sync(FULL, lq, 8);
         lq += __shfl_xor_sync(FULL, lq, 16);
+#ifdef TQ_DEBUG
+        if (hh < nh && (int64_t)b * a.Hq + h0 + hh >= (int64_t)a.B * a.Hq) {
+          if (gq == 0) atomicOr(&g_decode_error, 8u);
+          continue;
+        }
+#endif
         if (hh < nh) {
           float* dst = a.part + ((int64_t)b * a.Hq + h0 + hh) * hstride + (a.pmax + warp) * PART;
           if (gq == 0) {
@@ -1383,6 +1405,12 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         consumers_sync<NW>();
         for (int idx = tid; idx < 4 * D; idx += NW * 32) {
           const int r = idx / D, dd = idx % D;
+#ifdef TQ_DEBUG
+          if (4 * nb + r < nh && (j < 0 || j >= a.pmax || (int64_t)b * a.Hq + h0 + 4 * nb + r >= (int64_t)a.B * a.Hq)) {
+            atomicOr(&g_decode_error, 8u);
+            continue;
+          }
+#endif
           if (4 * nb + r < nh) {
             float M = -1e30f;
 #pragma unroll

@@ -275,8 +275,9 @@ tq_status tq_decode_attn(const tq_params* params, const void* q, int q_dtype, in
  * its shared-memory pipeline are bounded (about two seconds each); one that gives up records it
  * here and the call's output is not valid.
  *   bit 0: a pipeline wait timed out;  bit 1: the device's shared memory per block was too small
- *   for the pipeline.  0 = no error since the library was loaded; -1 if the device could not be
- *   queried.
+ *   for the pipeline;  bits 2 and 3 (only in the library built with -DTQ_DEBUG): a pipeline stage's
+ *   cache rows or shared-memory slot, or a partial's slot, failed its bounds check and was skipped.
+ *   0 = no error since the library was loaded; -1 if the device could not be queried.
  */
 int tq_decode_device_errors(void);
 
