@@ -1116,6 +1116,40 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
         const unsigned char* stage = smem + ctl.stage_off[slot];
         const int r0 = 16 * warp + gq, r1 = r0 + 8;  // this lane's token rows in the stage
 
+        // Value codes of the lane's four tokens (rows 2t, 2t+1, 2t+8, 2t+9 of the warp's 16), paired
+        // for the value MMAs.  With 4-bit values and one n-block they are loaded before the score
+        // MMAs, which do not depend on them, so they fill the MMA chains' latency (2% at 128K x 4);
+        // otherwise (measured slower with two n-blocks) they are loaded after the softmax.
+        constexpr bool EARLY_V = VB == 4 && NB == 1;
+        VPairs<VB> p01, p89;
+        auto load_vpairs = [&]() {
+          const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
+          uint64_t cv0, cv1, cv2, cv3;
+          if constexpr (VB == 4) {
+            // lanes with odd t read their odd row first, so that in each load the four t-lanes
+            // of a column group hit two bank groups instead of one (64-byte rows)
+            const int sw = t & 1;
+            const uint2 a0 = lds64(vbase + (2 * t + sw) * Lay::V_ROW + 8 * gq);
+            const uint2 a1 = lds64(vbase + (2 * t + 1 - sw) * Lay::V_ROW + 8 * gq);
+            const uint2 a2 = lds64(vbase + (2 * t + 8 + sw) * Lay::V_ROW + 8 * gq);
+            const uint2 a3 = lds64(vbase + (2 * t + 9 - sw) * Lay::V_ROW + 8 * gq);
+            const uint64_t x0 = (uint64_t)a0.x | ((uint64_t)a0.y << 32), x1 = (uint64_t)a1.x | ((uint64_t)a1.y << 32);
+            const uint64_t x2 = (uint64_t)a2.x | ((uint64_t)a2.y << 32), x3 = (uint64_t)a3.x | ((uint64_t)a3.y << 32);
+            cv0 = sw ? x1 : x0;
+            cv1 = sw ? x0 : x1;
+            cv2 = sw ? x3 : x2;
+            cv3 = sw ? x2 : x3;
+          } else {
+            cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
+            cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
+            cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
+            cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
+          }
+          p01.build(cv0, cv1);
+          p89.build(cv2, cv3);
+        };
+        if constexpr (!MX && EARLY_V) load_vpairs();
+
         // ---- scores for tokens r0, r1 and heads 4nb + t ----
         // two accumulators per product (even / odd k-steps) halve the dependent MMA chains
         float kacc[NB][4], qacc[NB][4], kacc2[NB][4], qacc2[NB][4];
@@ -1303,31 +1337,7 @@ __global__ void __launch_bounds__(Shape<NB>::THREADS, 1) split_kernel(const __gr
 #undef TQ_VSTEP_R
 #undef TQ_VPAIR_R
         } else {
-          const unsigned char* vbase = stage + Lay::OFF_VC + (16 * warp) * Lay::V_ROW;
-          uint64_t cv0, cv1, cv2, cv3;
-          if constexpr (VB == 4) {
-            // lanes with odd t read their odd row first, so that in each load the four t-lanes
-            // of a column group hit two bank groups instead of one (64-byte rows)
-            const int sw = t & 1;
-            const uint2 a0 = lds64(vbase + (2 * t + sw) * Lay::V_ROW + 8 * gq);
-            const uint2 a1 = lds64(vbase + (2 * t + 1 - sw) * Lay::V_ROW + 8 * gq);
-            const uint2 a2 = lds64(vbase + (2 * t + 8 + sw) * Lay::V_ROW + 8 * gq);
-            const uint2 a3 = lds64(vbase + (2 * t + 9 - sw) * Lay::V_ROW + 8 * gq);
-            const uint64_t x0 = (uint64_t)a0.x | ((uint64_t)a0.y << 32), x1 = (uint64_t)a1.x | ((uint64_t)a1.y << 32);
-            const uint64_t x2 = (uint64_t)a2.x | ((uint64_t)a2.y << 32), x3 = (uint64_t)a3.x | ((uint64_t)a3.y << 32);
-            cv0 = sw ? x1 : x0;
-            cv1 = sw ? x0 : x1;
-            cv2 = sw ? x3 : x2;
-            cv3 = sw ? x2 : x3;
-          } else {
-            cv0 = load_v_chunk<VB>(vbase + (2 * t) * Lay::V_ROW, gq);
-            cv1 = load_v_chunk<VB>(vbase + (2 * t + 1) * Lay::V_ROW, gq);
-            cv2 = load_v_chunk<VB>(vbase + (2 * t + 8) * Lay::V_ROW, gq);
-            cv3 = load_v_chunk<VB>(vbase + (2 * t + 9) * Lay::V_ROW, gq);
-          }
-          VPairs<VB> p01, p89;
-          p01.build(cv0, cv1);
-          p89.build(cv2, cv3);
+          if constexpr (!EARLY_V) load_vpairs();
 #define TQ_VSTEP(DB)                                                                          \
           {                                                                                   \
             const uint32_t A[4] = {v_pair<KB, VB, 2 * (DB)>(lut, p01), v_pair<KB, VB, 2 * (DB) + 1>(lut, p01), \
