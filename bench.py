@@ -219,7 +219,19 @@ def oracle_sample(w: W.Workload, tokens: int):
     return t1 - t0, t2 - t1, sw
 
 
-def cpu_baseline(w: W.Workload, budget_s: float = 20.0):
+def blas_threads() -> int:
+    """Threads of numpy's BLAS pool: the oracle's matrix products run on up to this many; its
+    other numpy work runs on one."""
+    try:
+        import numpy  # noqa: F401  (the pool is visible once numpy is loaded)
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except ImportError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 20.0, single_thread: bool = True):
     tokens = 2048
     qt, dt, sw = oracle_sample(w, tokens)
     # grow the sample toward the time budget
@@ -227,20 +239,32 @@ def cpu_baseline(w: W.Workload, budget_s: float = 20.0):
         tokens = min(w.T, tokens * 2)
         qt, dt, sw = oracle_sample(w, tokens)
     dec_bytes = sw.decode_bytes()
-    cores = os.cpu_count()
-    return {
-        "value": dec_bytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+    threads = blas_threads()
+    cb = {
+        "value": dec_bytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
         "sample": f"one (batch, kv-head) unit of {w.name}: {tokens} tokens, {w.group} query heads; "
-                  f"numpy float64 (BLAS threads up to {cores})",
+                  f"numpy float64, matrix products on up to {threads} BLAS threads "
+                  f"({os.cpu_count()} host CPUs)",
         "quantize_tokens_per_s": tokens / qt, "decode_s": dt, "quantize_s": qt,
     }
+    if single_thread:
+        # the same sample with the BLAS pool held to one thread
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(1):
+                qt1, dt1, _ = oracle_sample(w, tokens)
+            cb["single_thread"] = {"value": dec_bytes / dt1 / 1e9, "unit": "GB/s",
+                                   "quantize_tokens_per_s": tokens / qt1}
+        except ImportError:
+            pass
+    return cb
 
 
 def run_reference(args, w):
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    cb = cpu_baseline(w, budget_s=20.0)
+    cb = cpu_baseline(w, budget_s=20.0, single_thread=False)
     steps = []
     tokens = int(cb["sample"].split(": ")[1].split(" ")[0])
     for _ in range(args.warmup + args.steps):
