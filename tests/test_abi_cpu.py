@@ -28,6 +28,19 @@ def test_library_exports_every_declared_function():
     assert tq.version() >= 100
 
 
+def test_debug_library_exports_the_same_functions():
+    """libtq_b200_debug.so (decode bounds checks, built by build(debug=True)) loads and exports
+    every declared function too, so TQ_DEBUG=1 can stand in for the release library."""
+    from decode_attention_11_b200.build import DEBUG_LIB
+    if not os.path.exists(DEBUG_LIB):
+        pytest.skip("debug library not built (python -m decode_attention_11_b200.build --debug)")
+    L = ctypes.CDLL(DEBUG_LIB)
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    L.tq_version.restype = ctypes.c_int
+    assert L.tq_version() == tq.version()
+
+
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
 def test_codebook_matches_oracle_bit_exact(bits):
     c, t, dist = tq.build_codebook(bits)
