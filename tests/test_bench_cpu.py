@@ -35,3 +35,30 @@ def test_reference_arm_other_ranks_print_nothing():
     r = _run({"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"}, "--gpus", "2", "--steps", "1")
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_traffic_capture_digest_ignores_comments_and_debug_blocks(tmp_path):
+    """A committed ncu capture stays attached to a kernel while only its comments, blank lines or
+    #ifdef TQ_DEBUG blocks (compiled out of the timed library) change; any code change detaches it."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    base = "int f(int x) {\n  int y = x + 1;\n  return y;\n}\n"
+    variants_same = [
+        "// header\nint f(int x) {\n  int y = x + 1;  // add\n\n  return y;\n}\n",
+        "int f(int x) {\n  /* block\n     comment */\n  int y = x + 1;\n  return y;\n}\n",
+        "int f(int x) {\n  int y = x + 1;\n#ifdef TQ_DEBUG\n  if (y < 0) return -1;\n#endif\n  return y;\n}\n",
+    ]
+    variants_diff = ["int f(int x) {\n  int y = x + 2;\n  return y;\n}\n",
+                     "int f(int x) {\n  int y = x + 1;\n#ifdef OTHER\n  y = 0;\n#endif\n  return y;\n}\n"]
+
+    def digest(text, name):
+        p = tmp_path / name
+        p.write_text(text)
+        return bench.source_digest(str(p))
+
+    d0 = digest(base, "base.cu")
+    for i, v in enumerate(variants_same):
+        assert digest(v, f"same{i}.cu") == d0, i
+    for i, v in enumerate(variants_diff):
+        assert digest(v, f"diff{i}.cu") != d0, i
