@@ -321,6 +321,7 @@ def test_quantize_then_decode_end_to_end():
 
 STEP_CASES = {
     "llama3_8b_32k": {},                                    # bf16, 4 heads per kv-head: fused
+    "llama3_8b_128k_b4": {},                                # 4-bit K and V, 4 heads per kv-head: fused
     "moe_1m": {},                                           # bf16, 4-bit, 8 heads per kv-head: fused
     "single_head_4k": {},                                   # fp32, 16 heads: two head groups, fused
     "many_short_units": dict(base="llama3_8b_32k", T=40, B=4, Hkv=8, Hq=16),  # quantize + decode
