@@ -173,7 +173,7 @@ def decode_on_oracle_cache(w, seq_lens, scale=None, q_dtype=torch.float32):
 @pytest.mark.parametrize("name", list(SMALL))
 def test_decode_parity_small(name):
     w = small(name)
-    # full and ragged lengths, down to one token (7 and 129: one below and one above a warp's 16)
+    # full and ragged lengths down to one token (7: under one warp's 16 tokens; 129: one past 128)
     for got, ref in decode_on_oracle_cache(w, [w.T, w.T - 37, 129, 65, 16, 7, 1]):
         assert_attention_close(got, ref)
 
